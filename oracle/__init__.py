@@ -1,0 +1,177 @@
+"""CPU oracle for the BitLinear W1.58·A8 matmul (ctypes + numpy over plain C).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, the smoke check in
+``__graft_entry__`` and the benchmark's CPU-baseline / reference arm may import
+this package.  It shares no code with the CUDA library and never imports it.
+
+Pinned functions (the pins live in ``tests/test_oracle_pins.py``):
+``absmean``, ``ternarize``, ``pack``, ``quantize_act``, ``ternary_matmul``,
+``dequant``, ``forward``.  No function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bitlinear_oracle.c")
+_HDR = os.path.join(_HERE, "bitlinear_oracle.h")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F32, BF16 = 0, 1
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no GPU involved); returns the library path."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    p, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    lib.orc_abs_exponent_bins.argtypes = [p, i32, i64, p]
+    lib.orc_ternarize.argtypes = [p, i32, i64, f32, p]
+    lib.orc_packed_row_bytes.argtypes = [i64]
+    lib.orc_packed_row_bytes.restype = i64
+    lib.orc_pack.argtypes = [p, i64, i64, p]
+    lib.orc_pack.restype = None
+    lib.orc_quantize_act.argtypes = [p, i32, i64, i64, p, p]
+    lib.orc_ternary_matmul.argtypes = [p, p, i64, i64, i64, p, i32]
+    lib.orc_dequant.argtypes = [p, p, f32, p, i64, i64, p]
+    lib.orc_dequant.restype = None
+    lib.orc_forward.argtypes = [p, i32, i64, i64, p, f32, p, i64, p, p, p, p, i32]
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = configure(ctypes.CDLL(build()))
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def _as_input(a: np.ndarray):
+    """float32 array, or bfloat16 given as its uint16 bit pattern."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.uint16:
+        return a, BF16
+    raise TypeError(f"oracle inputs are float32 or bf16 bits (uint16), got {a.dtype}")
+
+
+def packed_row_bytes(K: int) -> int:
+    return int(_load().orc_packed_row_bytes(K))
+
+
+def absmean(W: np.ndarray) -> np.float32:
+    """α = mean(|W|) of the whole tensor ([BitNet 三值权重实战] §2.3).
+
+    The sum of |W| is exact (integer bins per binary32 exponent); the mean is
+    rounded once to binary64 (Python's int/int true division is correctly
+    rounded) and then to binary32: α = RN32(RN64(Σ|W| / count)).
+    """
+    W, dt = _as_input(W)
+    if W.size == 0:
+        raise ValueError("empty weight tensor")
+    bins = np.zeros(256, dtype=np.int64)
+    if _load().orc_abs_exponent_bins(_ptr(W), dt, W.size, _ptr(bins)) != 0:
+        raise ValueError("non-finite weight")
+    # |w| = sig * 2^(max(E,1) - 150), so 2^149 * Σ|w| = Σ bins[E] << (max(E,1) - 1)
+    scaled = sum(int(b) << (max(e, 1) - 1) for e, b in enumerate(bins.tolist()) if b)
+    return np.float32(scaled / (W.size << 149))
+
+
+def ternarize(W: np.ndarray, alpha) -> np.ndarray:
+    """Codes ŵ = clip(round(W/α), -1, 1) as int8, same shape as W (§2.3, §4.1)."""
+    W, dt = _as_input(W)
+    out = np.empty(W.shape, dtype=np.int8)
+    _load().orc_ternarize(_ptr(W), dt, W.size, ctypes.c_float(float(np.float32(alpha))), _ptr(out))
+    return out
+
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    """2-bit packed rows [N][16·ceil(K/64)] uint8 of int8 codes [N][K]."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    N, K = codes.shape
+    out = np.empty((N, packed_row_bytes(K)), dtype=np.uint8)
+    _load().orc_pack(_ptr(codes), N, K, _ptr(out))
+    return out
+
+
+def quantize_weights(W: np.ndarray):
+    """(packed, α, codes) for a weight matrix [N][K]."""
+    alpha = absmean(W)
+    codes = ternarize(W, alpha)
+    return pack(codes), alpha, codes
+
+
+def quantize_act(x: np.ndarray):
+    """(x̃ int8 [M][K], β float32 [M]) per token (§2.4, §4.1)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    xq = np.empty((M, K), dtype=np.int8)
+    beta = np.empty(M, dtype=np.float32)
+    _load().orc_quantize_act(_ptr(x), dt, M, K, _ptr(xq), _ptr(beta))
+    return xq, beta
+
+
+def ternary_matmul(xq: np.ndarray, codes: np.ndarray, threads: int = 1) -> np.ndarray:
+    """int32 acc[M][N] = x̃·Ŵᵀ by add / subtract / skip ([1.58 位大模型] §3.3)."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    M, K = xq.shape
+    N = codes.shape[0]
+    assert codes.shape[1] == K
+    acc = np.empty((M, N), dtype=np.int32)
+    if _load().orc_ternary_matmul(_ptr(xq), _ptr(codes), M, N, K, _ptr(acc), threads) != 0:
+        raise OverflowError("accumulator outside int32")
+    return acc
+
+
+def dequant(acc: np.ndarray, beta: np.ndarray, alpha, bias: np.ndarray | None = None) -> np.ndarray:
+    """y = fp32(acc)·fp32(α·β/127) (+ bias) (§2.4–§2.5, §4.2)."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    beta = np.ascontiguousarray(beta, dtype=np.float32)
+    M, N = acc.shape
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((M, N), dtype=np.float32)
+    _load().orc_dequant(_ptr(acc), _ptr(beta), ctypes.c_float(float(np.float32(alpha))), _ptr(bias), M, N, _ptr(y))
+    return y
+
+
+def forward(x: np.ndarray, codes: np.ndarray, alpha, bias: np.ndarray | None = None, threads: int = 1):
+    """Inference forward on cached codes: returns (x̃, β, acc, y)."""
+    x, dt = _as_input(x)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    M, K = x.shape
+    N = codes.shape[0]
+    xq = np.empty((M, K), dtype=np.int8)
+    beta = np.empty(M, dtype=np.float32)
+    acc = np.empty((M, N), dtype=np.int32)
+    y = np.empty((M, N), dtype=np.float32)
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+    rc = _load().orc_forward(_ptr(x), dt, M, K, _ptr(codes), ctypes.c_float(float(np.float32(alpha))),
+                             _ptr(bias), N, _ptr(xq), _ptr(beta), _ptr(acc), _ptr(y), threads)
+    if rc != 0:
+        raise OverflowError("accumulator outside int32")
+    return xq, beta, acc, y
