@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the BitLinear W1.58·A8 decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Workload (default): one 7B-shaped decoder layer set at M = 1 token — q, k, v, o
+(4096→4096), gate, up (4096→11008), down (11008→4096) — each with its own
+bfloat16 input (0.1% ×20 outlier channels) and W ~ N(0, 0.02) weights that are
+absmean-ternarised once (not timed).  One step = the whole path over that set:
+per-token int8 activation quantisation of the seven inputs (one grouped
+launch) and the ternary GEMV + dequant of the seven matrices (one grouped
+launch).  The metric is algorithmic HBM bytes per step ÷ time per step.
+
+Timing: W warm-up steps, then exactly K steps captured in one CUDA graph and
+replayed between a barrier + synchronize on both sides, timed with CUDA events
+on the replay stream; the GEMV launches carry their own events inside the
+graph.  Weight copies rotate across steps so every step reads its weights from
+HBM (the replicas together exceed 4× the L2).  Multi-GPU: one process per GPU,
+each runs its own replica of the workload (weak scaling, no data-path
+collective); the step time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the method written out in plain C)
+on the host cores over a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+import hashlib
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary GEMV HBM GB/s (% of 8 TB/s); prefill int8 TOPS (% of peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------------------- workload
+def workload_specs():
+    from bitlinear_w1_a8_03_b200 import workloads
+    return workloads.decode_7b_layer_set(M=1)
+
+
+def bytes_per_step(specs) -> int:
+    """Algorithmic HBM bytes of one step: the packed weights once, plus the
+    activation quantisation (x bf16 in, x̃ + β out) and the GEMV's x̃ + β in and
+    fp32 y out, for every matrix."""
+    total = 0
+    for s in specs:
+        rb = 16 * ((s.K + 63) // 64)
+        total += s.N * rb                      # packed ternary weights
+        total += s.M * s.K * 2 + s.M * s.K + 4 * s.M   # act quant: x in, x̃ out, β out
+        total += s.M * s.K + 4 * s.M + 4 * s.M * s.N   # GEMV: x̃, β in; y out
+    return total
+
+
+def gemv_bytes_per_launch(specs) -> int:
+    """Algorithmic bytes of one grouped GEMV launch (weights + x̃ + β + y)."""
+    return sum(s.N * 16 * ((s.K + 63) // 64) + s.M * s.K + 4 * s.M + 4 * s.M * s.N for s in specs)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def recorded_traffic(kernel_tag: str, source: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/, valid
+    only while the kernel source is unchanged (sha256 recorded beside it)."""
+    src = os.path.join(ROOT, "bitlinear_w1_a8_03_b200", "csrc", source)
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    pat = re.compile(rf"^traffic\[{re.escape(kernel_tag)}\]:\s*(\d+)\s+bytes/launch\s+source_sha256:\s*([0-9a-f]+)", re.M)
+    for name in sorted(os.listdir(pdir)):
+        if not name.endswith((".md", ".txt")):
+            continue
+        for m in pat.finditer(open(os.path.join(pdir, name), encoding="utf-8").read()):
+            if m.group(2) == sha:
+                return int(m.group(1))
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sms, maxes, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                maxes.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# ----------------------------------------------------------------------------- native arm
+def run_native(args, rank, world, local_rank):
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    specs = workload_specs()
+
+    # weights: generate, quantise once on the device (cached, not timed)
+    packed0, alphas = [], []
+    for s in specs:
+        W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+        p, a = bl.bitlinear_quantize_weights(W)
+        packed0.append(p)
+        alphas.append(a)
+        del W
+    torch.cuda.synchronize()
+    set_bytes = sum(p.numel() for p in packed0)
+    replicas = max(2, math.ceil(4 * props.L2_cache_size / set_bytes) + 1)
+    packed = [packed0] + [[p.clone() for p in packed0] for _ in range(replicas - 1)]
+
+    # inputs (bf16, M = 1) in one buffer so the end-to-end leg copies them at once
+    x_host = np.concatenate([synth.f32_to_bf16_bits(synth.activations(s.x_seed, s.M, s.K, outliers=s.outliers)).ravel()
+                             for s in specs])
+    x_dev = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
+    xs, xq, beta, ys = [], [], [], []
+    y_dev = torch.empty(sum(s.M * s.N for s in specs), dtype=torch.float32, device=dev)
+    ox = oy = 0
+    for s in specs:
+        xs.append(x_dev[ox:ox + s.M * s.K].view(s.M, s.K))
+        xq.append(torch.empty((s.M, s.K), dtype=torch.int8, device=dev))
+        beta.append(torch.empty(s.M, dtype=torch.float32, device=dev))
+        ys.append(y_dev[oy:oy + s.M * s.N].view(s.M, s.N))
+        ox += s.M * s.K
+        oy += s.M * s.N
+    act_arr = (bl.ActProblem * len(specs))()
+    for i, s in enumerate(specs):
+        act_arr[i] = bl.ActProblem(xs[i].data_ptr(), xq[i].data_ptr(), beta[i].data_ptr(), s.M, s.K)
+    fwd_arrs = [bl.make_forward_problems([dict(x_q=xq[i], beta=beta[i], W_packed=packed[r][i], alpha=alphas[i],
+                                               N=s.N, y=ys[i]) for i, s in enumerate(specs)])
+                for r in range(replicas)]
+    L = bl.lib()
+    nprob = len(specs)
+
+    def step(i, stream_handle, ev=None):
+        bl.check(L.bitlinear_quantize_act_grouped(act_arr, nprob, bl.BL_BF16, stream_handle), "act")
+        if ev is not None:
+            ev[0].record()
+        bl.check(L.bitlinear_forward_grouped(fwd_arrs[i % replicas], nprob, stream_handle), "forward")
+        if ev is not None:
+            ev[1].record()
+
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):  # first calls also initialise the library's caches
+            step(i, sh)
+    stream.synchronize()
+
+    K = args.steps
+    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    kev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(K)]
+    with torch.cuda.graph(g_warm, stream=stream):
+        for i in range(replicas):
+            step(i, sh)
+    with torch.cuda.graph(g_timed, stream=stream):
+        for i in range(K):
+            step(i, sh, kev[i])
+
+    # warm-up: W steps in the graph form, then ≈1 s of identical replays while the clock sampler runs
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, math.ceil(args.warmup / replicas))):
+            g_warm.replay()
+    stream.synchronize()
+    gpu_id = "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local_rank)
+    sampler = ClockSampler(gpu_id)
+    t_end = time.time() + 1.0
+    with torch.cuda.stream(stream):
+        while time.time() < t_end:
+            g_warm.replay()
+            stream.synchronize()
+
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g_timed.replay()
+        t1.record()
+    t1.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    # a little more identical load for the clock window, then stop sampling
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_warm.replay()
+    stream.synchronize()
+    clocks = sampler.stop()
+
+    # end to end through the public binding: pinned host inputs in, results out, every step
+    x_pinned = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pinned = torch.empty(y_dev.numel(), dtype=torch.float32).pin_memory()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            x_dev.copy_(x_pinned, non_blocking=True)
+            bl.bitlinear_quantize_act_grouped(xs, list(zip(xq, beta)))
+            bl.bitlinear_forward_grouped(fwd_arrs[i % replicas])
+            y_pinned.copy_(y_dev, non_blocking=True)
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record()
+        for i in range(K):
+            x_dev.copy_(x_pinned, non_blocking=True)
+            bl.bitlinear_quantize_act_grouped(xs, list(zip(xq, beta)))
+            bl.bitlinear_forward_grouped(fwd_arrs[i % replicas])
+            y_pinned.copy_(y_dev, non_blocking=True)
+        e1.record()
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms, max(kernel_ms)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+
+    bps = bytes_per_step(specs)
+    value = world * bps * K / (elapsed_ms * 1e-3) / 1e9
+    e2e_value = world * bps * K / (e2e_ms * 1e-3) / 1e9
+    gbytes = gemv_bytes_per_launch(specs)
+    kavg = statistics.mean(kernel_ms)
+    achieved = gbytes / (kavg * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    traffic = recorded_traffic("gemv_ternary_kernel<1,8>:decode7b", "gemv_ternary.cu")
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / K, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8 x ternary(2-bit) -> int32, fp32 dequant",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; W ~ N(0,0.02) ternarised once, x bf16 ~ N(0,1) + 0.1% x20 outliers)",
+        "config": {
+            "workload": "7B decode layer set, M=1: q,k,v,o 4096->4096; gate,up 4096->11008; down 11008->4096",
+            "bytes_per_step": bps,
+            "weight_bytes_per_step": set_bytes,
+            "l2": f"inputs larger than L2: {replicas} rotating weight replicas, {replicas * set_bytes / 1e6:.0f} MB "
+                  f"(L2 {props.L2_cache_size / 1e6:.0f} MB)",
+            "launch": "K steps captured in one CUDA graph; per step 1 grouped act-quant + 1 grouped GEMV launch",
+            "parallelism": f"replicas x{world}",
+            "pct_of_8TBps": round(100 * value / world / 8000.0, 2),
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "gemv_ternary_kernel<MT=1,R=8> (grouped, 7 matrices)",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json copy bandwidth)" if peak_src == "measured"
+                           else "fallback 6650 GB/s",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "bytes_per_launch": gbytes,
+            "avg_launch_us": round(kavg * 1e3, 3),
+        },
+        "e2e": {
+            "value": round(e2e_value, 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": int(x_host.nbytes),
+            "d2h_bytes_per_step": int(y_dev.numel() * 4),
+            "how": "public binding per step: pinned x -> device, grouped act-quant, grouped GEMV, y -> pinned host",
+        },
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    return result
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_full():
+    """Oracle inputs for the same workload: α and codes from the oracle's own
+    weight quantisation of the full matrices (not timed)."""
+    import oracle
+    from bitlinear_w1_a8_03_b200 import synth
+    items = []
+    for s in workload_specs():
+        W = synth.weights(s.seed, s.N, s.K, s.w_std)
+        alpha = oracle.absmean(W)
+        codes = oracle.ternarize(W, alpha)
+        del W
+        x = synth.f32_to_bf16_bits(synth.activations(s.x_seed, s.M, s.K, outliers=s.outliers))
+        items.append((s, x, codes, alpha))
+    return items
+
+
+def oracle_sample(full, rows_frac: float):
+    """The first round(N·rows_frac) output rows of every matrix (full K)."""
+    out = []
+    for s, x, codes, alpha in full:
+        n = max(1, int(round(s.N * rows_frac)))
+        out.append((s, x, np.ascontiguousarray(codes[:n]), alpha, n))
+    return out
+
+
+def oracle_bytes(items) -> int:
+    total = 0
+    for s, x, codes, alpha, n in items:
+        rb = 16 * ((s.K + 63) // 64)
+        total += n * rb + s.M * s.K * 3 + 4 * s.M + s.M * s.K + 4 * s.M + 4 * s.M * n
+    return total
+
+
+def time_oracle(items, threads: int, steps: int, budget_s: float):
+    import oracle
+    done, t_total = 0, 0.0
+    while done < steps:
+        t = time.perf_counter()
+        for s, x, codes, alpha, n in items:
+            oracle.forward(x, codes, alpha, threads=threads)
+        t_total += time.perf_counter() - t
+        done += 1
+        if t_total >= budget_s:
+            break
+    return done, t_total
+
+
+def sized_sample(full, threads: int, step_seconds: float):
+    """Row fraction whose oracle step takes about ``step_seconds`` here."""
+    probe = oracle_sample(full, 0.02)
+    _, tp = time_oracle(probe, threads, 1, 0.0)
+    frac = min(1.0, max(1e-4, 0.02 * step_seconds / max(tp, 1e-4)))
+    return frac, oracle_sample(full, frac)
+
+
+def cpu_baseline(args):
+    threads = os.cpu_count() or 1
+    full = oracle_full()
+    frac, items = sized_sample(full, threads, 1.0)
+    steps, secs = time_oracle(items, threads, 1000, 12.0)
+    gbs = oracle_bytes(items) * steps / secs / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {frac:.4f} of the output rows of each of the 7 matrices (full K), {steps} whole steps "
+                      f"in {secs:.1f} s; act quant + add/sub/skip product + dequant, OpenMP over output elements"}
+
+
+def run_reference(args):
+    threads = os.cpu_count() or 1
+    total_steps = args.steps + args.warmup
+    budget = 150.0  # seconds for the whole timed + warm-up run
+    full = oracle_full()
+    frac, items = sized_sample(full, threads, budget / max(total_steps, 1))
+    for _ in range(args.warmup):
+        time_oracle(items, threads, 1, 0.0)
+    steps, secs = time_oracle(items, threads, args.steps, float("inf"))
+    value = oracle_bytes(items) * steps / secs / 1e9
+    sample = (f"first {frac:.5f} of the output rows of each of the 7 matrices (full K) per step; "
+              "act quant + add/sub/skip product + dequant, OpenMP over output elements")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": 1,
+        "steps": steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8 x ternary -> int64 (checked into int32), fp32 dequant",
+        "data": "synthetic (same seeds as the native arm)",
+        "config": {"workload": "7B decode layer set, M=1: q,k,v,o 4096->4096; gate,up 4096->11008; down 11008->4096",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    result = run_native(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1:
+            result["cpu_baseline"] = cpu_baseline(args)
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

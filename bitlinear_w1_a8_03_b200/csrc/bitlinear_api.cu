@@ -1,0 +1,170 @@
+// C ABI of libbitlinear.so (declared in include/bitlinear.h).
+//
+// Every entry point validates its arguments on the host first and returns an
+// error before touching the device, then checks that the current device is
+// compute capability 10.0, then enqueues kernels on the caller's stream.
+#include <mutex>
+
+#include "bl_launch.h"
+
+namespace bl {
+
+cudaError_t device_info(DeviceInfo* out) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!have[dev]) {
+        DeviceInfo d;
+        err = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (err == cudaSuccess) err = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (err == cudaSuccess) err = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+        cache[dev] = d;
+        have[dev] = true;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
+}  // namespace bl
+
+namespace {
+
+constexpr int64_t kMaxRows = (int64_t)1 << 31;
+constexpr int64_t kMaxWeights = (int64_t)1 << 40;
+
+bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+bitlinear_status check_device() {
+    bl::DeviceInfo d;
+    cudaError_t err = bl::device_info(&d);
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return BL_ERR_CUDA;
+    }
+    if (d.major != 10 || d.minor != 0) return BL_ERR_ARCH;
+    return BL_OK;
+}
+
+bitlinear_status from_cuda(cudaError_t err) {
+    if (err == cudaSuccess) return BL_OK;
+    cudaGetLastError();
+    return BL_ERR_CUDA;
+}
+
+bitlinear_status check_act(const bitlinear_act_problem& p) {
+    if (!p.x || !p.x_q || !p.beta) return BL_ERR_NULL;
+    if (p.M < 1 || p.K < 1 || p.K > BITLINEAR_MAX_K || p.M > kMaxRows) return BL_ERR_SHAPE;
+    if (misaligned(p.beta, 4)) return BL_ERR_ALIGN;
+    return BL_OK;
+}
+
+bitlinear_status check_forward(const bitlinear_forward_problem& p) {
+    if (!p.x_q || !p.beta || !p.W_packed || !p.alpha || !p.y) return BL_ERR_NULL;
+    if (p.M < 1 || p.N < 1 || p.K < 1 || p.K > BITLINEAR_MAX_K || p.M > kMaxRows || p.N > kMaxRows)
+        return BL_ERR_SHAPE;
+    if (misaligned(p.W_packed, 16) || misaligned(p.beta, 4) || misaligned(p.alpha, 4) || misaligned(p.y, 4) ||
+        misaligned(p.bias, 4) || misaligned(p.acc_out, 4))
+        return BL_ERR_ALIGN;
+    return BL_OK;
+}
+
+bool valid_dtype(bitlinear_dtype d) { return d == BL_F32 || d == BL_BF16; }
+
+}  // namespace
+
+extern "C" {
+
+size_t bitlinear_packed_row_bytes(int64_t K) {
+    if (K < 1) return 0;
+    return (size_t)(16 * ((K + 63) / 64));
+}
+
+size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K) {
+    if (N < 1 || K < 1) return 0;
+    return bl::quantize_weights_workspace_bytes(N, K);
+}
+
+bitlinear_status bitlinear_quantize_weights(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
+                                            uint8_t* W_packed, float* alpha, void* workspace,
+                                            size_t workspace_bytes, bitlinear_stream_t stream) {
+    if (!W || !W_packed || !alpha) return BL_ERR_NULL;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (N < 1 || K < 1 || K > BITLINEAR_MAX_K || N > kMaxWeights / K) return BL_ERR_SHAPE;
+    if (misaligned(W_packed, 16) || misaligned(alpha, 4) || misaligned(W, dtype == BL_F32 ? 4 : 2))
+        return BL_ERR_ALIGN;
+    if (!workspace || workspace_bytes < bl::quantize_weights_workspace_bytes(N, K)) return BL_ERR_WORKSPACE;
+    if (misaligned(workspace, 8)) return BL_ERR_ALIGN;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_quantize_weights(W, dtype, N, K, W_packed, alpha, workspace,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bitlinear_status bitlinear_quantize_act(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K, int8_t* x_q,
+                                        float* beta, bitlinear_stream_t stream) {
+    bitlinear_act_problem p{x, x_q, beta, M, K};
+    return bitlinear_quantize_act_grouped(&p, 1, dtype, stream);
+}
+
+bitlinear_status bitlinear_quantize_act_grouped(const bitlinear_act_problem* problems, int count,
+                                                bitlinear_dtype dtype, bitlinear_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) {
+        bitlinear_status st = check_act(problems[i]);
+        if (st != BL_OK) return st;
+        if (misaligned(problems[i].x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+        rows += problems[i].M;
+    }
+    if (rows >= kMaxRows) return BL_ERR_SHAPE;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_quantize_act(problems, count, dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bitlinear_status bitlinear_forward(const int8_t* x_q, const float* beta, int64_t M, int64_t K,
+                                   const uint8_t* W_packed, const float* alpha, int64_t N, const float* bias,
+                                   float* y, int32_t* acc_out, bitlinear_stream_t stream) {
+    bitlinear_forward_problem p{x_q, beta, W_packed, alpha, bias, y, acc_out, M, N, K};
+    return bitlinear_forward_grouped(&p, 1, stream);
+}
+
+bitlinear_status bitlinear_forward_grouped(const bitlinear_forward_problem* problems, int count,
+                                           bitlinear_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
+    for (int i = 0; i < count; ++i) {
+        bitlinear_status st = check_forward(problems[i]);
+        if (st != BL_OK) return st;
+    }
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_forward(problems, count, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char* bitlinear_status_string(bitlinear_status status) {
+    switch (status) {
+        case BL_OK: return "ok";
+        case BL_ERR_NULL: return "a required pointer is NULL";
+        case BL_ERR_SHAPE: return "a size is out of range";
+        case BL_ERR_ALIGN: return "a pointer is not aligned as required";
+        case BL_ERR_DTYPE: return "unknown dtype";
+        case BL_ERR_WORKSPACE: return "workspace missing or too small";
+        case BL_ERR_ARCH: return "device is not compute capability 10.0 (B200)";
+        case BL_ERR_CUDA: return "CUDA runtime error";
+        case BL_ERR_COUNT: return "group count out of range";
+    }
+    return "unknown status";
+}
+
+int bitlinear_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Device helpers shared by the BitLinear kernels (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bitlinear.h"
+
+namespace bl {
+
+constexpr int kMaxGroup = BITLINEAR_MAX_GROUP;
+
+// bfloat16 is the upper half of a binary32, so widening is exact.
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+template <typename T>
+__device__ __forceinline__ float load_as_f32(const T* p, int64_t i);
+template <>
+__device__ __forceinline__ float load_as_f32<float>(const float* p, int64_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float load_as_f32<uint16_t>(const uint16_t* p, int64_t i) {
+    return bf16_bits_to_f32(p[i]);
+}
+
+// d = c + Σ_i a.u8[i] · b.s8[i]  (unsigned codes times signed activations)
+__device__ __forceinline__ int dp4a_u8s8(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// d = c + Σ_i a.s8[i] · b.s8[i]
+__device__ __forceinline__ int dp4a_s8s8(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// 16-byte read of data used once: read-only path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte read of data shared by many warps (activations): read-only, L1-cached.
+__device__ __forceinline__ uint4 ld_shared_ro16(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int j) {
+    return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+}
+
+// Dequantisation scale of one token: RN32(RN64(α·β / 127)).  α and β are
+// binary32, so their product is exact in binary64.
+__device__ __forceinline__ float dequant_scale(float alpha, float beta) {
+    double s = __dmul_rn((double)alpha, (double)beta);
+    s = __ddiv_rn(s, 127.0);
+    return __double2float_rn(s);
+}
+
+}  // namespace bl

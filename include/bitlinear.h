@@ -1,0 +1,181 @@
+/*
+ * bitlinear.h — C ABI of libbitlinear.so, the BitNet b1.58 BitLinear W1.58·A8
+ * matmul for NVIDIA B200 (sm_100a).
+ *
+ * The three calls follow the pages' statement of the layer: quantise the
+ * weights once and cache them, quantise the activations on every forward,
+ * multiply in integers, then dequantise and add the bias ("1.58-bit 大模型极限
+ * 量化实战：从 BitNet 三值权重到单颗 CPU 跑起 100B 模型", chenxutan.com/d/5049.html,
+ * §3.2 and §4.2).
+ *
+ * Conventions for every call:
+ *  - Tensor pointers are DEVICE pointers owned by the caller; the library keeps
+ *    none of them after the call returns and allocates no device memory.
+ *  - Work is enqueued asynchronously on `stream` (NULL = the legacy default
+ *    stream).  Outputs are valid once the stream reaches that point.
+ *  - Every call returns a bitlinear_status and never throws or aborts.
+ *    Argument errors are found on the host before anything is launched, and
+ *    then no output is touched.  BL_ERR_CUDA reports a launch failure.
+ *  - Calls are thread-safe; calls on one stream run in order.
+ *  - Arithmetic is IEEE binary32 with round-to-nearest-even except where a
+ *    call says otherwise; the integer path is exact.  Results are bit-for-bit
+ *    reproducible for a given input, whatever the device's SM count.
+ *  - The library runs only on compute capability 10.0 (B200); elsewhere calls
+ *    return BL_ERR_ARCH.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BITLINEAR_API __attribute__((visibility("default")))
+#else
+#define BITLINEAR_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* bitlinear_stream_t;
+
+typedef enum bitlinear_status {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,      /* a required pointer is NULL */
+    BL_ERR_SHAPE = 2,     /* a size is < 1 or above its stated maximum */
+    BL_ERR_ALIGN = 3,     /* a pointer breaks its stated alignment */
+    BL_ERR_DTYPE = 4,     /* unknown bitlinear_dtype */
+    BL_ERR_WORKSPACE = 5, /* workspace NULL or smaller than required */
+    BL_ERR_ARCH = 6,      /* current device is not compute capability 10.0 */
+    BL_ERR_CUDA = 7,      /* the CUDA runtime reported an error */
+    BL_ERR_COUNT = 8      /* group count outside 1..BITLINEAR_MAX_GROUP */
+} bitlinear_status;
+
+typedef enum bitlinear_dtype {
+    BL_F32 = 0,  /* IEEE binary32 */
+    BL_BF16 = 1  /* bfloat16; widened exactly to binary32 before any arithmetic */
+} bitlinear_dtype;
+
+/* Largest K (input features) accepted; keeps every int32 accumulator exact. */
+#define BITLINEAR_MAX_K ((int64_t)1 << 20)
+/* Largest number of problems in one grouped call. */
+#define BITLINEAR_MAX_GROUP 16
+
+/* Bytes of one packed weight row: 16·ceil(K/64) (0 if K < 1).
+ *
+ * Packed weight layout ("W_packed", row-major [N][bitlinear_packed_row_bytes(K)]
+ * uint8, 16-byte aligned): 2 bits per weight with codes 00/01/10 for the
+ * ternary values -1/0/+1 (the pages' storage, chenxutan.com/d/5049.html §5.3);
+ * row n holds output feature n, contiguous along the K input features.  The
+ * row is read as little-endian 32-bit words of 16 weights each: weight
+ * k = 16g + 4s + b lives in byte b of word g, bits 2s..2s+1.  So masking a word
+ * with 0x03030303 << 2s yields the codes of weights 16g+4s .. 16g+4s+3 in the
+ * four bytes, in order.  Weights k >= K are padding with code 01 (zero); code
+ * 11 is never written and reads as zero. */
+BITLINEAR_API size_t bitlinear_packed_row_bytes(int64_t K);
+
+/* Device workspace bytes bitlinear_quantize_weights needs for an N×K matrix. */
+BITLINEAR_API size_t bitlinear_quantize_weights_workspace_bytes(int64_t N, int64_t K);
+
+/* Absmean ternary weight quantisation (chenxutan.com/d/5049.html §2.3, §4.1):
+ *   α = mean(|W|) over the whole tensor, Ŵ = clip(round(W/α), -1, 1),
+ * round = half to even, W/α one binary32 division (a NaN quotient, possible
+ * only when α underflows to 0, gives the zero weight).  The sum of |W| is
+ * exact; α = RN32(RN64(Σ|W| / (N·K))).
+ *
+ *   W          [N][K] row-major, `dtype`, aligned to its element size.
+ *   W_packed   out: [N][bitlinear_packed_row_bytes(K)] uint8, 16-byte aligned.
+ *   alpha      out: 1 float.
+ *   workspace  device scratch of at least
+ *              bitlinear_quantize_weights_workspace_bytes(N, K) bytes, 8-byte
+ *              aligned; its contents are undefined afterwards.
+ * Errors: BL_ERR_NULL, BL_ERR_SHAPE (N < 1, K < 1, K > BITLINEAR_MAX_K,
+ * N·K > 2^40), BL_ERR_ALIGN, BL_ERR_DTYPE, BL_ERR_WORKSPACE, BL_ERR_ARCH,
+ * BL_ERR_CUDA.  Non-finite weights give an undefined α. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_weights(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
+                                            uint8_t* W_packed, float* alpha, void* workspace,
+                                            size_t workspace_bytes, bitlinear_stream_t stream);
+
+/* Per-token absmax int8 activation quantisation (chenxutan.com/d/5049.html
+ * §2.4, §4.1; per token as in nxmr.cn/news/148658 §3.2), for each row m:
+ *   β_m = max_k |x[m][k]| + 1e-8   (binary32 add)
+ *   x̃[m][k] = clip(round((x[m][k]·127) / β_m), -127, 127)
+ * with the product and the quotient each rounded to binary32, half to even.
+ *
+ *   x     [M][K] row-major, `dtype`, aligned to its element size.
+ *   x_q   out: [M][K] int8 row-major (row stride K).
+ *   beta  out: [M] float.
+ * Errors: BL_ERR_NULL, BL_ERR_SHAPE (M < 1, K < 1, K > BITLINEAR_MAX_K,
+ * M > 2^31), BL_ERR_ALIGN, BL_ERR_DTYPE, BL_ERR_ARCH, BL_ERR_CUDA.  Non-finite
+ * inputs give undefined results. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_act(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K,
+                                        int8_t* x_q, float* beta, bitlinear_stream_t stream);
+
+/* Ternary product and dequantisation (chenxutan.com/d/5049.html §2.4–§2.5,
+ * §4.2; add / subtract / skip as in nxmr.cn/news/148658 §3.3):
+ *   acc[m][n] = Σ_k x̃[m][k]·Ŵ[n][k]                       (exact int32)
+ *   s_m       = RN32( RN64( (double)α·(double)β_m / 127 ) )
+ *   y[m][n]   = RN32( fp32(acc[m][n])·s_m )  (+ bias[n], binary32 add)
+ *
+ *   x_q, beta  from bitlinear_quantize_act ([M][K] int8, [M] float).
+ *   W_packed, alpha  from bitlinear_quantize_weights for an N×K matrix;
+ *              W_packed 16-byte aligned.
+ *   bias       optional [N] float (NULL = no bias).
+ *   y          out: [M][N] float row-major.
+ *   acc_out    optional out: [M][N] int32 accumulators (NULL = not written).
+ * Kernel choice is by shape only and never changes a result.
+ * Errors: BL_ERR_NULL, BL_ERR_SHAPE (M, N, K < 1, K > BITLINEAR_MAX_K,
+ * M or N > 2^31), BL_ERR_ALIGN, BL_ERR_ARCH, BL_ERR_CUDA. */
+BITLINEAR_API bitlinear_status bitlinear_forward(const int8_t* x_q, const float* beta, int64_t M, int64_t K,
+                                   const uint8_t* W_packed, const float* alpha, int64_t N,
+                                   const float* bias, float* y, int32_t* acc_out,
+                                   bitlinear_stream_t stream);
+
+/* One problem of a grouped activation quantisation; fields as in
+ * bitlinear_quantize_act. */
+typedef struct bitlinear_act_problem {
+    const void* x;
+    int8_t* x_q;
+    float* beta;
+    int64_t M, K;
+} bitlinear_act_problem;
+
+/* bitlinear_quantize_act on `count` independent problems of one dtype in a
+ * single launch (e.g. the several inputs of one transformer layer).
+ * `problems` is a HOST array; it may be reused as soon as the call returns.
+ * Errors: as bitlinear_quantize_act, plus BL_ERR_COUNT. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_act_grouped(const bitlinear_act_problem* problems, int count,
+                                                bitlinear_dtype dtype, bitlinear_stream_t stream);
+
+/* One problem of a grouped forward; fields as in bitlinear_forward. */
+typedef struct bitlinear_forward_problem {
+    const int8_t* x_q;
+    const float* beta;
+    const uint8_t* W_packed;
+    const float* alpha;
+    const float* bias;
+    float* y;
+    int32_t* acc_out;
+    int64_t M, N, K;
+} bitlinear_forward_problem;
+
+/* bitlinear_forward on `count` independent problems in a single launch, so
+ * that the weight streams of several small matrices overlap (e.g. the seven
+ * linears of one decoder layer).  `problems` is a HOST array.
+ * Errors: as bitlinear_forward, plus BL_ERR_COUNT. */
+BITLINEAR_API bitlinear_status bitlinear_forward_grouped(const bitlinear_forward_problem* problems, int count,
+                                           bitlinear_stream_t stream);
+
+/* Static description of a status code. */
+BITLINEAR_API const char* bitlinear_status_string(bitlinear_status status);
+
+/* ABI version: 100·major + minor. */
+BITLINEAR_API int bitlinear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITLINEAR_H */
