@@ -63,6 +63,7 @@ def lib():
             L.bitlinear_quantize_weights_workspace_bytes.argtypes = [i64, i64]
             L.bitlinear_quantize_weights_workspace_bytes.restype = sz
             L.bitlinear_quantize_weights.argtypes = [p, i32, i64, i64, p, p, p, sz, p]
+            L.bitlinear_quantize_weights_static.argtypes = [p, i32, i64, i64, p, p, p]
             L.bitlinear_quantize_act.argtypes = [p, i32, i64, i64, p, p, p]
             L.bitlinear_forward.argtypes = [p, p, i64, i64, p, p, i64, p, p, p, p]
             L.bitlinear_quantize_act_grouped.argtypes = [ctypes.POINTER(ActProblem), i32, i32, p]
@@ -70,7 +71,8 @@ def lib():
             L.bitlinear_status_string.argtypes = [i32]
             L.bitlinear_status_string.restype = ctypes.c_char_p
             L.bitlinear_version.argtypes = []
-            for name in ("bitlinear_quantize_weights", "bitlinear_quantize_act", "bitlinear_forward",
+            for name in ("bitlinear_quantize_weights", "bitlinear_quantize_weights_static",
+                         "bitlinear_quantize_act", "bitlinear_forward",
                          "bitlinear_quantize_act_grouped", "bitlinear_forward_grouped", "bitlinear_version"):
                 getattr(L, name).restype = i32
             _lib = L

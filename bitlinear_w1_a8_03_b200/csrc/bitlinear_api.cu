@@ -106,6 +106,20 @@ bitlinear_status bitlinear_quantize_weights(const void* W, bitlinear_dtype dtype
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+bitlinear_status bitlinear_quantize_weights_static(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
+                                                   uint8_t* W_packed, float* alpha, bitlinear_stream_t stream) {
+    if (!W || !W_packed || !alpha) return BL_ERR_NULL;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (N < 1 || K < 1 || K > BITLINEAR_MAX_K || N > kMaxWeights / K) return BL_ERR_SHAPE;
+    if (bl::quantize_weights_workspace_bytes(N, K) > bl::quantize_weights_static_scratch_bytes()) return BL_ERR_SHAPE;
+    if (misaligned(W_packed, 16) || misaligned(alpha, 4) || misaligned(W, dtype == BL_F32 ? 4 : 2))
+        return BL_ERR_ALIGN;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_quantize_weights_static(W, dtype, N, K, W_packed, alpha,
+                                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 bitlinear_status bitlinear_quantize_act(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K, int8_t* x_q,
                                         float* beta, bitlinear_stream_t stream) {
     bitlinear_act_problem p{x, x_q, beta, M, K};

@@ -22,6 +22,11 @@ size_t quantize_weights_workspace_bytes(int64_t N, int64_t K);
 cudaError_t launch_quantize_weights(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K, uint8_t* W_packed,
                                     float* alpha, void* workspace, cudaStream_t stream);
 
+// Allocation-free weight quantisation: scratch in a static device array.
+size_t quantize_weights_static_scratch_bytes();
+cudaError_t launch_quantize_weights_static(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
+                                           uint8_t* W_packed, float* alpha, cudaStream_t stream);
+
 cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream);
 
 }  // namespace bl

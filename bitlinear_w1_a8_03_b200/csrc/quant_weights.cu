@@ -13,6 +13,8 @@
 //
 // Three launches: per-CTA partial sums -> one-CTA finalise (writes α) ->
 // quantise + pack (reads α).  All are HBM-bound on W; the matrix is read twice.
+#include <mutex>
+
 #include "bl_common.cuh"
 #include "bl_launch.h"
 
@@ -257,6 +259,60 @@ cudaError_t launch_quantize_weights(const void* W, bitlinear_dtype dtype, int64_
             w, N, K, row_words, alpha, reinterpret_cast<uint32_t*>(W_packed));
     }
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant (bitlinear_quantize_weights_static).
+//
+// Some callers may not allocate device memory at all: a plugin running inside
+// a host application that owns the whole device-memory budget, or a
+// latency-critical loop in which cudaMalloc/cudaFree (which can synchronise
+// the device) are not allowed.  For them the partial sums of α live in this
+// fixed module-scope array instead of a caller workspace.  Its size is fixed:
+// kMaxPartials × kLimbs 64-bit words (80 KiB), which covers every accepted
+// matrix because the partial-sum grid never exceeds kMaxPartials CTAs.  Every
+// GPU that loads the library holds the array until the process exits.
+//
+// Each call overwrites the partial sums it reads (nothing has to start at
+// zero), and every call on a device shares the one array: calls that overlap
+// on the GPU (for example on two streams without ordering) race and give
+// wrong α.  In host code the array's name is only a host-side handle, so its
+// device address is looked up once per device with cudaGetSymbolAddress, on
+// that device's first call; that first call should therefore come before any
+// stream capture.
+static __device__ __align__(256) unsigned long long g_static_partials[kMaxPartials * kLimbs];
+
+namespace {
+
+cudaError_t static_partials(unsigned long long** out) {
+    static std::mutex mu;
+    static unsigned long long* addr[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_static_partials);
+        if (err != cudaSuccess) return err;
+        addr[dev] = static_cast<unsigned long long*>(p);
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t quantize_weights_static_scratch_bytes() { return sizeof(g_static_partials); }
+
+cudaError_t launch_quantize_weights_static(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
+                                           uint8_t* W_packed, float* alpha, cudaStream_t stream) {
+    if (quantize_weights_workspace_bytes(N, K) > sizeof(g_static_partials)) return cudaErrorInvalidValue;
+    unsigned long long* scratch = nullptr;
+    cudaError_t err = static_partials(&scratch);
+    if (err != cudaSuccess) return err;
+    return launch_quantize_weights(W, dtype, N, K, W_packed, alpha, scratch, stream);
 }
 
 }  // namespace bl

@@ -99,6 +99,27 @@ BITLINEAR_API bitlinear_status bitlinear_quantize_weights(const void* W, bitline
                                             uint8_t* W_packed, float* alpha, void* workspace,
                                             size_t workspace_bytes, bitlinear_stream_t stream);
 
+/* bitlinear_quantize_weights without a workspace argument, for callers that
+ * may not allocate device memory at all: a plugin running inside a host
+ * application that owns the whole device-memory budget, or a latency-critical
+ * loop in which cudaMalloc/cudaFree (which can synchronise the device) are
+ * not allowed.  The pages have no counterpart: this is a packaging variant of
+ * the same quantisation, with identical results.
+ *
+ * Its scratch (the partial sums of α) is a fixed 80 KiB array inside the
+ * library that every GPU loading the library holds until the process exits;
+ * the call allocates nothing.  Every call on a device shares that array and
+ * overwrites what it reads, so calls that overlap on the GPU (e.g. on two
+ * unordered streams) race and give wrong results; order them on one stream.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and so should come before any stream capture.
+ * Arguments, layouts and errors are those of bitlinear_quantize_weights; the
+ * maximum size is the same (N·K <= 2^40, K <= BITLINEAR_MAX_K), and larger
+ * sizes return BL_ERR_SHAPE. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_weights_static(const void* W, bitlinear_dtype dtype, int64_t N,
+                                                                 int64_t K, uint8_t* W_packed, float* alpha,
+                                                                 bitlinear_stream_t stream);
+
 /* Per-token absmax int8 activation quantisation (chenxutan.com/d/5049.html
  * §2.4, §4.1; per token as in nxmr.cn/news/148658 §3.2), for each row m:
  *   β_m = max_k |x[m][k]| + 1e-8   (binary32 add)
