@@ -23,8 +23,10 @@ MAX_K = 1 << 20
 BL_F32, BL_BF16 = 0, 1
 STATUS = {
     0: "BL_OK", 1: "BL_ERR_NULL", 2: "BL_ERR_SHAPE", 3: "BL_ERR_ALIGN", 4: "BL_ERR_DTYPE",
-    5: "BL_ERR_WORKSPACE", 6: "BL_ERR_ARCH", 7: "BL_ERR_CUDA", 8: "BL_ERR_COUNT",
+    5: "BL_ERR_WORKSPACE", 6: "BL_ERR_ARCH", 7: "BL_ERR_CUDA", 8: "BL_ERR_COUNT", 9: "BL_ERR_TIMEOUT",
+    10: "BL_ERR_FLAGS",
 }
+BL_LINEAR_WEIGHTS_STATIC = 1
 
 _lock = threading.Lock()
 _lib = None
@@ -48,6 +50,13 @@ class ForwardProblem(ctypes.Structure):
                 ("K", ctypes.c_int64)]
 
 
+class LinearProblem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("x_q", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("W_packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("acc_out", ctypes.c_void_p), ("M", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
 def lib():
     """The loaded ctypes library; raises if the CUDA library was not built."""
     global _lib
@@ -68,12 +77,18 @@ def lib():
             L.bitlinear_forward.argtypes = [p, p, i64, i64, p, p, i64, p, p, p, p]
             L.bitlinear_quantize_act_grouped.argtypes = [ctypes.POINTER(ActProblem), i32, i32, p]
             L.bitlinear_forward_grouped.argtypes = [ctypes.POINTER(ForwardProblem), i32, p]
+            L.bitlinear_linear.argtypes = [p, i32, i64, i64, p, p, i64, p, p, p, p, p, p]
+            L.bitlinear_linear_grouped.argtypes = [ctypes.POINTER(LinearProblem), i32, i32, ctypes.c_uint32, p]
+            L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+            L.bitlinear_selftest_timeout.argtypes = [ctypes.c_uint32, p]
             L.bitlinear_status_string.argtypes = [i32]
             L.bitlinear_status_string.restype = ctypes.c_char_p
             L.bitlinear_version.argtypes = []
             for name in ("bitlinear_quantize_weights", "bitlinear_quantize_weights_static",
                          "bitlinear_quantize_act", "bitlinear_forward",
-                         "bitlinear_quantize_act_grouped", "bitlinear_forward_grouped", "bitlinear_version"):
+                         "bitlinear_quantize_act_grouped", "bitlinear_forward_grouped", "bitlinear_linear",
+                         "bitlinear_linear_grouped", "bitlinear_device_error", "bitlinear_selftest_timeout",
+                         "bitlinear_version"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -186,3 +201,50 @@ def bitlinear_forward_grouped(problems, stream=None):
     """Several independent forwards in one launch (see make_forward_problems)."""
     arr = problems if isinstance(problems, ctypes.Array) else make_forward_problems(problems)
     check(lib().bitlinear_forward_grouped(arr, len(arr), _stream(stream)), "bitlinear_forward_grouped")
+
+
+def bitlinear_linear(x, W_packed, alpha, N: int, bias=None, x_q=None, beta=None, y=None, acc_out=None, stream=None):
+    """Quantise x and multiply in one call (two overlapped kernels); returns y."""
+    torch = _torch()
+    _need(x, "x")
+    M, K = x.shape
+    if x_q is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if beta is None:
+        beta = torch.empty(M, dtype=torch.float32, device=x.device)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    check(lib().bitlinear_linear(_ptr(x), _dtype_code(x), M, K, _ptr(W_packed), _ptr(alpha), N, _ptr(bias),
+                                 _ptr(x_q), _ptr(beta), _ptr(y), _ptr(acc_out), _stream(stream)), "bitlinear_linear")
+    return y
+
+
+def make_linear_problems(problems):
+    """ctypes array for bitlinear_linear_grouped from dicts with keys
+    x, x_q, beta, W_packed, alpha, N, y and optional bias, acc_out."""
+    arr = (LinearProblem * len(problems))()
+    for i, p in enumerate(problems):
+        M, K = p["x"].shape
+        arr[i] = LinearProblem(_ptr(p["x"]), _ptr(p["x_q"]), _ptr(p["beta"]), _ptr(p["W_packed"]), _ptr(p["alpha"]),
+                               _ptr(p.get("bias")), _ptr(p["y"]), _ptr(p.get("acc_out")), M, p["N"], K)
+    return arr
+
+
+def bitlinear_linear_grouped(problems, dtype_code: int | None = None, flags: int = 0, stream=None):
+    """Several independent linears in one grouped quantisation + one grouped
+    product.  flags=BL_LINEAR_WEIGHTS_STATIC: no work in flight writes the weights."""
+    if isinstance(problems, ctypes.Array):
+        arr = problems
+        assert dtype_code is not None
+    else:
+        arr = make_linear_problems(problems)
+        dtype_code = _dtype_code(problems[0]["x"]) if dtype_code is None else dtype_code
+    check(lib().bitlinear_linear_grouped(arr, len(arr), dtype_code, flags, _stream(stream)),
+          "bitlinear_linear_grouped")
+
+
+def bitlinear_device_error() -> int:
+    """Read and clear the device error word (0 = none)."""
+    code = ctypes.c_int(0)
+    check(lib().bitlinear_device_error(ctypes.byref(code)), "bitlinear_device_error")
+    return code.value

@@ -161,7 +161,55 @@ bitlinear_status bitlinear_forward_grouped(const bitlinear_forward_problem* prob
     }
     bitlinear_status st = check_device();
     if (st != BL_OK) return st;
-    return from_cuda(bl::launch_forward(problems, count, reinterpret_cast<cudaStream_t>(stream)));
+    return from_cuda(bl::launch_forward(problems, count, reinterpret_cast<cudaStream_t>(stream), false));
+}
+
+bitlinear_status bitlinear_linear(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K,
+                                  const uint8_t* W_packed, const float* alpha, int64_t N, const float* bias,
+                                  int8_t* x_q, float* beta, float* y, int32_t* acc_out, bitlinear_stream_t stream) {
+    bitlinear_linear_problem p{x, x_q, beta, W_packed, alpha, bias, y, acc_out, M, N, K};
+    return bitlinear_linear_grouped(&p, 1, dtype, 0u, stream);
+}
+
+bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* problems, int count, bitlinear_dtype dtype,
+                                          uint32_t flags, bitlinear_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (flags & ~(uint32_t)BL_LINEAR_WEIGHTS_STATIC) return BL_ERR_FLAGS;
+    bitlinear_act_problem act[BITLINEAR_MAX_GROUP];
+    bitlinear_forward_problem fwd[BITLINEAR_MAX_GROUP];
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_linear_problem& q = problems[i];
+        act[i] = bitlinear_act_problem{q.x, q.x_q, q.beta, q.M, q.K};
+        fwd[i] = bitlinear_forward_problem{q.x_q, q.beta, q.W_packed, q.alpha, q.bias, q.y, q.acc_out, q.M, q.N, q.K};
+        bitlinear_status st = check_act(act[i]);
+        if (st == BL_OK) st = check_forward(fwd[i]);
+        if (st != BL_OK) return st;
+        if (misaligned(q.x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+        rows += q.M;
+    }
+    if (rows >= kMaxRows) return BL_ERR_SHAPE;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = from_cuda(bl::launch_quantize_act(act, count, dtype, s, true, (flags & BL_LINEAR_WEIGHTS_STATIC) != 0));
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_forward(fwd, count, s, true));
+}
+
+bitlinear_status bitlinear_device_error(int* code) {
+    if (!code) return BL_ERR_NULL;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::read_device_error(code));
+}
+
+bitlinear_status bitlinear_selftest_timeout(uint32_t polls, bitlinear_stream_t stream) {
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_wait_timeout_selftest(polls, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char* bitlinear_status_string(bitlinear_status status) {
@@ -175,6 +223,8 @@ const char* bitlinear_status_string(bitlinear_status status) {
         case BL_ERR_ARCH: return "device is not compute capability 10.0 (B200)";
         case BL_ERR_CUDA: return "CUDA runtime error";
         case BL_ERR_COUNT: return "group count out of range";
+        case BL_ERR_TIMEOUT: return "a kernel's bounded wait expired";
+        case BL_ERR_FLAGS: return "unknown flag bits";
     }
     return "unknown status";
 }

@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/bitlinear.h"
+#include "bitlinear.h"
 
 namespace bl {
 

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/bitlinear.h"
+#include "bitlinear.h"
 
 namespace bl {
 
@@ -15,8 +15,12 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// pdl: launch with programmatic dependent launch (the kernel waits for its
+// predecessor before reading x); early_trigger: let the next PDL kernel start
+// before that wait (only when no work in flight writes the next kernel's
+// weights).
 cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
-                                cudaStream_t stream);
+                                cudaStream_t stream, bool pdl = false, bool early_trigger = false);
 
 size_t quantize_weights_workspace_bytes(int64_t N, int64_t K);
 cudaError_t launch_quantize_weights(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K, uint8_t* W_packed,
@@ -27,6 +31,13 @@ size_t quantize_weights_static_scratch_bytes();
 cudaError_t launch_quantize_weights_static(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
                                            uint8_t* W_packed, float* alpha, cudaStream_t stream);
 
-cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream);
+// pdl: launch with programmatic dependent launch; only valid right after the
+// library's own activation-quantisation kernel on the same stream (the weight
+// stream starts before the dependency wait).
+cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl);
+
+// Device-side error word (bounded waits that expired): read and clear.
+cudaError_t read_device_error(int* code);
+cudaError_t launch_wait_timeout_selftest(uint32_t polls, cudaStream_t stream);
 
 }  // namespace bl

@@ -1,63 +1,153 @@
 // Ternary GEMV / skinny GEMM on CUDA cores: y = (x̃·Ŵᵀ)·(α·β/127) + bias.
 //
 // The product is the pages' add / subtract / skip ("1.58 位大模型",
-// nxmr.cn/news/148658 §3.3): Y[m][n] = Σ_{W=+1} x̃ - Σ_{W=-1} x̃.  Here it is
+// nxmr.cn/news/148658 §3.3): Y[m][n] = Σ_{W=+1} x̃ - Σ_{W=-1} x̃.  It is
 // evaluated as Σ c·x̃ - Σ x̃ with the stored code c = w + 1 ∈ {0, 1, 2}: one
-// mask of a packed word yields four codes as unsigned bytes, and one dp4a
-// adds their products with four int8 activations, so a zero weight costs
-// nothing extra and ±1 weights become adds and subtracts.  Dequantisation
-// and bias follow "1.58-bit 大模型极限量化实战" (chenxutan.com/d/5049.html)
-// §2.4–§2.5 and §4.2.
+// mask of a packed word yields four codes as unsigned bytes (×4^s), and one
+// dp4a adds their products with four int8 activations, so a zero weight costs
+// nothing extra and ±1 weights become adds and subtracts.  Dequantisation and
+// bias follow "1.58-bit 大模型极限量化实战" (chenxutan.com/d/5049.html) §2.4–§2.5
+// and §4.2.
 //
-// Decode is bound by HBM bytes of the packed weights ("1.58-bit 大模型极限量化
-// 实战" §5.1–§5.2; 2kiu.com/news/4928193 §3.1, §3.3): every weight byte is read
-// once per token group, coalesced 16 bytes per lane, 512 bytes per warp.
-//
-// Work split: a warp owns R consecutive output rows and MT tokens; its lanes
-// walk the row's 16-byte chunks (64 weights) with stride 32, keep exact int32
-// partial sums, then a butterfly shuffle reduces them and R·MT lanes run the
-// epilogue.  Warps take tasks from a grid-stride loop over all problems of a
-// grouped launch, so several small matrices stream back to back.
+// Decode is bound by the HBM bytes of the packed weights ("1.58-bit 大模型极限
+// 量化实战" §5.1–§5.2; 2kiu.com/news/4928193 §3.1, §3.3), so the kernel is built
+// to keep HBM streaming while the arithmetic runs:
+//  * persistent grid, one CTA per SM; the work (row groups of 8 rows × 16-byte
+//    chunks, over every problem of a grouped launch) is cut into contiguous
+//    ranges of equal chunk count, snapped to row-group boundaries;
+//  * inside a CTA the range is split evenly over 8 warps at chunk
+//    granularity; a row group shared by several warps is summed exactly in
+//    shared memory (int32 atomics) and finished by its last contributor;
+//  * each warp streams its own segments (8 rows × up to 64 chunks) into two
+//    private shared-memory stages with 1-D bulk copies (TMA), the rows issued
+//    by eight lanes at once; a waiting warp sleeps in the mbarrier (bounded);
+//  * everything a segment needs from global memory besides its weights (the
+//    activations, α, β) is requested before the warp waits for the weights,
+//    so those latencies overlap the copy;
+//  * lanes read staged rows with conflict-free 16-byte shared loads, the
+//    activations serve all 8 rows, and a reduce-scatter of shuffles leaves
+//    each row's sum in one lane.
+// The weight stream does not depend on the previous kernel, so it starts
+// before griddepcontrol.wait (programmatic dependent launch).
 #include <mutex>
 
 #include "bl_common.cuh"
 #include "bl_launch.h"
+#include "bl_ptx.cuh"
 
 namespace bl {
+
+// Set (first error wins) by a kernel whose bounded wait expired; read and
+// cleared by bitlinear_device_error().
+static __device__ int g_device_error;
+
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+#ifndef BL_GEMV_WARPS
+#define BL_GEMV_WARPS 8
+#endif
+#ifndef BL_GEMV_STAGES
+#define BL_GEMV_STAGES 2
+#endif
+constexpr int kWarps = BL_GEMV_WARPS;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStages = BL_GEMV_STAGES;         // private stages per warp
+constexpr int kRG = 8;                          // rows per row group
+constexpr int kSegChunks = 64;                  // 16-byte chunks per row per segment
+constexpr int kIt = kSegChunks / 32;            // chunks per lane per row per segment
+constexpr int kRowStride = kSegChunks * 16;     // bytes per staged row
+constexpr int kStageBytes = kRG * kRowStride;   // 8 KiB
+constexpr int kSlots = kWarps;                  // row groups shared between warps
+constexpr int kMaxMT = 4;
 
-struct GemvProblem {
+struct SProblem {
     const int8_t* xq;
     const float* beta;
-    const uint32_t* W;  // packed rows, row_words 32-bit words each
+    const uint8_t* W;
     const float* alpha;
     const float* bias;
     float* y;
     int32_t* acc_out;
-    int64_t M, N, K;
-    int64_t row_words;
-    int64_t row_groups;
-    int64_t task_begin;
+    int32_t M, N, K;
+    int32_t row_bytes;    // 16·ceil(K/64)
+    int32_t C;            // 16-byte chunks per row
+    int32_t full_chunks;  // chunks entirely inside K (the activation tail needs guards)
+    int32_t rgn;          // row groups of kRG rows
+    int32_t tgn;          // token groups of MT tokens
+    int64_t unit_begin;   // first unit (token group, row group, chunk) of this problem
 };
 
-struct GemvParams {
-    GemvProblem p[kMaxGroup];
+struct SParams {
+    SProblem p[kMaxGroup];
     int count;
-    int64_t total_tasks;
+    int64_t total_units;
 };
 
-// The 16 activation words (64 int8) of chunk c of one token row; zero past K
-// and for tokens past M.  Full chunks need a 16-byte aligned row.
-__device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int64_t K, int64_t c, bool full, bool valid,
+struct SharedLayout {
+    alignas(128) uint8_t stage[kWarps][kStages][kStageBytes];
+    alignas(8) uint64_t full[kWarps][kStages];
+    int64_t bound[kWarps + 1];  // warp unit ranges inside the CTA
+    int slot_acc[kSlots][kRG * kMaxMT];
+    int slot_count[kSlots];
+};
+
+// Position in the unit sequence: problem, (token group, row group), chunk.
+struct Cursor {
+    int p;
+    int tgrg;
+    int c;
+    int64_t u, end;
+};
+
+__device__ __forceinline__ void cursor_seek(const SParams& P, Cursor& cur, int64_t u, int64_t end) {
+    int p = 0;
+    while (p + 1 < P.count && u >= P.p[p + 1].unit_begin) ++p;
+    const int64_t local = u - P.p[p].unit_begin;
+    cur.p = p;
+    cur.tgrg = (int)(local / P.p[p].C);
+    cur.c = (int)(local - (int64_t)cur.tgrg * P.p[p].C);
+    cur.u = u;
+    cur.end = end;
+}
+
+// Length (chunks) of the segment starting at the cursor.
+__device__ __forceinline__ int cursor_len(const SParams& P, const Cursor& cur) {
+    int64_t n = P.p[cur.p].C - cur.c;
+    if (n > kSegChunks) n = kSegChunks;
+    if (n > cur.end - cur.u) n = (int)(cur.end - cur.u);
+    return (int)n;
+}
+
+__device__ __forceinline__ void cursor_advance(const SParams& P, Cursor& cur, int n) {
+    cur.u += n;
+    cur.c += n;
+    if (cur.c == P.p[cur.p].C) {
+        cur.c = 0;
+        if (++cur.tgrg == P.p[cur.p].tgn * P.p[cur.p].rgn) {
+            cur.tgrg = 0;
+            ++cur.p;
+        }
+    }
+}
+
+// Start of the row group containing unit t, rounded to the nearer boundary.
+__device__ int64_t snap_to_row_group(const SParams& P, int64_t t) {
+    if (t >= P.total_units) return P.total_units;
+    int p = 0;
+    while (p + 1 < P.count && t >= P.p[p + 1].unit_begin) ++p;
+    const int64_t local = t - P.p[p].unit_begin;
+    int64_t g = local / P.p[p].C;
+    if (2 * (local - g * P.p[p].C) >= P.p[p].C) ++g;
+    return P.p[p].unit_begin + g * P.p[p].C;
+}
+
+__device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int K, int chunk, bool full, bool valid,
                                                uint32_t (&a)[16]) {
     if (!valid) {
 #pragma unroll
         for (int q = 0; q < 16; ++q) a[q] = 0u;
     } else if (full) {
-        const int8_t* p = xrow + 64 * c;
+        const int8_t* p = xrow + 64 * chunk;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const uint4 u = ld_shared_ro16(p + 16 * v);
@@ -72,7 +162,7 @@ __device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int64_t K, in
             uint32_t w = 0;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const int64_t k = 64 * c + 4 * q + b;
+                const int k = 64 * chunk + 4 * q + b;
                 if (k < K) w |= (uint32_t)(uint8_t)xrow[k] << (8 * b);
             }
             a[q] = w;
@@ -80,114 +170,318 @@ __device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int64_t K, in
     }
 }
 
-template <int MT, int R>
-__global__ void __launch_bounds__(kThreads) gemv_ternary_kernel(const __grid_constant__ GemvParams P) {
-    constexpr int NS = (MT == 1) ? 4 : 1;  // MT == 1: one accumulator per code field
+// Issues the bulk copies of one segment (rows of one row group, chunks
+// [c, c+n)) into a stage.  Called by the whole warp: lane 0 arms the
+// barrier, then lane r copies row r, so the rows go out in one instruction.
+__device__ __forceinline__ void issue_segment(const SProblem& pr, int rg, int c, int n, uint32_t dst, uint32_t bar,
+                                              uint64_t policy, int lane) {
+    const int row0 = rg * kRG;
+    const int rows = min(kRG, pr.N - row0);
+    const uint32_t bytes = (uint32_t)n * 16u;
+    if (lane == 0) mbar_arrive_expect_tx(bar, bytes * (uint32_t)rows);
+    __syncwarp();
+    if (lane < rows)
+        bulk_copy_g2s(dst + lane * kRowStride, pr.W + (int64_t)(row0 + lane) * pr.row_bytes + (int64_t)c * 16, bytes,
+                      bar, policy);
+}
+
+// Sums v[0..V-1] over the 32 lanes of the warp (V a power of two <= 32).
+// Returns the total of index idx in every lane; lanes whose low 5-log2(V)
+// bits are zero hold distinct indices 0..V-1.  V-1 + 5-log2(V) shuffles.
+template <int V>
+__device__ __forceinline__ int reduce_scatter(int (&v)[V], int lane, int& idx) {
+    idx = 0;
+#pragma unroll
+    for (int half = V / 2, off = 16; half >= 1; half >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const int send = upper ? v[i] : v[i + half];
+            const int keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+        if (upper) idx += half;
+    }
+    int r = v[0];
+#pragma unroll
+    for (int off = 16 / V; off >= 1; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+    return r;
+}
+
+// The token a lane finishes after reduce_scatter over kRG·MT values.
+template <int MT>
+__device__ __forceinline__ int lane_token(int lane) {
+    constexpr int V = kRG * MT;
+    int idx = 0;
+#pragma unroll
+    for (int half = V / 2, off = 16; half >= 1; half >>= 1, off >>= 1)
+        if (lane & off) idx += half;
+    return idx / kRG;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_constant__ SParams P) {
+    constexpr bool kMask = MT <= 2;  // one accumulator per code field (no shifts)
+    constexpr int NS = kMask ? 4 : 1;
+    constexpr int V = kRG * MT;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    SharedLayout& S = *reinterpret_cast<SharedLayout*>(smem_raw);
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
 
-    for (int64_t t = warp0; t < P.total_tasks; t += nwarps) {
-        int pi = 0;
-        while (pi + 1 < P.count && t >= P.p[pi + 1].task_begin) ++pi;
-        const GemvProblem& pr = P.p[pi];
-        const int64_t lt = t - pr.task_begin;
-        const int64_t tg = lt / pr.row_groups;
-        const int64_t n0 = (lt - tg * pr.row_groups) * R;
-        const int64_t m0 = tg * MT;
-        const int64_t chunks = pr.row_words >> 2;
-        const int64_t full_chunks = pr.K >> 6;
+    // the next kernel on the stream (the next step's activation quantisation)
+    // may be scheduled now; it waits for this grid before touching memory
+    griddep_launch_dependents();
 
-        int acc[R][MT][NS];
-        int sx[MT];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int m = 0; m < MT; ++m)
-#pragma unroll
-                for (int s = 0; s < NS; ++s) acc[r][m][s] = 0;
-#pragma unroll
-        for (int m = 0; m < MT; ++m) sx[m] = 0;
+    // ---- CTA and warp ranges (equal chunk counts, CTA edges on row groups)
+    const int64_t G = gridDim.x;
+    const int64_t a = snap_to_row_group(P, (P.total_units * (int64_t)blockIdx.x) / G);
+    const int64_t b = snap_to_row_group(P, (P.total_units * ((int64_t)blockIdx.x + 1)) / G);
+    if (threadIdx.x <= kWarps) S.bound[threadIdx.x] = a + ((b - a) * threadIdx.x) / kWarps;
+    for (int i = threadIdx.x; i < kSlots * kRG * kMaxMT; i += kThreads) (&S.slot_acc[0][0])[i] = 0;
+    if (threadIdx.x < kSlots) S.slot_count[threadIdx.x] = 0;
+    if (threadIdx.x < kWarps * kStages) mbar_init(smem_addr(&S.full[0][0] + threadIdx.x), 1);
+    fence_mbar_init();
+    __syncthreads();
 
-        for (int64_t c = lane; c < chunks; c += 32) {
-            uint4 w[R];
+    const int64_t wu0 = S.bound[warp], wu1 = S.bound[warp + 1];
+    const uint64_t policy = policy_evict_first();
+    const uint32_t stage0 = smem_addr(&S.stage[warp][0][0]);
+    const uint32_t bar0 = smem_addr(&S.full[warp][0]);
+
+    // ---- prologue: weights do not depend on the previous kernel
+    Cursor prod;
+    cursor_seek(P, prod, wu0, wu1);
+    int issued = 0;  // segments whose copies this warp has issued
+    for (int st = 0; st < kStages && prod.u < prod.end; ++st, ++issued) {
+        const int n = cursor_len(P, prod);
+        const SProblem& pr = P.p[prod.p];
+        issue_segment(pr, prod.tgrg % pr.rgn, prod.c, n, stage0 + st * kStageBytes, bar0 + 8 * st, policy, lane);
+        cursor_advance(P, prod, n);
+    }
+    griddep_wait();  // x̃, β (and α) may come from the preceding kernels
+
+    // ---- main loop over this warp's segments
+    Cursor cons;
+    cursor_seek(P, cons, wu0, wu1);
+    const int my_tok = lane_token<MT>(lane);
+    int acc[kRG][MT][NS];
+    int sx[MT];
+    int sx_cache[MT];
+    int cache_p = -1, cache_tg = -1;
+    int scale_p = -1, scale_tg = -1;
+    float scale = 0.0f;                   // dequant scale of this lane's output token
+    float alpha_v = 0.0f, beta_v = 0.0f;  // this lane's α and β, loaded ahead of use
+    bool sx_from_cache = false;
+    int rg_chunks = 0;  // chunks of the current row group done by this warp
 #pragma unroll
-            for (int r = 0; r < R; ++r)
-                w[r] = (n0 + r < pr.N) ? ld_stream16(pr.W + (n0 + r) * pr.row_words + 4 * c)
-                                       : make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
-            uint32_t a[MT][16];
+    for (int m = 0; m < MT; ++m) sx_cache[m] = 0;
+
+    for (int seg = 0; cons.u < cons.end; ++seg) {
+        const int st = seg % kStages;
+        const uint32_t phase = (uint32_t)((seg / kStages) & 1);
+        const SProblem& pr = P.p[cons.p];
+        const int n = cursor_len(P, cons);
+        const int tg = cons.tgrg / pr.rgn;
+        const int rg = cons.tgrg - tg * pr.rgn;
+        const int m0 = tg * MT;
+
+        if (rg_chunks == 0) {  // first segment of a row group for this warp
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                load_act_chunk(pr.xq + (m0 + m) * pr.K, pr.K, c, c < full_chunks, m0 + m < pr.M, a[m]);
+            for (int r = 0; r < kRG; ++r)
 #pragma unroll
-                for (int q = 0; q < 16; ++q) sx[m] = dp4a_s8s8(0x01010101u, a[m][q], sx[m]);
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int q = 0; q < NS; ++q) acc[r][m][q] = 0;
+            // Σx̃ over this lane's chunks: reuse the cached value when the whole
+            // row group is ours with the usual lane-to-chunk mapping.
+            const bool whole = cons.c == 0 && (cons.end - cons.u) >= pr.C;
+            sx_from_cache = whole && cache_p == cons.p && cache_tg == tg;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) sx[m] = sx_from_cache ? sx_cache[m] : 0;
+        }
+        if (scale_p != cons.p || scale_tg != tg) {  // start the α, β loads early
+            const int tok = m0 + my_tok;
+            alpha_v = *pr.alpha;
+            beta_v = tok < pr.M ? pr.beta[tok] : 0.0f;
+        }
+
+        // This segment's activations do not depend on the stage: load them
+        // before the wait so their latency overlaps it (single token).
+        constexpr bool kPreload = (MT == 1);
+        uint32_t pre[kPreload ? kIt : 1][16];
+        if constexpr (kPreload) {
+#pragma unroll
+            for (int it = 0; it < kIt; ++it) {
+                const int chunk = cons.c + it * 32 + lane;
+                load_act_chunk(pr.xq + (int64_t)m0 * pr.K, pr.K, chunk, chunk < pr.full_chunks,
+                               it * 32 + lane < n && m0 < pr.M, pre[it]);
             }
+        }
+
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * st, phase))) {
+            // Give up: record the error, let this warp's copies in flight land
+            // (bounded again), then leave.
+            if (lane == 0) atomicCAS(&g_device_error, 0, (int)BL_ERR_TIMEOUT);
+            for (int i = seg + 1; i < issued; ++i) mbar_wait_bounded(bar0 + 8 * (i % kStages), (i / kStages) & 1);
+            return;
+        }
+        const uint32_t sbase = stage0 + st * kStageBytes;
+        constexpr int kItUnroll = (MT == 1) ? kIt : 1;  // keep MT > 1 within registers
+#pragma unroll(kItUnroll)
+        for (int it = 0; it < kIt; ++it) {
+            const int j = it * 32 + lane;
+            if (j < n) {
+                const int chunk = cons.c + j;
+                uint32_t av[MT][16];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
+                for (int m = 0; m < MT; ++m) {
+                    if constexpr (kPreload) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t word = word_of(w[r], j);
+                        for (int q = 0; q < 16; ++q) av[m][q] = pre[it][q];
+                    } else {
+                        load_act_chunk(pr.xq + (int64_t)(m0 + m) * pr.K, pr.K, chunk, chunk < pr.full_chunks,
+                                       m0 + m < pr.M, av[m]);
+                    }
+                    if (!sx_from_cache) {
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        if constexpr (MT == 1) {
-                            // codes of weights 16j+4s .. 16j+4s+3, each times 4^s
-                            const uint32_t codes = word & (0x03030303u << (2 * s));
-                            acc[r][0][s] = dp4a_u8s8(codes, a[0][4 * j + s], acc[r][0][s]);
-                        } else {
-                            const uint32_t codes = (word >> (2 * s)) & 0x03030303u;
+                        for (int q = 0; q < 16; ++q) sx[m] = dp4a_s8s8(0x01010101u, av[m][q], sx[m]);
+                    }
+                }
 #pragma unroll
-                            for (int m = 0; m < MT; ++m) acc[r][m][0] = dp4a_u8s8(codes, a[m][4 * j + s], acc[r][m][0]);
+                for (int r = 0; r < kRG; ++r) {
+                    const uint4 w = lds128(sbase + r * kRowStride + j * 16);
+#pragma unroll
+                    for (int wj = 0; wj < 4; ++wj) {
+                        const uint32_t word = word_of(w, wj);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if constexpr (kMask) {
+                                const uint32_t codes = word & (0x03030303u << (2 * q));
+#pragma unroll
+                                for (int m = 0; m < MT; ++m)
+                                    acc[r][m][q] = dp4a_u8s8(codes, av[m][4 * wj + q], acc[r][m][q]);
+                            } else {
+                                const uint32_t codes = (word >> (2 * q)) & 0x03030303u;
+#pragma unroll
+                                for (int m = 0; m < MT; ++m)
+                                    acc[r][m][0] = dp4a_u8s8(codes, av[m][4 * wj + q], acc[r][m][0]);
+                            }
                         }
                     }
                 }
             }
         }
+        rg_chunks += n;
+        const bool rg_whole = (cons.c + n == pr.C) && (rg_chunks == pr.C);
+        const bool rg_done = (cons.c + n == pr.C) || (cons.u + n == cons.end);
+        const int seg_p = cons.p;
+        const int64_t rg_u0 = pr.unit_begin + (int64_t)cons.tgrg * pr.C;
 
-        // Σ (c - 1)·x̃ per (row, token), exact in int32; then all-reduce over the warp.
-        int v[R * MT];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                int d;
-                if constexpr (MT == 1)
-                    d = acc[r][0][0] + (acc[r][0][1] >> 2) + (acc[r][0][2] >> 4) + (acc[r][0][3] >> 6);
-                else
-                    d = acc[r][m][0];
-                v[m * R + r] = d - sx[m];
-            }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-            for (int i = 0; i < R * MT; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], off);
+        // refill this stage with the segment kStages ahead
+        __syncwarp();
+        if (prod.u < prod.end) {
+            const int pn = cursor_len(P, prod);
+            const SProblem& pp = P.p[prod.p];
+            issue_segment(pp, prod.tgrg % pp.rgn, prod.c, pn, sbase, bar0 + 8 * st, policy, lane);
+            cursor_advance(P, prod, pn);
+            ++issued;
+        }
+        cursor_advance(P, cons, n);
 
-        if (lane < R * MT) {
-            int val = 0;
+        if (rg_done) {
+            if (rg_whole && !sx_from_cache) {
+                // a whole row group from chunk 0 (segments at multiples of 64
+                // chunks, so chunk j always fell to lane j mod 32): cache Σx̃
+                cache_p = seg_p;
+                cache_tg = tg;
 #pragma unroll
-            for (int i = 0; i < R * MT; ++i)
-                if (i == lane) val = v[i];
-            const int r = lane % R, m = lane / R;
-            const int64_t n = n0 + r, mm = m0 + m;
-            if (n < pr.N && mm < pr.M) {
-                const float s = dequant_scale(*pr.alpha, pr.beta[mm]);
-                float out = __fmul_rn((float)val, s);
-                if (pr.bias) out = __fadd_rn(out, pr.bias[n]);
-                pr.y[mm * pr.N + n] = out;
-                if (pr.acc_out) pr.acc_out[mm * pr.N + n] = val;
+                for (int m = 0; m < MT; ++m) sx_cache[m] = sx[m];
             }
+            int v[V];
+#pragma unroll
+            for (int r = 0; r < kRG; ++r)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    int d;
+                    if constexpr (kMask)
+                        d = acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6);
+                    else
+                        d = acc[r][m][0];
+                    v[m * kRG + r] = d - sx[m];
+                }
+            int idx;
+            int val = reduce_scatter<V>(v, lane, idx);
+            const bool writer = (lane & (32 / V - 1)) == 0;
+
+            bool finish = rg_whole;
+            if (!rg_whole) {
+                // shared row group: add into its slot; the last contributor finishes it
+                int slot = 0;
+                for (int w = 1; w <= kWarps - 1; ++w) {
+                    const int64_t bw = S.bound[w];
+                    if (bw > rg_u0 && bw < rg_u0 + pr.C) {
+                        slot = w;
+                        break;
+                    }
+                }
+                if (writer) atomicAdd(&S.slot_acc[slot][idx], val);
+                __threadfence_block();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = (atomicAdd(&S.slot_count[slot], rg_chunks) + rg_chunks == pr.C);
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence_block();
+                    if (writer) val = atomicAdd(&S.slot_acc[slot][idx], 0);
+                    finish = true;
+                }
+            }
+            if (finish) {
+                const int r = idx % kRG, m = idx / kRG;
+                const int row = rg * kRG + r, tok = m0 + m;
+                if (scale_p != seg_p || scale_tg != tg) {  // once per (problem, token group)
+                    scale_p = seg_p;
+                    scale_tg = tg;
+                    scale = dequant_scale(alpha_v, beta_v);
+                }
+                if (writer && row < pr.N && tok < pr.M) {
+                    float out = __fmul_rn((float)val, scale);
+                    if (pr.bias) out = __fadd_rn(out, pr.bias[row]);
+                    pr.y[(int64_t)tok * pr.N + row] = out;
+                    if (pr.acc_out) pr.acc_out[(int64_t)tok * pr.N + row] = val;
+                }
+            }
+            rg_chunks = 0;
         }
     }
 }
 
 // Any K and any x̃ alignment: one warp per output element, byte loads.
-__global__ void __launch_bounds__(kThreads) gemv_generic_kernel(const __grid_constant__ GemvParams P) {
+struct GenericProblem {
+    const int8_t* xq;
+    const float* beta;
+    const uint32_t* W;
+    const float* alpha;
+    const float* bias;
+    float* y;
+    int32_t* acc_out;
+    int64_t M, N, K, row_words, task_begin;
+};
+struct GenericParams {
+    GenericProblem p[kMaxGroup];
+    int count;
+    int64_t total_tasks;
+};
+
+__global__ void __launch_bounds__(256) gemv_generic_kernel(const __grid_constant__ GenericParams P) {
     const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const int64_t warp0 = ((int64_t)blockIdx.x * 256 + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * 256) >> 5;
     for (int64_t t = warp0; t < P.total_tasks; t += nwarps) {
         int pi = 0;
         while (pi + 1 < P.count && t >= P.p[pi + 1].task_begin) ++pi;
-        const GemvProblem& pr = P.p[pi];
+        const GenericProblem& pr = P.p[pi];
         const int64_t lt = t - pr.task_begin;
         const int64_t m = lt / pr.N, n = lt - m * pr.N;
         const int8_t* xrow = pr.xq + m * pr.K;
@@ -217,56 +511,77 @@ __global__ void __launch_bounds__(kThreads) gemv_generic_kernel(const __grid_con
     }
 }
 
-template <int MT, int R>
-cudaError_t launch_fast(GemvParams& P, const DeviceInfo& dev, cudaStream_t stream) {
-    int64_t total = 0;
-    for (int i = 0; i < P.count; ++i) {
-        GemvProblem& q = P.p[i];
-        q.row_groups = (q.N + R - 1) / R;
-        q.task_begin = total;
-        total += q.row_groups * ((q.M + MT - 1) / MT);
-    }
-    P.total_tasks = total;
-    static int occ[64] = {};
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[0], gemv_ternary_kernel<MT, R>, kThreads, 0);
-    });
-    const int per_sm = occ[0] > 0 ? occ[0] : 1;
-    int64_t blocks = (total + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)dev.sm_count * per_sm;
-    if (blocks > cap) blocks = cap;
-    gemv_ternary_kernel<MT, R><<<(unsigned)blocks, kThreads, 0, stream>>>(P);
-    return cudaGetLastError();
+// Waits on an mbarrier that nothing ever completes, with a caller-chosen
+// bound, to exercise the timeout path (sets the device error, then returns).
+__global__ void wait_timeout_selftest_kernel(uint32_t polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+    __syncthreads();
+    bool ok = false;
+    for (uint32_t i = 0; i < polls && !ok; ++i) ok = mbar_try_wait(smem_addr(&bar), 0, 1000);
+    if (!ok && threadIdx.x == 0) atomicCAS(&g_device_error, 0, (int)BL_ERR_TIMEOUT);
 }
 
-cudaError_t launch_generic(GemvParams& P, const DeviceInfo& dev, cudaStream_t stream) {
-    int64_t total = 0;
-    for (int i = 0; i < P.count; ++i) {
-        P.p[i].task_begin = total;
-        total += P.p[i].M * P.p[i].N;
-    }
-    P.total_tasks = total;
-    int64_t blocks = (total + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)dev.sm_count * 8;
-    if (blocks > cap) blocks = cap;
-    gemv_generic_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(P);
-    return cudaGetLastError();
-}
-
-}  // namespace
-
-cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream) {
-    DeviceInfo dev;
-    cudaError_t err = device_info(&dev);
-    if (err != cudaSuccess) return err;
-    GemvParams P{};
+template <int MT>
+cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
+                          cudaStream_t stream, bool pdl) {
+    SParams P{};
     P.count = count;
-    bool fast = true;
-    int64_t max_m = 0;
+    int64_t total = 0, row_groups = 0;
     for (int i = 0; i < count; ++i) {
         const bitlinear_forward_problem& s = problems[i];
-        GemvProblem& q = P.p[i];
+        SProblem& q = P.p[i];
+        q.xq = s.x_q;
+        q.beta = s.beta;
+        q.W = s.W_packed;
+        q.alpha = s.alpha;
+        q.bias = s.bias;
+        q.y = s.y;
+        q.acc_out = s.acc_out;
+        q.M = (int32_t)s.M;
+        q.N = (int32_t)s.N;
+        q.K = (int32_t)s.K;
+        q.row_bytes = (int32_t)bitlinear_packed_row_bytes(s.K);
+        q.C = q.row_bytes / 16;
+        q.full_chunks = q.K / 64;
+        q.rgn = (q.N + kRG - 1) / kRG;
+        q.tgn = (q.M + MT - 1) / MT;
+        q.unit_begin = total;
+        total += (int64_t)q.tgn * q.rgn * q.C;
+        row_groups += (int64_t)q.tgn * q.rgn;
+    }
+    P.total_units = total;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)sizeof(SharedLayout));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    int64_t grid = dev.sm_count;
+    if (grid > row_groups) grid = row_groups;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sizeof(SharedLayout);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MT>, P);
+}
+
+cudaError_t launch_generic(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
+                           cudaStream_t stream) {
+    GenericParams P{};
+    P.count = count;
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_forward_problem& s = problems[i];
+        GenericProblem& q = P.p[i];
         q.xq = s.x_q;
         q.beta = s.beta;
         q.W = reinterpret_cast<const uint32_t*>(s.W_packed);
@@ -278,13 +593,48 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
         q.N = s.N;
         q.K = s.K;
         q.row_words = (int64_t)bitlinear_packed_row_bytes(s.K) / 4;
+        q.task_begin = total;
+        total += s.M * s.N;
+    }
+    P.total_tasks = total;
+    int64_t blocks = (total + 7) / 8;
+    const int64_t cap = (int64_t)dev.sm_count * 8;
+    if (blocks > cap) blocks = cap;
+    gemv_generic_kernel<<<(unsigned)blocks, 256, 0, stream>>>(P);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl) {
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    bool fast = true;
+    int64_t max_m = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_forward_problem& s = problems[i];
         fast = fast && (s.K % 16 == 0) && ((reinterpret_cast<uintptr_t>(s.x_q) & 15) == 0);
+        // the streaming kernel indexes (token group, row group) pairs in 32 bits
+        fast = fast && ((s.M + 3) / 4) * ((s.N + kRG - 1) / kRG) < ((int64_t)1 << 30);
         if (s.M > max_m) max_m = s.M;
     }
-    if (!fast) return launch_generic(P, dev, stream);
-    if (max_m == 1) return launch_fast<1, 8>(P, dev, stream);
-    if (max_m == 2) return launch_fast<2, 4>(P, dev, stream);
-    return launch_fast<4, 4>(P, dev, stream);
+    if (!fast) return launch_generic(problems, count, dev, stream);
+    if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl);
+    if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl);
+    return launch_stream<4>(problems, count, dev, stream, pdl);
+}
+
+cudaError_t read_device_error(int* code) {
+    int zero = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(code, g_device_error, sizeof(int));
+    if (err != cudaSuccess) return err;
+    return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+}
+
+cudaError_t launch_wait_timeout_selftest(uint32_t polls, cudaStream_t stream) {
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(polls);
+    return cudaGetLastError();
 }
 
 }  // namespace bl

@@ -51,7 +51,9 @@ typedef enum bitlinear_status {
     BL_ERR_WORKSPACE = 5, /* workspace NULL or smaller than required */
     BL_ERR_ARCH = 6,      /* current device is not compute capability 10.0 */
     BL_ERR_CUDA = 7,      /* the CUDA runtime reported an error */
-    BL_ERR_COUNT = 8      /* group count outside 1..BITLINEAR_MAX_GROUP */
+    BL_ERR_COUNT = 8,     /* group count outside 1..BITLINEAR_MAX_GROUP */
+    BL_ERR_TIMEOUT = 9,   /* a kernel's bounded wait expired (see bitlinear_device_error) */
+    BL_ERR_FLAGS = 10     /* unknown flag bits */
 } bitlinear_status;
 
 typedef enum bitlinear_dtype {
@@ -189,6 +191,60 @@ typedef struct bitlinear_forward_problem {
  * Errors: as bitlinear_forward, plus BL_ERR_COUNT. */
 BITLINEAR_API bitlinear_status bitlinear_forward_grouped(const bitlinear_forward_problem* problems, int count,
                                            bitlinear_stream_t stream);
+
+/* One problem of a grouped linear (activation quantisation + forward);
+ * fields as in bitlinear_quantize_act and bitlinear_forward.  x_q and beta are
+ * outputs of the first step and inputs of the second. */
+typedef struct bitlinear_linear_problem {
+    const void* x;
+    int8_t* x_q;
+    float* beta;
+    const uint8_t* W_packed;
+    const float* alpha;
+    const float* bias;
+    float* y;
+    int32_t* acc_out;
+    int64_t M, N, K;
+} bitlinear_linear_problem;
+
+/* The BitLinear forward on cached weights (chenxutan.com/d/5049.html §3.2,
+ * steps 2-4): bitlinear_quantize_act on x, then bitlinear_forward, with
+ * identical results.  Both kernels use programmatic dependent launch: the
+ * quantisation kernel waits for the work before it on `stream` before reading
+ * x, and the product kernel starts streaming its weights as soon as the
+ * quantisation kernel releases it, then waits for x̃ and β.  So consecutive
+ * calls overlap each other's start-up and drain.
+ * Errors: the union of both calls'. */
+BITLINEAR_API bitlinear_status bitlinear_linear(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K,
+                                                const uint8_t* W_packed, const float* alpha, int64_t N,
+                                                const float* bias, int8_t* x_q, float* beta, float* y,
+                                                int32_t* acc_out, bitlinear_stream_t stream);
+
+/* Flag for bitlinear_linear_grouped: the weights (W_packed, alpha) of this
+ * call are not written by any work still running on the stream.  The product
+ * kernel may then begin streaming weights while the work before the call is
+ * still finishing (e.g. the previous layer's product), instead of after it. */
+#define BL_LINEAR_WEIGHTS_STATIC 1u
+
+/* bitlinear_linear on `count` independent problems of one input dtype: one
+ * grouped quantisation launch and one grouped product launch.  `problems` is a
+ * HOST array.  flags: 0 or BL_LINEAR_WEIGHTS_STATIC.
+ * Errors: as bitlinear_linear, plus BL_ERR_COUNT, BL_ERR_FLAGS. */
+BITLINEAR_API bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* problems, int count,
+                                                        bitlinear_dtype dtype, uint32_t flags,
+                                                        bitlinear_stream_t stream);
+
+/* Reads and clears the current device's error word, which a kernel sets when
+ * one of its bounded waits expires (it then stops early and its outputs are
+ * undefined).  Synchronous: call after the streams that ran the kernels have
+ * been synchronised.  *code receives 0 or a bitlinear_status code; returns
+ * BL_OK, BL_ERR_NULL or BL_ERR_CUDA. */
+BITLINEAR_API bitlinear_status bitlinear_device_error(int* code);
+
+/* Self-test of the timeout path: launches one CTA that waits on an mbarrier
+ * nothing ever completes, for at most `polls` polls, after which it sets the
+ * device error word to BL_ERR_TIMEOUT and returns.  No other state changes. */
+BITLINEAR_API bitlinear_status bitlinear_selftest_timeout(uint32_t polls, bitlinear_stream_t stream);
 
 /* Static description of a status code. */
 BITLINEAR_API const char* bitlinear_status_string(bitlinear_status status);

@@ -13,7 +13,7 @@ import bitlinear_w1_a8_03_b200 as bl
 from bitlinear_w1_a8_03_b200 import build as blbuild
 
 HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bitlinear.h")
-OK, NULL, SHAPE, ALIGN, DTYPE, WORKSPACE, ARCH, CUDA, COUNT = range(9)
+OK, NULL, SHAPE, ALIGN, DTYPE, WORKSPACE, ARCH, CUDA, COUNT, TIMEOUT, FLAGS = range(11)
 P = 0x7F0000000000  # 16-byte aligned fake device address (never dereferenced)
 
 
@@ -49,7 +49,7 @@ def test_packed_row_bytes(L):
 
 
 def test_status_strings(L):
-    for s in range(9):
+    for s in range(11):
         assert L.bitlinear_status_string(s)
     assert b"unknown" in L.bitlinear_status_string(99)
 
@@ -96,6 +96,9 @@ def test_forward_argument_errors(L):
     assert f(P, P, 1, 64, P, P, 8, P + 2, P, None, None) == ALIGN  # bias
     arr = (bl.ForwardProblem * 1)()
     assert L.bitlinear_forward_grouped(arr, 0, None) == COUNT
+    lin = (bl.LinearProblem * 1)()
+    assert L.bitlinear_linear_grouped(lin, 1, 0, 2, None) == 10  # BL_ERR_FLAGS
+    assert L.bitlinear_linear_grouped(lin, 1, 0, 0, None) == NULL
     assert L.bitlinear_forward_grouped(None, 1, None) == NULL
 
 

@@ -219,3 +219,92 @@ def test_outputs_stay_in_bounds():
         raw = np_(t.view(torch.uint8))
         es = t.element_size()
         assert np.all(raw[: G * es] == 0x5A) and np.all(raw[(G + n) * es:] == 0x5A)
+
+
+# ---------------------------------------------------------------- fused linear (PDL) path
+@pytest.mark.parametrize("M,K,N", [(1, 4096, 300), (2, 1024, 77), (3, 512, 64), (5, 4096 + 16, 40), (1, 100, 9)])
+def test_linear_matches_oracle(M, K, N):
+    import bitlinear_w1_a8_03_b200 as bl
+    W = synth.weights(K + N, N, K, 0.02)
+    x = synth.activations(K + M, M, K, outliers=True)
+    bias = synth.activations(7, 1, N)[0]
+    packed, alpha, codes, a_ref = check_weights(W, "f32")
+    xd, xo = as_input(x, "bf16")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    beta = torch.empty(M, dtype=torch.float32, device="cuda")
+    y = bl.bitlinear_linear(xd, packed, alpha, N, bias=dev_f32(bias), x_q=xq, beta=beta, acc_out=acc)
+    xq_r, beta_r, acc_r, y_r = oracle.forward(xo, codes, a_ref, bias=bias)
+    assert np.array_equal(np_(xq), xq_r) and np.array_equal(np_(beta), beta_r)
+    assert np.array_equal(np_(acc), acc_r)
+    assert_y_close(np_(y), y_r)
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_linear_grouped_back_to_back_inputs_change(flags):
+    """Steps with different inputs on the same buffers, queued without any
+    host sync: each product must see its own step's x̃ (the weight stream
+    starts before the quantisation kernel finishes)."""
+    import bitlinear_w1_a8_03_b200 as bl
+    shapes = [(4096, 4096), (4096, 1000), (1024, 512)]
+    Ws = [synth.weights(70 + i, N, K, 0.02) for i, (K, N) in enumerate(shapes)]
+    quant = [check_weights(W, "f32") for W in Ws]
+    x_dev = [torch.empty((1, K), dtype=torch.bfloat16, device="cuda") for K, _ in shapes]
+    xq = [torch.empty((1, K), dtype=torch.int8, device="cuda") for K, _ in shapes]
+    beta = [torch.empty(1, dtype=torch.float32, device="cuda") for _ in shapes]
+    steps = 4
+    ys = [[torch.empty((1, N), dtype=torch.float32, device="cuda") for _, N in shapes] for _ in range(steps)]
+    xo_all = []
+    for t in range(steps):
+        xo_step = []
+        for i, (K, N) in enumerate(shapes):
+            xd, xo = as_input(synth.activations(900 + 10 * t + i, 1, K, outliers=True), "bf16")
+            x_dev[i].copy_(xd, non_blocking=True)
+            xo_step.append(xo)
+        xo_all.append(xo_step)
+        probs = [dict(x=x_dev[i], x_q=xq[i], beta=beta[i], W_packed=quant[i][0], alpha=quant[i][1], N=N, y=ys[t][i])
+                 for i, (K, N) in enumerate(shapes)]
+        bl.bitlinear_linear_grouped(probs, flags=flags)
+    torch.cuda.synchronize()
+    for t in range(steps):
+        for i, (K, N) in enumerate(shapes):
+            packed, alpha, codes, a_ref = quant[i]
+            _, _, _, y_r = oracle.forward(xo_all[t][i], codes, a_ref)
+            assert_y_close(np_(ys[t][i]), y_r)
+
+
+# ---------------------------------------------------------------- failure detection
+def test_bounded_wait_reports_timeout():
+    """A wait on an mbarrier that nothing completes gives up after its bound,
+    records BL_ERR_TIMEOUT in the device error word and returns; the context
+    stays usable."""
+    import bitlinear_w1_a8_03_b200 as bl
+    assert bl.bitlinear_device_error() == 0
+    bl.check(bl.lib().bitlinear_selftest_timeout(2000, torch.cuda.current_stream().cuda_stream), "selftest")
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 9
+    assert bl.bitlinear_device_error() == 0  # read clears it
+    t = torch.ones(1000, device="cuda")
+    assert float(t.sum()) == 1000.0
+
+
+def test_linear_right_after_weight_quantisation_without_sync():
+    """Default flags: the product kernel may not read weights that work still
+    in flight is writing, so quantising and using them back to back with no
+    host synchronisation must give the oracle's result."""
+    import bitlinear_w1_a8_03_b200 as bl
+    K, N = 4096, 2048
+    W = synth.weights(31, N, K, 0.02)
+    x = synth.activations(31, 1, K, outliers=True)
+    Wd, Wo = as_input(W, "f32")
+    xd, xo = as_input(x, "bf16")
+    torch.cuda.synchronize()
+    for rep in range(3):
+        packed = torch.empty((N, bl.packed_row_bytes(K)), dtype=torch.uint8, device="cuda")
+        packed.fill_(0xAA)  # garbage a premature read would see
+        alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+        bl.bitlinear_quantize_weights(Wd, W_packed=packed, alpha=alpha)
+        y = bl.bitlinear_linear(xd, packed, alpha, N)
+        _, a_ref, codes = oracle.quantize_weights(Wo)
+        _, _, _, y_r = oracle.forward(xo, codes, a_ref)
+        assert_y_close(np_(y), y_r)
