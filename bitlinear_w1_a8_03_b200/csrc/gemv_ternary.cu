@@ -141,12 +141,22 @@ __device__ int64_t snap_to_row_group(const SParams& P, int64_t t) {
     return P.p[p].unit_begin + g * P.p[p].C;
 }
 
+// The last activation chunk of a row when K is not a multiple of 64: bytes
+// past K read as zero.  Kept out of line so the full-chunk path stays lean.
+__device__ __noinline__ void load_act_tail(const int8_t* xrow, int K, int chunk, uint32_t* a) {
+    for (int q = 0; q < 16; ++q) {
+        uint32_t w = 0;
+        for (int b = 0; b < 4; ++b) {
+            const int k = 64 * chunk + 4 * q + b;
+            if (k < K) w |= (uint32_t)(uint8_t)xrow[k] << (8 * b);
+        }
+        a[q] = w;
+    }
+}
+
 __device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int K, int chunk, bool full, bool valid,
                                                uint32_t (&a)[16]) {
-    if (!valid) {
-#pragma unroll
-        for (int q = 0; q < 16; ++q) a[q] = 0u;
-    } else if (full) {
+    if (valid && full) {
         const int8_t* p = xrow + 64 * chunk;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -156,17 +166,14 @@ __device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int K, int ch
             a[4 * v + 2] = u.z;
             a[4 * v + 3] = u.w;
         }
+    } else if (valid) {
+        uint32_t tmp[16];  // only this rare path goes through local memory
+        load_act_tail(xrow, K, chunk, tmp);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) a[q] = tmp[q];
     } else {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            uint32_t w = 0;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int k = 64 * chunk + 4 * q + b;
-                if (k < K) w |= (uint32_t)(uint8_t)xrow[k] << (8 * b);
-            }
-            a[q] = w;
-        }
+        for (int q = 0; q < 16; ++q) a[q] = 0u;
     }
 }
 
