@@ -203,7 +203,11 @@ bitlinear_status bitlinear_device_error(int* code) {
     if (!code) return BL_ERR_NULL;
     bitlinear_status st = check_device();
     if (st != BL_OK) return st;
-    return from_cuda(bl::read_device_error(code));
+    int a = 0, b = 0;
+    cudaError_t err = bl::read_device_error(&a);
+    if (err == cudaSuccess) err = bl::read_gemm_error(&b);
+    *code = a ? a : b;
+    return from_cuda(err);
 }
 
 bitlinear_status bitlinear_selftest_timeout(uint32_t polls, bitlinear_stream_t stream) {

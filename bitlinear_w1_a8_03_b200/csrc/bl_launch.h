@@ -36,6 +36,11 @@ cudaError_t launch_quantize_weights_static(const void* W, bitlinear_dtype dtype,
 // stream starts before the dependency wait).
 cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl);
 
+// Tensor-core GEMM for many tokens (tcgen05, int8): one problem per launch.
+bool gemm_tc_supported(const bitlinear_forward_problem& p);
+cudaError_t launch_gemm_tc(const bitlinear_forward_problem& p, cudaStream_t stream, bool pdl);
+cudaError_t read_gemm_error(int* code);
+
 // Device-side error word (bounded waits that expired): read and clear.
 cudaError_t read_device_error(int* code);
 cudaError_t launch_wait_timeout_selftest(uint32_t polls, cudaStream_t stream);

@@ -59,6 +59,7 @@ constexpr int kRowStride = kSegChunks * 16;     // bytes per staged row
 constexpr int kStageBytes = kRG * kRowStride;   // 8 KiB
 constexpr int kSlots = kWarps;                  // row groups shared between warps
 constexpr int kMaxMT = 4;
+constexpr int kGemvMaxTokens = 4;  // more tokens go to the tensor-core GEMM
 
 struct SProblem {
     const int8_t* xq;
@@ -627,6 +628,18 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
         if (s.M > max_m) max_m = s.M;
     }
     if (!fast) return launch_generic(problems, count, dev, stream);
+    if (max_m > kGemvMaxTokens) {
+        // many tokens: the int8 tensor cores, one launch per problem
+        bool tc = true;
+        for (int i = 0; i < count; ++i) tc = tc && gemm_tc_supported(problems[i]);
+        if (tc) {
+            for (int i = 0; i < count; ++i) {
+                err = launch_gemm_tc(problems[i], stream, pdl && i == 0);
+                if (err != cudaSuccess) return err;
+            }
+            return cudaSuccess;
+        }
+    }
     if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl);
     if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl);
     return launch_stream<4>(problems, count, dev, stream, pdl);

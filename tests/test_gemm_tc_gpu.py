@@ -1,0 +1,49 @@
+"""Tensor-core (tcgen05) GEMM path: more than four tokens go through the int8
+tensor cores.  Bit-exact int32 accumulators and x̃ against the oracle, fp32
+outputs within 1e-5 relative, over token counts that cover every tile width
+(16 .. 256 tokens) with ragged edges in tokens, rows and K."""
+import numpy as np
+import pytest
+import torch
+
+import bitlinear_w1_a8_03_b200 as bl
+import oracle
+from bitlinear_w1_a8_03_b200 import synth
+from tests.gpu_util import as_input, dev_f32, np_
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(M, K, N, seed, bias=False, dtype="bf16"):
+    W = synth.weights(seed, N, K, 0.02)
+    x = synth.activations(seed, M, K, outliers=True)
+    Wd, Wo = as_input(W, "f32")
+    packed, alpha = bl.bitlinear_quantize_weights(Wd)
+    p_ref, a_ref, codes = oracle.quantize_weights(Wo)
+    assert np_(alpha)[0] == a_ref and np.array_equal(np_(packed), p_ref)
+    xd, xo = as_input(x, dtype)
+    b = synth.activations(seed + 1, 1, N)[0] if bias else None
+    xq, beta = bl.bitlinear_quantize_act(xd)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    y = bl.bitlinear_forward(xq, beta, packed, alpha, N, bias=None if b is None else dev_f32(b), acc_out=acc)
+    xq_r, beta_r, acc_r, y_r = oracle.forward(xo, codes, a_ref, bias=b, threads=8)
+    assert np.array_equal(np_(xq), xq_r)
+    assert np.array_equal(np_(acc), acc_r)
+    err = np.abs(np_(y).astype(np.float64) - y_r)
+    assert np.all(err <= 1e-5 * np.abs(y_r) + 1e-37)
+    assert bl.bitlinear_device_error() == 0
+
+
+@pytest.mark.parametrize("M", [5, 8, 16, 17, 32, 33, 64, 65, 128, 129, 256, 300])
+def test_gemm_token_counts(M):
+    run_case(M, 256, 200, seed=600 + M, bias=(M % 2 == 1))
+
+
+@pytest.mark.parametrize("K,N", [(16, 130), (48, 128), (128, 127), (192, 257), (1024, 384), (4096 + 64, 256)])
+def test_gemm_ragged_k_and_rows(K, N):
+    run_case(37, K, N, seed=700 + K + N)
+
+
+def test_gemm_prefill_shape_small_rows():
+    """2048 tokens (the prefill token count) on a few hundred rows."""
+    run_case(2048, 1024, 256, seed=800, dtype="f32")
