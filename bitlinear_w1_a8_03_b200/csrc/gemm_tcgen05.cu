@@ -7,19 +7,26 @@
 // GEMM-shaped batched case) and the dequantisation y = fp32(acc)·α·β/127 +
 // bias ("1.58-bit 大模型极限量化实战", chenxutan.com/d/5049.html §2.4–§2.5, §4.2).
 //
-// Tile: 128 weight rows (the MMA's M side) × NT tokens (its N side) per CTA,
-// K in blocks of 128.  Warp roles:
-//   warp 0  one thread loads x̃ tiles [NT tokens][128 bytes] with TMA (128-byte
-//           swizzle) into a ring of stages;
-//   warp 1  owns the tensor memory (NT int32 columns) and one thread issues
-//           tcgen05.mma.kind::i8 (4 per K block) and the commits that free a
-//           stage / publish the accumulator;
-//   warps 2-5 expand the 2-bit codes of their row (one row per thread) into
-//           signed bytes {-1, 0, +1} in the UMMA K-major 128-byte-swizzled
-//           layout, then run the epilogue: tcgen05.ld of the row's
-//           accumulators, scale, store (consecutive threads = consecutive rows).
-// Every wait is bounded; on expiry the kernel records BL_ERR_TIMEOUT, lets
-// its copies and MMAs drain (bounded) and frees its tensor memory.
+// Persistent kernel, one CTA per SM.  A tile is 128 weight rows (the MMA's M
+// side) × NT tokens (its N side); K runs in blocks of 128.  Tiles are dealt
+// round-robin to the CTAs.  Warp roles (11 warps):
+//   warp 0      one thread loads x̃ tiles [NT tokens][128 B] by TMA (128-byte
+//               swizzle) into ring B;
+//   warp 10     one thread loads packed-code tiles [128 rows][32 B] by TMA
+//               into ring W, running ahead of the tensor cores;
+//   warps 2-5   expand the 2-bit codes of one row each (one row per thread)
+//               from ring W into signed bytes {-1, 0, +1} in ring A, laid out
+//               K-major with the 128-byte swizzle the MMA descriptors expect;
+//   warp 1      owns the tensor memory (two NT-column int32 accumulators) and
+//               one thread issues tcgen05.mma.kind::i8 (4 per K block) and the
+//               commits that free ring slots / publish an accumulator;
+//   warps 6-9   epilogue: tcgen05.ld of a row's accumulators, scale by the
+//               token's α·β/127, add bias, store (consecutive threads write
+//               consecutive rows); overlaps the next tile's MMAs because the
+//               accumulator is double-buffered.
+// Every wait is bounded; on expiry the kernel records BL_ERR_TIMEOUT, the
+// other roles stop at their next wait, copies and MMAs in flight drain
+// (bounded) and the tensor memory is freed.
 #include <cuda.h>
 
 #include <mutex>
@@ -34,30 +41,41 @@ static __device__ int g_gemm_error;
 
 namespace {
 
-constexpr int kKB = 128;          // K bytes (= weights) per block
+constexpr int kKB = 128;          // K (bytes of x̃ = weights) per block
+constexpr int kWB = kKB / 4;      // packed bytes of one row per K block
 constexpr int kRowsTile = 128;    // weight rows per tile (MMA M)
-constexpr int kThreads = 6 * 32;  // producer, MMA, 4 expander/epilogue warps
-constexpr int kExp = 128;         // expander threads
+constexpr int kWarps = 11;
+constexpr int kThreads = kWarps * 32;
+constexpr int kWarpTmaX = 0, kWarpMma = 1, kWarpExp0 = 2, kWarpEpi0 = 6, kWarpTmaW = 10;
+constexpr int kExpWarps = 4, kEpiWarps = 4;
+constexpr size_t kSmemLimit = 232448;  // opt-in dynamic shared memory per block on sm_100
 
 template <int NT>
 struct Cfg {
-    static constexpr int kStages = NT >= 256 ? 3 : 4;
-    static constexpr int kABytes = kRowsTile * kKB;  // 16 KiB
-    static constexpr int kBBytes = NT * kKB;         // NT × 128 B
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kTmemCols = NT < 32 ? 32 : NT;
+    static constexpr int kABytes = kRowsTile * kKB;  // 16 KiB of expanded codes
+    static constexpr int kBBytes = NT * kKB;         // NT × 128 B of x̃
+    static constexpr int kWBytes = kRowsTile * kWB;  // 4 KiB of packed codes
+    static constexpr int kSA = NT >= 256 ? 2 : (NT >= 128 ? 3 : 4);
+    static constexpr int kSW = NT >= 256 ? 6 : (NT >= 128 ? 8 : 16);
+    static constexpr int kSB = NT >= 256 ? 5 : (NT >= 128 ? 8 : (NT >= 64 ? 10 : 12));
+    static constexpr int kBars = 2 * (kSA + kSB + kSW) + 5;
+    static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;  // two accumulators
+    static constexpr size_t kRingBytes =
+        (size_t)kSA * kABytes + (size_t)kSB * kBBytes + (size_t)kSW * kWBytes;
+    static constexpr size_t kSmem = 1024 + kRingBytes + kBars * 8 + 16;
+    static_assert(kSmem <= kSmemLimit, "shared memory budget");
+    static_assert(kSmem > kSmemLimit / 2, "one CTA per SM (the tensor memory is sized for one)");
 };
 
 struct GemmParams {
-    const uint8_t* W;  // packed rows
     const float* alpha;
     const float* beta;
     const float* bias;
     float* y;
     int32_t* acc_out;
-    int M, N, K;
-    int row_bytes;
+    int M, N;
     int kblocks;
+    int tiles_m, tiles;
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -99,6 +117,7 @@ __device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t
         : "memory");
 }
 
+// The mbarrier arrives once every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -127,172 +146,232 @@ __device__ __forceinline__ uint32_t field_s8(uint32_t w, int s) {
     return (c - 0x01010101u) ^ 0x80808080u;
 }
 
+__device__ __forceinline__ void record_timeout(volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicCAS(&g_gemm_error, 0, (int)BL_ERR_TIMEOUT);
+}
+
+// Waits for phase `parity` of `bar` unless the CTA is aborting; false (and
+// the abort recorded) if it did not complete.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait_bounded(bar, parity)) return true;
+    record_timeout(abort_flag);
+    return false;
+}
+
+// A TMA producer's loop: one box per K block of every tile of this CTA into a
+// ring of S slots, each reused once the consumer frees it.  On the way out it
+// waits (bounded) for the copies it issued, so no copy lands after the CTA
+// has exited.
+template <int S, typename Coord>
+__device__ void tma_producer(const CUtensorMap* map, uint8_t* ring, uint32_t slot_bytes, uint64_t* full,
+                             uint64_t* empty, const GemmParams& P, volatile int* abort_flag, Coord coord) {
+    int it = 0;
+    for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+        for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
+            const int s = it % S;
+            if (it >= S && !wait_or_abort(smem_addr(&empty[s]), ((it / S) - 1) & 1, abort_flag)) goto drain;
+            int x, y;
+            coord(tile, kb, x, y);
+            mbar_arrive_expect_tx(smem_addr(&full[s]), slot_bytes);
+            tma_load_2d(smem_addr(ring + (size_t)s * slot_bytes), map, x, y, smem_addr(&full[s]));
+        }
+    }
+drain:
+    for (int j = it - 1; j >= 0 && j >= it - S; --j)
+        if (!mbar_wait_bounded(smem_addr(&full[j % S]), (j / S) & 1)) record_timeout(abort_flag);
+}
+
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                               const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
+                   const __grid_constant__ GemmParams P) {
     using C = Cfg<NT>;
-    constexpr int S = C::kStages;
+    constexpr int SA = C::kSA, SB = C::kSB, SW = C::kSW;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // stages first (each 1024-aligned), then barriers and small arrays
-    uint8_t* stage_base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full_b = reinterpret_cast<uint64_t*>(stage_base + S * C::kStageBytes);
-    uint64_t* full_a = full_b + S;
-    uint64_t* empty = full_a + S;
-    uint64_t* acc_full = empty + S;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
-    float* scale_s = reinterpret_cast<float*>(tmem_slot + 4);  // [NT]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(scale_s + NT);
+    uint8_t* ringA = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ringB = ringA + (size_t)SA * C::kABytes;
+    uint8_t* ringW = ringB + (size_t)SB * C::kBBytes;
+    uint64_t* fullA = reinterpret_cast<uint64_t*>(ringW + (size_t)SW * C::kWBytes);
+    uint64_t* emptyA = fullA + SA;
+    uint64_t* fullB = emptyA + SA;
+    uint64_t* emptyB = fullB + SB;
+    uint64_t* fullW = emptyB + SB;
+    uint64_t* emptyW = fullW + SW;
+    uint64_t* accFull = emptyW + SW;  // [2]
+    uint64_t* accEmpty = accFull + 2;  // [2]
+    uint64_t* drain = accEmpty + 2;    // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     griddep_launch_dependents();  // a following PDL kernel may be scheduled; it waits for us
-    const int n0 = blockIdx.x * kRowsTile;
-    const int m0 = blockIdx.y * NT;
-    const int KB = P.kblocks;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&full_b[s]), 1);
-            mbar_init(smem_addr(&full_a[s]), kExp / 32);
-            mbar_init(smem_addr(&empty[s]), 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(smem_addr(&fullA[s]), kExpWarps);
+            mbar_init(smem_addr(&emptyA[s]), 1);
         }
-        mbar_init(smem_addr(acc_full), 1);
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(smem_addr(&fullB[s]), 1);
+            mbar_init(smem_addr(&emptyB[s]), 1);
+        }
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(smem_addr(&fullW[s]), 1);
+            mbar_init(smem_addr(&emptyW[s]), kExpWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_addr(&accFull[b]), 1);
+            mbar_init(smem_addr(&accEmpty[b]), kEpiWarps);
+        }
+        mbar_init(smem_addr(drain), 1);
         *abort_flag = 0;
     }
     fence_mbar_init();
-    if (warp == 1) {  // tensor memory for the accumulator
+    if (warp == kWarpMma) {  // tensor memory for the two accumulators
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                      "r"(C::kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
-    griddep_wait();  // x̃ and β may come from the preceding kernel
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + NT) {  // dequant scales of this tile's tokens
-        const int t = threadIdx.x - 64;
-        scale_s[t] = (m0 + t < P.M) ? dequant_scale(*P.alpha, P.beta[m0 + t]) : 0.0f;
-    }
-    if (NT > kExp && threadIdx.x >= 64) {
-        for (int t = threadIdx.x - 64 + kExp; t < NT; t += kExp)
-            scale_s[t] = (m0 + t < P.M) ? dequant_scale(*P.alpha, P.beta[m0 + t]) : 0.0f;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
 
-    if (warp == 0) {
-        // ---- x̃ tiles by TMA
+    if (warp == kWarpTmaX) {
+        // ---- x̃ tiles (written by the preceding kernel under PDL: wait for it first)
         if (lane == 0) {
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % S;
-                if (kb >= S && !mbar_wait_bounded(smem_addr(&empty[s]), ((kb / S) - 1) & 1)) {
-                    *abort_flag = 1;
-                    atomicCAS(&g_gemm_error, 0, (int)BL_ERR_TIMEOUT);
-                    break;
-                }
-                const uint32_t bar = smem_addr(&full_b[s]);
-                mbar_arrive_expect_tx(bar, C::kBBytes);
-                tma_load_2d(smem_addr(stage_base + s * C::kStageBytes + C::kABytes), &xmap, kb * kKB, m0, bar);
-            }
+            griddep_wait();
+            tma_producer<SB>(&xmap, ringB, C::kBBytes, fullB, emptyB, P, abort_flag,
+                             [&](int tile, int kb, int& x, int& y) {
+                                 x = kb * kKB;
+                                 y = (tile % P.tiles_m) * NT;
+                             });
         }
-    } else if (warp == 1) {
+    } else if (warp == kWarpTmaW) {
+        // ---- packed codes (weights are not written by a kernel this launch may overlap)
+        if (lane == 0)
+            tma_producer<SW>(&wmap, ringW, C::kWBytes, fullW, emptyW, P, abort_flag,
+                             [&](int tile, int kb, int& x, int& y) {
+                                 x = kb * kWB;
+                                 y = (tile / P.tiles_m) * kRowsTile;
+                             });
+    } else if (warp == kWarpMma) {
         // ---- MMA issue
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc_i8<NT>();
-            bool ok = true;
-            for (int kb = 0; kb < KB && ok; ++kb) {
-                const int s = kb % S;
-                ok = mbar_wait_bounded(smem_addr(&full_b[s]), (kb / S) & 1) &&
-                     mbar_wait_bounded(smem_addr(&full_a[s]), (kb / S) & 1);
-                if (!ok) break;
+            int it = 0, j = 0;
+            for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+                const int b = j & 1;
+                if (j >= 2 && !wait_or_abort(smem_addr(&accEmpty[b]), ((j >> 1) - 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a_addr = smem_addr(stage_base + s * C::kStageBytes);
-                const uint32_t b_addr = a_addr + C::kABytes;
+                const uint32_t d = tmem_d + (uint32_t)(b * NT);
+                bool ok = true;
+                for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
+                    const int sa = it % SA, sb = it % SB;
+                    ok = wait_or_abort(smem_addr(&fullA[sa]), (it / SA) & 1, abort_flag) &&
+                         wait_or_abort(smem_addr(&fullB[sb]), (it / SB) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_addr(ringA + (size_t)sa * C::kABytes);
+                    const uint32_t b_addr = smem_addr(ringB + (size_t)sb * C::kBBytes);
 #pragma unroll
-                for (int k = 0; k < kKB / 32; ++k)
-                    mma_i8(tmem_d, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k), idesc,
-                           (kb > 0 || k > 0) ? 1u : 0u);
-                mma_commit(smem_addr(&empty[s]));
+                    for (int k = 0; k < kKB / 32; ++k)
+                        mma_i8(d, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k), idesc,
+                               (kb > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(smem_addr(&emptyA[sa]));
+                    mma_commit(smem_addr(&emptyB[sb]));
+                }
+                if (!ok) break;
+                mma_commit(smem_addr(&accFull[b]));
             }
-            if (!ok) {
-                *abort_flag = 1;
-                atomicCAS(&g_gemm_error, 0, (int)BL_ERR_TIMEOUT);
+            // every MMA issued above completes before the tensor memory is freed
+            mma_commit(smem_addr(drain));
+            if (!mbar_wait_bounded(smem_addr(drain), 0)) record_timeout(abort_flag);
+        }
+    } else if (warp < kWarpEpi0) {
+        // ---- expand the codes of tile row t from ring W into ring A
+        const int t = 32 * (warp & 3) + lane;
+        const uint32_t w_off = (uint32_t)t * kWB;
+        const uint32_t a_row = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+            bool ok = true;
+            for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
+                const int sw = it % SW, sa = it % SA;
+                if (!(ok = wait_or_abort(smem_addr(&fullW[sw]), (it / SW) & 1, abort_flag))) break;
+                const uint32_t wsrc = smem_addr(ringW + (size_t)sw * C::kWBytes) + w_off;
+                const uint4 pk0 = lds128(wsrc);
+                const uint4 pk1 = lds128(wsrc + 16);
+                uint4 out[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    // weights 16q .. 16q+15 of the block: fields 0..3 of packed word q
+                    const uint32_t w = word_of(q < 4 ? pk0 : pk1, q & 3);
+                    out[q] = make_uint4(field_s8(w, 0), field_s8(w, 1), field_s8(w, 2), field_s8(w, 3));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive1(smem_addr(&emptyW[sw]));  // codes are in registers
+                if (it >= SA && !(ok = wait_or_abort(smem_addr(&emptyA[sa]), ((it / SA) - 1) & 1, abort_flag)))
+                    break;
+                uint8_t* rowp = ringA + (size_t)sa * C::kABytes + a_row;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(rowp + ((q ^ (t & 7)) << 4)) = out[q];
+                fence_proxy_async_smem();  // generic writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive1(smem_addr(&fullA[sa]));
             }
-            mma_commit(smem_addr(acc_full));  // fires once every MMA issued above has completed
+            if (!ok) break;
         }
     } else {
-        // ---- expand the weight codes of row n0 + t, then the epilogue
-        // tile row = TMEM lane; a warp may only touch lanes 32·(warp % 4) .. +31
-        const int t = 32 * (warp & 3) + lane;
-        const int row = n0 + t;
-        const bool row_ok = row < P.N;
-        const uint8_t* wrow = P.W + (int64_t)(row_ok ? row : 0) * P.row_bytes;
-        const int chunks = P.row_bytes / 16;
-        for (int kb = 0; kb < KB; ++kb) {
-            const int s = kb % S;
-            // packed codes of this K block: 2 chunks of 16 bytes (64 weights each)
-            uint4 pk[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int ch = kb * 2 + h;
-                pk[h] = (row_ok && ch < chunks) ? ld_stream16(wrow + 16 * ch)
-                                                : make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
-            }
-            if (kb >= S && !mbar_wait_bounded(smem_addr(&empty[s]), ((kb / S) - 1) & 1)) {
-                *abort_flag = 1;
-                atomicCAS(&g_gemm_error, 0, (int)BL_ERR_TIMEOUT);
-                break;
-            }
-            if (*abort_flag) break;
-            uint8_t* a_tile = stage_base + s * C::kStageBytes;
-            uint8_t* rowp = a_tile + (t >> 3) * 1024 + (t & 7) * 128;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t w = word_of(pk[h], q);  // weights 16·(4h+q) .. +15 of the block
-                    const int j = 4 * h + q;               // 16-byte chunk of the 128-byte row
-                    uint4 out;
-                    out.x = field_s8(w, 0);
-                    out.y = field_s8(w, 1);
-                    out.z = field_s8(w, 2);
-                    out.w = field_s8(w, 3);
-                    *reinterpret_cast<uint4*>(rowp + ((j ^ (t & 7)) << 4)) = out;
-                }
-            }
-            fence_proxy_async_smem();  // generic writes -> tensor-core reads
-            __syncwarp();
-            if (lane == 0) mbar_arrive1(smem_addr(&full_a[s]));
-        }
-        // ---- epilogue: row n0 + t, tokens m0 .. m0+NT-1
-        const bool done = mbar_wait_bounded(smem_addr(acc_full), 0);
-        if (!done) atomicCAS(&g_gemm_error, 0, (int)BL_ERR_TIMEOUT);
-        tc_fence_after();
-        if (done && !*abort_flag) {
-            const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-            const float b = (row_ok && P.bias) ? P.bias[row] : 0.0f;
+        // ---- epilogue: tile row t (TMEM lane; a warp may only touch lanes 32·(warp % 4) .. +31)
+        griddep_wait();  // β comes from, and y may be read by, the preceding kernel
+        const int q = warp & 3;
+        const int t = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const float alpha = *P.alpha;
+        int j = 0;
+        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+            const int b = j & 1;
+            const int m0 = (tile % P.tiles_m) * NT;
+            const int row = (tile / P.tiles_m) * kRowsTile + t;
+            const bool row_ok = row < P.N;
+            const float bias = (row_ok && P.bias) ? P.bias[row] : 0.0f;
+            if (!wait_or_abort(smem_addr(&accFull[b]), (j >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
 #pragma unroll 1
-            for (int c0 = 0; c0 < NT; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(tmem_d + lane_base + c0, r);
-                if (row_ok) {
+            for (int c0 = 0; c0 < NT; c0 += 32) {
+                // lane l holds the scale of token m0 + c0 + l; shuffled to the writers below
+                const int my_tok = m0 + c0 + lane;
+                const float my_scale = my_tok < P.M ? dequant_scale(alpha, P.beta[my_tok]) : 0.0f;
+#pragma unroll
+                for (int h = 0; h < 2 && c0 + 16 * h < NT; ++h) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c0 + 16 * h), r);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int tok = m0 + c0 + i;
-                        if (tok < P.M) {
+                        const float sc = __shfl_sync(0xffffffffu, my_scale, 16 * h + i);
+                        const int tok = m0 + c0 + 16 * h + i;
+                        if (row_ok && tok < P.M) {
                             const int acc = (int)r[i];
-                            float out = __fmul_rn((float)acc, scale_s[c0 + i]);
-                            if (P.bias) out = __fadd_rn(out, b);
+                            float out = __fmul_rn((float)acc, sc);
+                            if (P.bias) out = __fadd_rn(out, bias);
                             P.y[(int64_t)tok * P.N + row] = out;
                             if (P.acc_out) P.acc_out[(int64_t)tok * P.N + row] = acc;
                         }
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive1(smem_addr(&accEmpty[b]));
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(C::kTmemCols));
     }
@@ -315,27 +394,37 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int NT>
-size_t smem_bytes() {
-    using C = Cfg<NT>;
-    return 1024 + (size_t)C::kStages * C::kStageBytes + (3 * C::kStages + 1) * 8 + 16 + NT * 4 + 16;
+// 2-D uint8 tensor map over a row-major [rows][cols] array (row stride `cols`).
+cudaError_t encode_u8(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, uint32_t box_x, uint32_t box_y,
+                      CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)cols};
+    const cuuint32_t box[2] = {box_x, box_y};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int NT>
 cudaError_t launch_nt(const bitlinear_forward_problem& pr, cudaStream_t stream, bool pdl) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return cudaErrorNotSupported;
-    CUtensorMap map;
-    const cuuint64_t gdim[2] = {(cuuint64_t)pr.K, (cuuint64_t)pr.M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)pr.K};
-    const cuuint32_t box[2] = {(cuuint32_t)kKB, (cuuint32_t)NT};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(pr.x_q), gdim, gstride, box, estride,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    using C = Cfg<NT>;
+    // Out-of-range boxes read zeros: a zero x̃ beyond K or beyond M, and code
+    // 00 (-1) beyond a row's packed bytes or beyond N, which only ever meets a
+    // zero x̃ or lands in a row that is not stored.
+    CUtensorMap xmap, wmap;
+    cudaError_t err = encode_u8(&xmap, pr.x_q, pr.K, pr.M, kKB, NT, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (err != cudaSuccess) return err;
+    const int64_t row_bytes = (int64_t)bitlinear_packed_row_bytes(pr.K);
+    err = encode_u8(&wmap, pr.W_packed, row_bytes, pr.N, kWB, kRowsTile, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (err != cudaSuccess) return err;
+    DeviceInfo dev;
+    if ((err = device_info(&dev)) != cudaSuccess) return err;
+
     GemmParams P{};
-    P.W = pr.W_packed;
     P.alpha = pr.alpha;
     P.beta = pr.beta;
     P.bias = pr.bias;
@@ -343,34 +432,37 @@ cudaError_t launch_nt(const bitlinear_forward_problem& pr, cudaStream_t stream, 
     P.acc_out = pr.acc_out;
     P.M = (int)pr.M;
     P.N = (int)pr.N;
-    P.K = (int)pr.K;
-    P.row_bytes = (int)bitlinear_packed_row_bytes(pr.K);
     P.kblocks = (int)((pr.K + kKB - 1) / kKB);
-    const size_t smem = smem_bytes<NT>();
+    P.tiles_m = (int)((pr.M + NT - 1) / NT);
+    P.tiles = P.tiles_m * (int)((pr.N + kRowsTile - 1) / kRowsTile);
+
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [smem] {
-        attr_err = cudaFuncSetAttribute(gemm_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     });
     if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)((pr.N + kRowsTile - 1) / kRowsTile), (unsigned)((pr.M + NT - 1) / NT));
+    cfg.gridDim = dim3((unsigned)(P.tiles < dev.sm_count ? P.tiles : dev.sm_count));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<NT>, map, P);
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<NT>, xmap, wmap, P);
 }
 
 }  // namespace
 
 bool gemm_tc_supported(const bitlinear_forward_problem& p) {
-    return p.K % 16 == 0 && (reinterpret_cast<uintptr_t>(p.x_q) & 15) == 0 && p.M <= ((int64_t)1 << 30) &&
-           p.N <= ((int64_t)1 << 30) && encode_fn() != nullptr;
+    // TMA: x̃ rows (K bytes apart) and the x̃ base 16-byte aligned; tile counts in int
+    return p.K % 16 == 0 && (reinterpret_cast<uintptr_t>(p.x_q) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(p.W_packed) & 15) == 0 && p.M <= ((int64_t)1 << 30) &&
+           p.N <= ((int64_t)1 << 30) && ((p.M + 15) / 16) * ((p.N + kRowsTile - 1) / kRowsTile) < ((int64_t)1 << 31) &&
+           encode_fn() != nullptr;
 }
 
 cudaError_t launch_gemm_tc(const bitlinear_forward_problem& p, cudaStream_t stream, bool pdl) {
