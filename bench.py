@@ -22,6 +22,13 @@ HBM (the replicas together exceed 4× the L2).  Multi-GPU: one process per GPU,
 each runs its own replica of the workload (weak scaling, no data-path
 collective); the step time is the max over ranks.
 
+Prefill leg (same JSON line, key "prefill"): M = 2048 tokens through the three
+prefill shapes (K, N) = (4096, 4096), (4096, 11008), (11008, 4096), bf16 inputs
+with outliers; one step = one bitlinear_linear_grouped call over the three
+(grouped act quant + one tcgen05 int8 GEMM launch per matrix), K steps in one
+CUDA graph.  Its roofline is the GEMM's int8 TOPS (each launch timed with CUDA
+events, the three shapes rotating) against the measured bf16 tensor peak × 2.
+
 ``--impl reference`` times the CPU oracle (the method written out in plain C)
 on the host cores over a bounded row sample of the same workload.
 """
@@ -68,6 +75,11 @@ def bytes_per_step(specs) -> int:
         total += s.M * s.K * 2 + s.M * s.K + 4 * s.M   # act quant: x in, x̃ out, β out
         total += s.M * s.K + 4 * s.M + 4 * s.M * s.N   # GEMV: x̃, β in; y out
     return total
+
+
+def prefill_specs():
+    from bitlinear_w1_a8_03_b200 import workloads
+    return [workloads.prefill(4096, 4096), workloads.prefill(4096, 11008), workloads.prefill(11008, 4096)]
 
 
 def load_peaks():
@@ -337,6 +349,154 @@ def run_native(args, rank, world, local_rank):
     return result
 
 
+# ----------------------------------------------------------------------------- prefill leg
+def run_prefill(args, world, local_rank):
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    specs = prefill_specs()
+    probs, fwd = [], []
+    for s in specs:
+        W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+        p, a = bl.bitlinear_quantize_weights(W)
+        del W
+        xb = synth.f32_to_bf16_bits(synth.activations(s.x_seed, s.M, s.K, outliers=s.outliers))
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        pr = dict(x=x, x_q=torch.empty((s.M, s.K), dtype=torch.int8, device=dev),
+                  beta=torch.empty(s.M, dtype=torch.float32, device=dev), W_packed=p, alpha=a, N=s.N,
+                  y=torch.empty((s.M, s.N), dtype=torch.float32, device=dev))
+        probs.append(pr)
+    torch.cuda.synchronize()
+    ops = [2 * s.M * s.N * s.K for s in specs]
+    L = bl.lib()
+    arr = bl.make_linear_problems(probs)
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+
+    def step():
+        bl.check(L.bitlinear_linear_grouped(arr, len(specs), bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC, sh), "linear")
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    stream.synchronize()
+    K = args.steps
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(K):
+            step()
+    with torch.cuda.stream(stream):
+        g.replay()  # warm replay (W steps already ran eagerly)
+    stream.synchronize()
+    gpu_id = "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local_rank)
+    sampler = ClockSampler(gpu_id)
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    t1.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = t0.elapsed_time(t1) / K
+
+    # the GEMM alone, launch by launch (x̃ ready), the three shapes rotating so
+    # consecutive launches touch different data (together 3x the L2)
+    reps = max(5, min(50, K // 4))
+    gemm_ms = [0.0] * len(specs)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in specs]
+           for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for r in range(reps):
+            for i, (s, pr) in enumerate(zip(specs, probs)):
+                evs[r][i][0].record()
+                bl.check(L.bitlinear_forward(bl._ptr(pr["x_q"]), bl._ptr(pr["beta"]), s.M, s.K, bl._ptr(pr["W_packed"]),
+                                             bl._ptr(pr["alpha"]), s.N, None, bl._ptr(pr["y"]), None, sh), "forward")
+                evs[r][i][1].record()
+    stream.synchronize()
+    for r in range(reps):
+        for i in range(len(specs)):
+            gemm_ms[i] += evs[r][i][0].elapsed_time(evs[r][i][1]) / reps
+    # the grouped activation quantisation alone
+    aq = (bl.ActProblem * len(specs))()
+    for i, (s, pr) in enumerate(zip(specs, probs)):
+        aq[i] = bl.ActProblem(bl._ptr(pr["x"]), bl._ptr(pr["x_q"]), bl._ptr(pr["beta"]), s.M, s.K)
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            bl.check(L.bitlinear_quantize_act_grouped(aq, len(specs), bl.BL_BF16, sh), "act")
+        q0.record()
+        for _ in range(reps):
+            bl.check(L.bitlinear_quantize_act_grouped(aq, len(specs), bl.BL_BF16, sh), "act")
+        q1.record()
+    stream.synchronize()
+    clocks = sampler.stop()
+    aq_ms = q0.elapsed_time(q1) / reps
+    aq_bytes = sum(s.M * s.K * 3 + 4 * s.M for s in specs)
+
+    # context: cuBLAS int8 GEMM (torch._int_mm) on int8 operands of the same shapes
+    cublas = {}
+    try:
+        for s in specs:
+            a8 = torch.randint(-127, 128, (s.M, s.K), dtype=torch.int8, device=dev)
+            b8 = torch.randint(-1, 2, (s.N, s.K), dtype=torch.int8, device=dev).t()
+            for _ in range(3):
+                torch._int_mm(a8, b8)
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record()
+            for _ in range(10):
+                torch._int_mm(a8, b8)
+            c1.record()
+            c1.synchronize()
+            cublas[f"{s.M}x{s.K}x{s.N}"] = round(2 * s.M * s.N * s.K / (c0.elapsed_time(c1) / 10 * 1e-3) / 1e12, 1)
+            del a8, b8
+    except RuntimeError as e:  # context only
+        cublas = {"unavailable": str(e).splitlines()[0]}
+
+    peaks, peak_src = load_peaks()
+    peak = 2.0 * float(peaks["bf16_tflops"])
+    gemm_total_ms = sum(gemm_ms)
+    achieved = sum(ops) / (gemm_total_ms * 1e-3) / 1e12
+    value = world * sum(ops) / (step_ms * 1e-3) / 1e12
+    return {
+        "metric": "prefill int8 TOPS",
+        "value": round(value, 1),
+        "unit": "TOPS",
+        "ms_per_step": round(step_ms, 5),
+        "steps": K,
+        "workload": "prefill M=2048 tokens: (K,N) = (4096,4096), (4096,11008), (11008,4096); bf16 x ~ N(0,1) + 0.1% "
+                    "x20 outliers; per step grouped act quant + one tcgen05 GEMM (+dequant) per matrix",
+        "ops_per_step": sum(ops),
+        "l2": "per step the three problems hold x 79 MB, x_q 39 MB, packed W 27 MB, y 157 MB (>2x the L2)",
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "gemm_tc_kernel<256> (tcgen05.mma kind::i8, persistent, one CTA per SM)",
+            "achieved": round(achieved, 1),
+            "peak": round(peak, 1),
+            "peak_source": (f"{peak_src} bf16_tflops {peaks['bf16_tflops']} (cuBLAS bf16 burst) x 2, the nominal "
+                            "int8/bf16 dense ratio (4.5/2.25 PFLOP/s)"),
+            "unit": "TOPS",
+            "frac": round(achieved / peak, 4),
+            "traffic": recorded_traffic("gemm:prefill", "gemm_tcgen05.cu"),
+            "avg_launch_us": {f"{s.M}x{s.K}x{s.N}": round(t * 1e3, 2) for s, t in zip(specs, gemm_ms)},
+            "tops_by_shape": {f"{s.M}x{s.K}x{s.N}": round(o / (t * 1e-3) / 1e12, 1)
+                              for s, o, t in zip(specs, ops, gemm_ms)},
+        },
+        "act_quant": {"us_per_step": round(aq_ms * 1e3, 2), "GB/s": round(aq_bytes / (aq_ms * 1e-3) / 1e9, 1),
+                      "bytes_per_step": aq_bytes},
+        "cublas_int8_tops_context": cublas,
+        "gpu_launches": (1 + len(specs)) * K,
+        "clocks": clocks,
+    }
+
+
 # ----------------------------------------------------------------------------- oracle timing
 def oracle_full():
     """Oracle inputs for the same workload: α and codes from the oracle's own
@@ -445,7 +605,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--legs", default="decode,prefill",
+                    help="comma list: decode (the headline line), prefill (added under the key 'prefill')")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     args = ap.parse_args()
+    legs = [x for x in args.legs.split(",") if x]
     if args.warmup < 3:
         args.warmup = 3
 
@@ -465,9 +629,16 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    result = run_native(args, rank, world, local_rank)
+    result = run_native(args, rank, world, local_rank) if "decode" in legs else {"metric": METRIC}
+    if "prefill" in legs:
+        pre = run_prefill(args, world, local_rank)
+        result["prefill"] = pre
+        if "decode" not in legs:
+            result.update({"value": pre["value"], "unit": pre["unit"], "n_gpus": world, "steps": args.steps,
+                           "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True,
+                           "scaling": "weak", "vs_baseline": None})
     if rank == 0:
-        if world == 1:
+        if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(args)
         print(json.dumps(result), flush=True)
     if world > 1:

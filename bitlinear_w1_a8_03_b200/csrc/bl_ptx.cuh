@@ -39,8 +39,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
     return ok != 0;
 }
 
-// Waits for phase `parity` of the mbarrier to complete; false if the bound ran out.
+// Non-blocking test of phase `parity`: returns at once either way.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for phase `parity` of the mbarrier to complete; false if the bound ran
+// out.  A phase that has already completed is taken by the non-blocking test
+// (a suspending try_wait costs a few hundred cycles even then).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t polls = kPollLimit) {
+    if (mbar_test_wait(bar, parity)) return true;
     for (uint32_t i = 0; i < polls; ++i)
         if (mbar_try_wait(bar, parity, kPollSuspendNs)) return true;
     return false;

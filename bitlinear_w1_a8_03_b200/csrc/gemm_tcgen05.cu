@@ -50,14 +50,35 @@ constexpr int kWarpTmaX = 0, kWarpMma = 1, kWarpExp0 = 2, kWarpEpi0 = 6, kWarpTm
 constexpr int kExpWarps = 4, kEpiWarps = 4;
 constexpr size_t kSmemLimit = 232448;  // opt-in dynamic shared memory per block on sm_100
 
+// Ring depths (expanded codes A, x̃ tiles B, packed codes W) for the two
+// large tile widths; build-time knobs, the shared-memory budget is checked below.
+#ifndef BL_GEMM_SA_256
+#define BL_GEMM_SA_256 4
+#endif
+#ifndef BL_GEMM_SB_256
+#define BL_GEMM_SB_256 4
+#endif
+#ifndef BL_GEMM_SW_256
+#define BL_GEMM_SW_256 4
+#endif
+#ifndef BL_GEMM_SA_128
+#define BL_GEMM_SA_128 3
+#endif
+#ifndef BL_GEMM_SB_128
+#define BL_GEMM_SB_128 8
+#endif
+#ifndef BL_GEMM_SW_128
+#define BL_GEMM_SW_128 8
+#endif
+
 template <int NT>
 struct Cfg {
     static constexpr int kABytes = kRowsTile * kKB;  // 16 KiB of expanded codes
     static constexpr int kBBytes = NT * kKB;         // NT × 128 B of x̃
     static constexpr int kWBytes = kRowsTile * kWB;  // 4 KiB of packed codes
-    static constexpr int kSA = NT >= 256 ? 2 : (NT >= 128 ? 3 : 4);
-    static constexpr int kSW = NT >= 256 ? 6 : (NT >= 128 ? 8 : 16);
-    static constexpr int kSB = NT >= 256 ? 5 : (NT >= 128 ? 8 : (NT >= 64 ? 10 : 12));
+    static constexpr int kSA = NT >= 256 ? BL_GEMM_SA_256 : (NT >= 128 ? BL_GEMM_SA_128 : 4);
+    static constexpr int kSW = NT >= 256 ? BL_GEMM_SW_256 : (NT >= 128 ? BL_GEMM_SW_128 : 16);
+    static constexpr int kSB = NT >= 256 ? BL_GEMM_SB_256 : (NT >= 128 ? BL_GEMM_SB_128 : (NT >= 64 ? 10 : 12));
     static constexpr int kBars = 2 * (kSA + kSB + kSW) + 5;
     static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;  // two accumulators
     static constexpr size_t kRingBytes =
@@ -65,6 +86,7 @@ struct Cfg {
     static constexpr size_t kSmem = 1024 + kRingBytes + kBars * 8 + 16;
     static_assert(kSmem <= kSmemLimit, "shared memory budget");
     static_assert(kSmem > kSmemLimit / 2, "one CTA per SM (the tensor memory is sized for one)");
+    static_assert(kSA >= 2 && kSB >= 2, "rings of at least two slots");
 };
 
 struct GemmParams {
@@ -152,12 +174,23 @@ __device__ __forceinline__ void record_timeout(volatile int* abort_flag) {
 }
 
 // Waits for phase `parity` of `bar` unless the CTA is aborting; false (and
-// the abort recorded) if it did not complete.
+// the abort recorded) if it did not complete.  A completed phase returns at
+// once (one shared-memory access); the abort flag is read only when waiting.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (mbar_wait_bounded(bar, parity)) return true;
     record_timeout(abort_flag);
     return false;
+}
+
+// Both operands of one K block present: the two tests go out together.
+__device__ __forceinline__ bool operands_ready(uint32_t bar_a, uint32_t par_a, uint32_t bar_b, uint32_t par_b,
+                                               volatile int* abort_flag) {
+    const bool a = mbar_test_wait(bar_a, par_a);
+    const bool b = mbar_test_wait(bar_b, par_b);
+    if (a & b) return true;
+    return wait_or_abort(bar_a, par_a, abort_flag) && wait_or_abort(bar_b, par_b, abort_flag);
 }
 
 // A TMA producer's loop: one box per K block of every tile of this CTA into a
@@ -271,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
                     const int sa = it % SA, sb = it % SB;
-                    ok = wait_or_abort(smem_addr(&fullA[sa]), (it / SA) & 1, abort_flag) &&
-                         wait_or_abort(smem_addr(&fullB[sb]), (it / SB) & 1, abort_flag);
+                    ok = operands_ready(smem_addr(&fullA[sa]), (it / SA) & 1, smem_addr(&fullB[sb]), (it / SB) & 1,
+                                        abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t a_addr = smem_addr(ringA + (size_t)sa * C::kABytes);

@@ -4,10 +4,13 @@
 // β = max|x| + 1e-8, x̃ = clip(round(127·x/β), -127, 127), taken per token
 // (one row of x) as nxmr.cn/news/148658 §3.2 motivates.
 //
-// One CTA per token row.  Rows of up to kThreads·kVecPerThread 16-byte vectors
+// One CTA per token row.  Rows of up to blockDim·kVecPerThread 16-byte vectors
 // are loaded once into registers (one HBM read of x, one write of x̃); longer
 // or unaligned rows are read twice (the second read hits L1/L2).  The kernel
-// is HBM-bound: 2 (bf16) or 4 (fp32) bytes in + 1 byte out per element.
+// is HBM-bound: 2 (bf16) or 4 (fp32) bytes in + 1 byte out per element.  With
+// few rows (decode) each CTA has 512 threads so a row finishes soonest; with
+// many rows (prefill) the CTA is sized to the register buffer (kVecPerThread
+// vectors per thread), so an SM holds many rows' loads in flight at once.
 #include "bl_common.cuh"
 #include "bl_launch.h"
 #include "bl_ptx.cuh"
@@ -15,7 +18,7 @@
 namespace bl {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kMaxThreads = 512;
 constexpr int kVecPerThread = 8;
 
 struct ActParams {
@@ -25,9 +28,17 @@ struct ActParams {
     int early_trigger;  // release the next PDL kernel before waiting on the previous one
 };
 
-__device__ __forceinline__ int8_t quantize_one(float v, float beta) {
-    float t = __fdiv_rn(__fmul_rn(v, 127.0f), beta);
-    float r = rintf(t);  // round half to even
+// clip(rint(RN(RN(127·v) / β)), -127, 127), exactly.  With a = RN(127·v) and
+// |v| <= β, |a/β| <= 127·(1 + 2^-24), so q = RN(a·RN(1/β)) is within
+// 127·2^-23 < 1.6e-5 of a/β, and RN(a/β) within 127·2^-24 of it.  When q is
+// farther than 1e-4 from every half-integer, both lie on the same side of it
+// and round to the same integer; otherwise (rare, and for non-finite q) the
+// correctly rounded quotient is taken.  rbeta = RN(1/β).
+__device__ __forceinline__ int8_t quantize_one(float v, float beta, float rbeta) {
+    const float a = __fmul_rn(v, 127.0f);
+    const float q = __fmul_rn(a, rbeta);
+    float r = rintf(q);  // round half to even
+    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) r = rintf(__fdiv_rn(a, beta));
     r = fminf(fmaxf(r, -127.0f), 127.0f);
     return (int8_t)__float2int_rn(r);
 }
@@ -60,13 +71,13 @@ struct Vec<uint16_t> {
 };
 
 template <int V>
-__device__ __forceinline__ void store_codes(int8_t* q, const float* f, float beta) {
+__device__ __forceinline__ void store_codes(int8_t* q, const float* f, float beta, float rbeta) {
     uint32_t packed[V / 4];
 #pragma unroll
     for (int j = 0; j < V / 4; ++j) {
         uint32_t w = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)quantize_one(f[4 * j + b], beta) << (8 * b);
+        for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)quantize_one(f[4 * j + b], beta, rbeta) << (8 * b);
         packed[j] = w;
     }
     if constexpr (V == 4) {
@@ -76,20 +87,21 @@ __device__ __forceinline__ void store_codes(int8_t* q, const float* f, float bet
     }
 }
 
+// blockDim.x is a multiple of 32
 __device__ __forceinline__ float block_max(float mx) {
-    __shared__ float warp_max[kThreads / 32];
+    __shared__ float warp_max[kMaxThreads / 32];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = mx;
     __syncthreads();
+    const int nw = blockDim.x >> 5;
     mx = warp_max[0];
-#pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) mx = fmaxf(mx, warp_max[w]);
+    for (int w = 1; w < nw; ++w) mx = fmaxf(mx, warp_max[w]);
     return mx;
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) act_quant_kernel(const __grid_constant__ ActParams P) {
+__global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_constant__ ActParams P) {
     // Programmatic dependent launch: the product kernel that follows may start
     // and stream its weights once this kernel triggers; it waits for x̃ and β
     // itself.  By default the trigger comes after this kernel's own wait, i.e.
@@ -112,13 +124,14 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const __grid_consta
                      (K % V == 0);
 
     const int64_t nvec = K / V;
-    if (vec && nvec <= (int64_t)kThreads * kVecPerThread) {
+    const int nt = blockDim.x;
+    if (vec && nvec <= (int64_t)nt * kVecPerThread) {
         // single pass: the row stays in registers between absmax and quantise
         uint4 buf[kVecPerThread];
         float mx = 0.0f;
 #pragma unroll
         for (int j = 0; j < kVecPerThread; ++j) {
-            const int64_t i = threadIdx.x + (int64_t)j * kThreads;
+            const int64_t i = threadIdx.x + (int64_t)j * nt;
             if (i < nvec) {
                 buf[j] = ld_shared_ro16(x + i * V);
                 float f[V];
@@ -128,14 +141,15 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const __grid_consta
             }
         }
         const float beta = __fadd_rn(block_max(mx), 1e-8f);
+        const float rbeta = __frcp_rn(beta);
         if (threadIdx.x == 0) pr.beta[m] = beta;
 #pragma unroll
         for (int j = 0; j < kVecPerThread; ++j) {
-            const int64_t i = threadIdx.x + (int64_t)j * kThreads;
+            const int64_t i = threadIdx.x + (int64_t)j * nt;
             if (i < nvec) {
                 float f[V];
                 Vec<T>::unpack(buf[j], f);
-                store_codes<V>(q + i * V, f, beta);
+                store_codes<V>(q + i * V, f, beta, rbeta);
             }
         }
         return;
@@ -144,26 +158,27 @@ __global__ void __launch_bounds__(kThreads) act_quant_kernel(const __grid_consta
     // two passes: absmax, then quantise (the second read hits L1/L2)
     float mx = 0.0f;
     if (vec) {
-        for (int64_t i = (int64_t)threadIdx.x * V; i < K; i += (int64_t)kThreads * V) {
+        for (int64_t i = (int64_t)threadIdx.x * V; i < K; i += (int64_t)nt * V) {
             float f[V];
             Vec<T>::load(x + i, f);
 #pragma unroll
             for (int j = 0; j < V; ++j) mx = fmaxf(mx, fabsf(f[j]));
         }
     } else {
-        for (int64_t i = threadIdx.x; i < K; i += kThreads) mx = fmaxf(mx, fabsf(load_as_f32(x, i)));
+        for (int64_t i = threadIdx.x; i < K; i += nt) mx = fmaxf(mx, fabsf(load_as_f32(x, i)));
     }
     const float beta = __fadd_rn(block_max(mx), 1e-8f);
+    const float rbeta = __frcp_rn(beta);
     if (threadIdx.x == 0) pr.beta[m] = beta;
 
     if (vec) {
-        for (int64_t i = (int64_t)threadIdx.x * V; i < K; i += (int64_t)kThreads * V) {
+        for (int64_t i = (int64_t)threadIdx.x * V; i < K; i += (int64_t)nt * V) {
             float f[V];
             Vec<T>::load(x + i, f);
-            store_codes<V>(q + i, f, beta);
+            store_codes<V>(q + i, f, beta, rbeta);
         }
     } else {
-        for (int64_t i = threadIdx.x; i < K; i += kThreads) q[i] = quantize_one(load_as_f32(x, i), beta);
+        for (int64_t i = threadIdx.x; i < K; i += nt) q[i] = quantize_one(load_as_f32(x, i), beta, rbeta);
     }
 }
 
@@ -174,16 +189,27 @@ cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count
     ActParams P{};
     P.count = count;
     P.early_trigger = early_trigger ? 1 : 0;
-    int64_t rows = 0;
+    int64_t rows = 0, kmax = 0;
     for (int i = 0; i < count; ++i) {
         P.p[i] = problems[i];
         P.row_begin[i] = rows;
         rows += problems[i].M;
+        kmax = problems[i].K > kmax ? problems[i].K : kmax;
     }
     P.row_begin[count] = rows;
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    // many rows: kVecPerThread vectors per thread (at least 2 warps); few rows: 512 threads
+    int threads = kMaxThreads;
+    if (rows >= 2 * (int64_t)dev.sm_count) {
+        const int64_t nvec = (kmax * (dtype == BL_BF16 ? 2 : 4) + 15) / 16;
+        const int64_t want = ((nvec + kVecPerThread - 1) / kVecPerThread + 31) / 32 * 32;
+        threads = (int)(want < 64 ? 64 : (want > kMaxThreads ? kMaxThreads : want));
+    }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)rows);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+import bitlinear_w1_a8_03_b200 as bl
 import oracle
 from bitlinear_w1_a8_03_b200 import synth
 from tests.gpu_util import as_input, dev_f32, gpu_forward, gpu_quantize_weights, np_
@@ -308,3 +309,38 @@ def test_linear_right_after_weight_quantisation_without_sync():
         _, a_ref, codes = oracle.quantize_weights(Wo)
         _, _, _, y_r = oracle.forward(xo, codes, a_ref)
         assert_y_close(np_(y), y_r)
+
+
+def _near_half_integer_rows(beta_target, rows, K, seed):
+    """Rows whose max |x| is beta_target and whose other values put 127·x/β
+    next to a half-integer k + 1/2 (the rounding boundaries): a few ulps away,
+    just outside and inside a 1e-4 band, or anywhere."""
+    rng = np.random.default_rng(seed)
+    x = np.empty((rows, K), dtype=np.float32)
+    for r in range(rows):
+        k = rng.integers(-127, 127, size=K).astype(np.float64)
+        kind = rng.integers(0, 4, size=K)
+        off = np.choose(kind, [np.zeros(K), rng.choice([-1.1e-4, 1.1e-4, -0.9e-4, 0.9e-4], size=K),
+                               rng.uniform(-3e-4, 3e-4, size=K), rng.uniform(-0.5, 0.5, size=K)])
+        v = ((k + 0.5 + off) * beta_target / 127.0).astype(np.float32)
+        steps = np.where(kind == 0, rng.integers(-3, 4, size=K), 0)
+        for s in range(1, 4):
+            v = np.where(steps >= s, np.nextafter(v, np.float32(np.inf)), v)
+            v = np.where(steps <= -s, np.nextafter(v, np.float32(-np.inf)), v)
+        v[rng.integers(0, K)] = np.float32(beta_target) * (1 if r % 2 else -1)
+        x[r] = np.clip(v, -beta_target, beta_target)
+    return x
+
+
+@pytest.mark.parametrize("rows", [3, 400])
+@pytest.mark.parametrize("beta_target", [3.0, 0.7, 1e-3, 12345.678, 127.0])
+def test_act_quant_rounding_boundaries(rows, beta_target):
+    """Quotients 127·x/β next to k + 1/2 decide the int8 code: bit-exact with
+    the oracle's correctly rounded division, in few-row and many-row launches."""
+    x = _near_half_integer_rows(beta_target, rows, 1024, seed=int(beta_target * 1000) + rows)
+    for dtype in ("f32", "bf16"):
+        xd, xo = as_input(x, dtype)
+        xq, beta = bl.bitlinear_quantize_act(xd)
+        xq_r, beta_r = oracle.quantize_act(xo)
+        assert np.array_equal(np_(beta), beta_r)
+        assert np.array_equal(np_(xq), xq_r)
