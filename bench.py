@@ -497,6 +497,82 @@ def run_prefill(args, world, local_rank):
     }
 
 
+# ----------------------------------------------------------------------------- stack leg
+def run_stack(args, world, local_rank):
+    """The 32-layer 7B-shaped linear stack per decode step (M = 1 and 16)."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+    from bitlinear_w1_a8_03_b200.stack import MATRICES, LinearStack, shapes
+
+    dev = torch.device("cuda", local_rank)
+    hidden, ffn, L = 4096, 11008, 32
+    sh = shapes(hidden, ffn)
+    g = torch.Generator(device=dev)
+    layers = []
+    for l in range(L):
+        d = {}
+        for i, n in enumerate(MATRICES):
+            g.manual_seed(5000 + 7 * l + i)
+            W = torch.randn(sh[n], generator=g, device=dev) * 0.02
+            d[n] = bl.bitlinear_quantize_weights(W)
+            del W
+        layers.append(d)
+    torch.cuda.synchronize()
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    for M in (1, 16):
+        st = LinearStack(layers, hidden, ffn, M, dev)
+        st.h0.copy_(torch.from_numpy(synth.activations(5999, M, hidden, outliers=True)).to(dev))
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                st.run(stream)
+        stream.synchronize()
+        K = max(10, args.steps // 4)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for _ in range(K):
+                st.run(stream)
+        with torch.cuda.stream(stream):
+            gr.replay()
+        stream.synchronize()
+        import torch.distributed as dist
+        if world > 1:
+            dist.barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record()
+            gr.replay()
+            t1.record()
+        t1.synchronize()
+        ms = t0.elapsed_time(t1) / K
+        # per token and layer: quant(y_o + y_down) 8H in, H out; x_h read once, y_q,k,v 12H and y_gate,up
+        # 8F out; quant(y_v, y_up) 4H + 4F in, H + F out; x_v + x_up read, y_o + y_down 8H out
+        act_bytes = L * M * (36 * hidden + 14 * ffn)
+        bytes_step = st.weight_bytes + act_bytes
+        err = bl.bitlinear_device_error()
+        out[f"M{M}"] = {
+            "tokens_per_s": round(world * M / (ms * 1e-3), 1),
+            "ms_per_step": round(ms, 4),
+            "effective_GBps": round(bytes_step / (ms * 1e-3) / 1e9, 1),
+            "frac_of_hbm": round(bytes_step / (ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]), 4),
+            "bytes_per_step": bytes_step,
+            "steps": K,
+            "gpu_launches_per_step": st.launches(),
+            "device_error": err,
+        }
+        del gr, st
+    return {
+        "metric": "decode tokens/s through the 32-layer linear stack",
+        "workload": "7B-shaped stack: 32 layers x {q,k,v,o 4096->4096; gate,up 4096->11008; down 11008->4096}, "
+                    "1.62 GB packed weights (W ~ N(0,0.02) from the device generator, seed 5000+7*layer+matrix); "
+                    "per layer q,k,v,gate,up read quant(h), o reads quant(y_v), down reads quant(y_up), "
+                    "h' = y_o + y_down summed inside the next quantisation; one CUDA graph of K steps",
+        "l2": "weights 1.62 GB (13x the L2) streamed once per step",
+        **out,
+    }
+
+
 # ----------------------------------------------------------------------------- oracle timing
 def oracle_full():
     """Oracle inputs for the same workload: α and codes from the oracle's own
@@ -605,8 +681,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--legs", default="decode,prefill",
-                    help="comma list: decode (the headline line), prefill (added under the key 'prefill')")
+    ap.add_argument("--legs", default="decode,prefill,stack",
+                    help="comma list: decode (the headline line), prefill and stack (added under their keys)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     args = ap.parse_args()
     legs = [x for x in args.legs.split(",") if x]
@@ -637,6 +713,8 @@ def main():
             result.update({"value": pre["value"], "unit": pre["unit"], "n_gpus": world, "steps": args.steps,
                            "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True,
                            "scaling": "weak", "vs_baseline": None})
+    if "stack" in legs:
+        result["stack"] = run_stack(args, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(args)

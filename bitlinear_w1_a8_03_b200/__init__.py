@@ -57,6 +57,11 @@ class LinearProblem(ctypes.Structure):
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 
 
+class ActSumProblem(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("x_sum", ctypes.c_void_p), ("x_q", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("M", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
 def lib():
     """The loaded ctypes library; raises if the CUDA library was not built."""
     global _lib
@@ -79,6 +84,8 @@ def lib():
             L.bitlinear_forward_grouped.argtypes = [ctypes.POINTER(ForwardProblem), i32, p]
             L.bitlinear_linear.argtypes = [p, i32, i64, i64, p, p, i64, p, p, p, p, p, p]
             L.bitlinear_linear_grouped.argtypes = [ctypes.POINTER(LinearProblem), i32, i32, ctypes.c_uint32, p]
+            L.bitlinear_linear_block.argtypes = [ctypes.POINTER(ActSumProblem), i32, ctypes.POINTER(ForwardProblem), i32,
+                                                 ctypes.c_uint32, p]
             L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
             L.bitlinear_selftest_timeout.argtypes = [ctypes.c_uint32, p]
             L.bitlinear_status_string.argtypes = [i32]
@@ -87,7 +94,8 @@ def lib():
             for name in ("bitlinear_quantize_weights", "bitlinear_quantize_weights_static",
                          "bitlinear_quantize_act", "bitlinear_forward",
                          "bitlinear_quantize_act_grouped", "bitlinear_forward_grouped", "bitlinear_linear",
-                         "bitlinear_linear_grouped", "bitlinear_device_error", "bitlinear_selftest_timeout",
+                         "bitlinear_linear_grouped", "bitlinear_linear_block", "bitlinear_device_error",
+                         "bitlinear_selftest_timeout",
                          "bitlinear_version"):
                 getattr(L, name).restype = i32
             _lib = L
@@ -241,6 +249,28 @@ def bitlinear_linear_grouped(problems, dtype_code: int | None = None, flags: int
         dtype_code = _dtype_code(problems[0]["x"]) if dtype_code is None else dtype_code
     check(lib().bitlinear_linear_grouped(arr, len(arr), dtype_code, flags, _stream(stream)),
           "bitlinear_linear_grouped")
+
+
+def make_act_sum_problems(acts):
+    """ctypes array for bitlinear_linear_block from dicts with keys a, x_q, beta
+    and optional b (second float32 addend) and x_sum (stores a + b)."""
+    arr = (ActSumProblem * len(acts))()
+    for i, p in enumerate(acts):
+        M, K = p["a"].shape
+        arr[i] = ActSumProblem(_ptr(p["a"]), _ptr(p.get("b")), _ptr(p.get("x_sum")), _ptr(p["x_q"]), _ptr(p["beta"]),
+                               M, K)
+    return arr
+
+
+def bitlinear_linear_block(acts, fwds, flags: int = 0, stream=None):
+    """Quantise the inputs `acts` (each a, or a + b, float32) in one launch, then
+    run the products `fwds` (dicts as for make_forward_problems) in one launch.
+    Either may be empty; ctypes arrays from make_act_sum_problems /
+    make_forward_problems are passed through as they are."""
+    a_arr = acts if isinstance(acts, ctypes.Array) else (make_act_sum_problems(acts) if acts else None)
+    f_arr = fwds if isinstance(fwds, ctypes.Array) else (make_forward_problems(fwds) if fwds else None)
+    check(lib().bitlinear_linear_block(a_arr, len(acts), f_arr, len(fwds), flags, _stream(stream)),
+          "bitlinear_linear_block")
 
 
 def bitlinear_device_error() -> int:

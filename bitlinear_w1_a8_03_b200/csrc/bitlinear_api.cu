@@ -199,6 +199,44 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     return from_cuda(bl::launch_forward(fwd, count, s, true));
 }
 
+bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, int n_acts,
+                                        const bitlinear_forward_problem* fwd, int n_fwd, uint32_t flags,
+                                        bitlinear_stream_t stream) {
+    if ((n_acts > 0 && !acts) || (n_fwd > 0 && !fwd)) return BL_ERR_NULL;
+    if (n_acts < 0 || n_fwd < 0 || n_acts > BITLINEAR_MAX_GROUP || n_fwd > BITLINEAR_MAX_GROUP || n_acts + n_fwd == 0)
+        return BL_ERR_COUNT;
+    if (flags & ~(uint32_t)BL_LINEAR_WEIGHTS_STATIC) return BL_ERR_FLAGS;
+    bl::ActJob jobs[BITLINEAR_MAX_GROUP];
+    int64_t rows = 0;
+    for (int i = 0; i < n_acts; ++i) {
+        const bitlinear_act_sum_problem& p = acts[i];
+        if (!p.a || !p.x_q || !p.beta) return BL_ERR_NULL;
+        if (p.M < 1 || p.K < 1 || p.K > BITLINEAR_MAX_K || p.M > kMaxRows) return BL_ERR_SHAPE;
+        if (misaligned(p.a, 4) || misaligned(p.b, 4) || misaligned(p.x_sum, 4) || misaligned(p.beta, 4))
+            return BL_ERR_ALIGN;
+        jobs[i] = bl::ActJob{p.a, p.b, p.x_sum, p.x_q, p.beta, p.M, p.K};
+        rows += p.M;
+    }
+    if (rows >= kMaxRows) return BL_ERR_SHAPE;
+    for (int i = 0; i < n_fwd; ++i) {
+        bitlinear_status st = check_forward(fwd[i]);
+        if (st != BL_OK) return st;
+    }
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    if (n_acts > 0) {
+        st = from_cuda(bl::launch_quantize_act_jobs(jobs, n_acts, BL_F32, s, true, weights_static));
+        if (st != BL_OK) return st;
+    }
+    // The product kernel streams weights before its dependency wait: chained
+    // after this call's own quantisation kernel, or after any work when the
+    // caller vouches that nothing in flight writes the weights.
+    if (n_fwd > 0) return from_cuda(bl::launch_forward(fwd, n_fwd, s, n_acts > 0 || weights_static));
+    return BL_OK;
+}
+
 bitlinear_status bitlinear_device_error(int* code) {
     if (!code) return BL_ERR_NULL;
     bitlinear_status st = check_device();

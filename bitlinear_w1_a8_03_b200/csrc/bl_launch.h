@@ -15,10 +15,23 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// One activation-quantisation job: x = a, or a + b (float32 only) when b is
+// set; x_sum (nullable) receives x.
+struct ActJob {
+    const void* a;
+    const float* b;
+    float* x_sum;
+    int8_t* x_q;
+    float* beta;
+    int64_t M, K;
+};
+
 // pdl: launch with programmatic dependent launch (the kernel waits for its
 // predecessor before reading x); early_trigger: let the next PDL kernel start
 // before that wait (only when no work in flight writes the next kernel's
 // weights).
+cudaError_t launch_quantize_act_jobs(const ActJob* jobs, int count, bitlinear_dtype dtype, cudaStream_t stream,
+                                     bool pdl, bool early_trigger);
 cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
                                 cudaStream_t stream, bool pdl = false, bool early_trigger = false);
 

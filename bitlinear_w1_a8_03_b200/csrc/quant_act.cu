@@ -4,6 +4,10 @@
 // β = max|x| + 1e-8, x̃ = clip(round(127·x/β), -127, 127), taken per token
 // (one row of x) as nxmr.cn/news/148658 §3.2 motivates.
 //
+// Optionally the input is the float32 sum of two activations (the residual
+// addition between layers, which stays in floating point, §6.1), added
+// element-wise with one binary32 rounding and optionally stored.
+//
 // One CTA per token row.  Rows of up to blockDim·kVecPerThread 16-byte vectors
 // are loaded once into registers (one HBM read of x, one write of x̃); longer
 // or unaligned rows are read twice (the second read hits L1/L2).  The kernel
@@ -22,7 +26,7 @@ constexpr int kMaxThreads = 512;
 constexpr int kVecPerThread = 8;
 
 struct ActParams {
-    bitlinear_act_problem p[kMaxGroup];
+    ActJob p[kMaxGroup];
     int64_t row_begin[kMaxGroup + 1];
     int count;
     int early_trigger;  // release the next PDL kernel before waiting on the previous one
@@ -70,6 +74,28 @@ struct Vec<uint16_t> {
     __device__ static void load(const uint16_t* p, float* out) { unpack(ld_shared_ro16(p), out); }
 };
 
+// x (+ b) for one 16-byte vector of x; b only with float32 x.
+template <typename T>
+__device__ __forceinline__ uint4 load_sum16(const T* x, const float* b, int64_t i) {
+    uint4 v = ld_shared_ro16(x + i);
+    if constexpr (Vec<T>::n == 4) {
+        if (b) {
+            const uint4 w = ld_shared_ro16(b + i);
+            v.x = __float_as_uint(__fadd_rn(__uint_as_float(v.x), __uint_as_float(w.x)));
+            v.y = __float_as_uint(__fadd_rn(__uint_as_float(v.y), __uint_as_float(w.y)));
+            v.z = __float_as_uint(__fadd_rn(__uint_as_float(v.z), __uint_as_float(w.z)));
+            v.w = __float_as_uint(__fadd_rn(__uint_as_float(v.w), __uint_as_float(w.w)));
+        }
+    }
+    return v;
+}
+
+template <typename T>
+__device__ __forceinline__ float load_sum1(const T* x, const float* b, int64_t i) {
+    const float v = load_as_f32(x, i);
+    return b ? __fadd_rn(v, b[i]) : v;
+}
+
 template <int V>
 __device__ __forceinline__ void store_codes(int8_t* q, const float* f, float beta, float rbeta) {
     uint32_t packed[V / 4];
@@ -114,13 +140,16 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
     const int64_t row = blockIdx.x;
     int pi = 0;
     while (pi + 1 < P.count && row >= P.row_begin[pi + 1]) ++pi;
-    const bitlinear_act_problem& pr = P.p[pi];
+    const ActJob& pr = P.p[pi];
     const int64_t m = row - P.row_begin[pi];
     const int64_t K = pr.K;
-    const T* x = static_cast<const T*>(pr.x) + m * K;
+    const T* x = static_cast<const T*>(pr.a) + m * K;
+    const float* b = pr.b ? pr.b + m * K : nullptr;
+    float* xs = pr.x_sum ? pr.x_sum + m * K : nullptr;
     int8_t* q = pr.x_q + m * K;
     constexpr int V = Vec<T>::n;
     const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && ((reinterpret_cast<uintptr_t>(q) & (V - 1)) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(b) & 15) == 0) && ((reinterpret_cast<uintptr_t>(xs) & 15) == 0) &&
                      (K % V == 0);
 
     const int64_t nvec = K / V;
@@ -133,7 +162,10 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
         for (int j = 0; j < kVecPerThread; ++j) {
             const int64_t i = threadIdx.x + (int64_t)j * nt;
             if (i < nvec) {
-                buf[j] = ld_shared_ro16(x + i * V);
+                buf[j] = load_sum16(x, b, i * V);
+                if constexpr (V == 4) {  // only float32 x has a sum
+                    if (xs) *reinterpret_cast<uint4*>(xs + i * V) = buf[j];
+                }
                 float f[V];
                 Vec<T>::unpack(buf[j], f);
 #pragma unroll
@@ -160,12 +192,12 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
     if (vec) {
         for (int64_t i = (int64_t)threadIdx.x * V; i < K; i += (int64_t)nt * V) {
             float f[V];
-            Vec<T>::load(x + i, f);
+            Vec<T>::unpack(load_sum16(x, b, i), f);
 #pragma unroll
             for (int j = 0; j < V; ++j) mx = fmaxf(mx, fabsf(f[j]));
         }
     } else {
-        for (int64_t i = threadIdx.x; i < K; i += nt) mx = fmaxf(mx, fabsf(load_as_f32(x, i)));
+        for (int64_t i = threadIdx.x; i < K; i += nt) mx = fmaxf(mx, fabsf(load_sum1(x, b, i)));
     }
     const float beta = __fadd_rn(block_max(mx), 1e-8f);
     const float rbeta = __frcp_rn(beta);
@@ -173,12 +205,20 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
 
     if (vec) {
         for (int64_t i = (int64_t)threadIdx.x * V; i < K; i += (int64_t)nt * V) {
+            const uint4 v = load_sum16(x, b, i);
+            if constexpr (V == 4) {
+                if (xs) *reinterpret_cast<uint4*>(xs + i) = v;
+            }
             float f[V];
-            Vec<T>::load(x + i, f);
+            Vec<T>::unpack(v, f);
             store_codes<V>(q + i, f, beta, rbeta);
         }
     } else {
-        for (int64_t i = threadIdx.x; i < K; i += nt) q[i] = quantize_one(load_as_f32(x, i), beta, rbeta);
+        for (int64_t i = threadIdx.x; i < K; i += nt) {
+            const float v = load_sum1(x, b, i);
+            if (xs) xs[i] = v;
+            q[i] = quantize_one(v, beta, rbeta);
+        }
     }
 }
 
@@ -186,6 +226,14 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
 
 cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
                                 cudaStream_t stream, bool pdl, bool early_trigger) {
+    ActJob jobs[kMaxGroup];
+    for (int i = 0; i < count; ++i)
+        jobs[i] = ActJob{problems[i].x, nullptr, nullptr, problems[i].x_q, problems[i].beta, problems[i].M, problems[i].K};
+    return launch_quantize_act_jobs(jobs, count, dtype, stream, pdl, early_trigger);
+}
+
+cudaError_t launch_quantize_act_jobs(const ActJob* problems, int count, bitlinear_dtype dtype, cudaStream_t stream,
+                                     bool pdl, bool early_trigger) {
     ActParams P{};
     P.count = count;
     P.early_trigger = early_trigger ? 1 : 0;

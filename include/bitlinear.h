@@ -234,6 +234,37 @@ BITLINEAR_API bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_p
                                                         bitlinear_dtype dtype, uint32_t flags,
                                                         bitlinear_stream_t stream);
 
+/* One input of bitlinear_linear_block: x = a, or x = a + b added element-wise
+ * in binary32 (round to nearest) when b is not NULL — the residual addition
+ * that stays in floating point between BitLinear layers while every BitLinear
+ * input is quantised on entry ("1.58-bit 大模型极限量化实战",
+ * chenxutan.com/d/5049.html §6.1).  x is quantised exactly as by
+ * bitlinear_quantize_act into x_q [M][K] and beta [M]; x_sum (nullable,
+ * [M][K] float32) receives x itself.  a, b and x_sum are float32 [M][K]
+ * row-major, 4-byte aligned; x_q as in bitlinear_quantize_act. */
+typedef struct bitlinear_act_sum_problem {
+    const float* a;
+    const float* b;
+    float* x_sum;
+    int8_t* x_q;
+    float* beta;
+    int64_t M, K;
+} bitlinear_act_sum_problem;
+
+/* A block of linears that share quantised inputs (e.g. the q, k, v, gate and
+ * up projections of one layer all reading quant(h)): one grouped quantisation
+ * launch over the n_acts inputs, then one grouped product launch over the
+ * n_fwd problems, each reading an x_q / beta written by the first step (or
+ * any other), chained by programmatic dependent launch exactly as in
+ * bitlinear_linear_grouped.  Either count may be 0, not both; each is at most
+ * BITLINEAR_MAX_GROUP.  Both arrays are HOST arrays, reusable on return.
+ * flags: 0 or BL_LINEAR_WEIGHTS_STATIC.
+ * Errors: as bitlinear_quantize_act (per input) and bitlinear_forward (per
+ * problem), plus BL_ERR_COUNT and BL_ERR_FLAGS; nothing is launched then. */
+BITLINEAR_API bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, int n_acts,
+                                                      const bitlinear_forward_problem* fwd, int n_fwd,
+                                                      uint32_t flags, bitlinear_stream_t stream);
+
 /* Reads and clears the current device's error word, which a kernel sets when
  * one of its bounded waits expires (it then stops early and its outputs are
  * undefined).  Synchronous: call after the streams that ran the kernels have

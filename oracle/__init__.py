@@ -4,9 +4,10 @@ TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, the smoke check in
 ``__graft_entry__`` and the benchmark's CPU-baseline / reference arm may import
 this package.  It shares no code with the CUDA library and never imports it.
 
-Pinned functions (the pins live in ``tests/test_oracle_pins.py``):
-``absmean``, ``ternarize``, ``pack``, ``quantize_act``, ``ternary_matmul``,
-``dequant``, ``forward``.  No function here is "parity unpinned".
+Pinned functions (the pins live in ``tests/test_oracle_pins.py`` and, for the
+layer stack, ``tests/test_oracle_stack.py``): ``absmean``, ``ternarize``,
+``pack``, ``quantize_act``, ``ternary_matmul``, ``dequant``, ``forward``,
+``stack_layer``, ``stack_forward``.  No function here is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -175,3 +176,38 @@ def forward(x: np.ndarray, codes: np.ndarray, alpha, bias: np.ndarray | None = N
     if rc != 0:
         raise OverflowError("accumulator outside int32")
     return xq, beta, acc, y
+
+
+# ----------------------------------------------------------------------------- layer stack
+STACK_MATRICES = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+def stack_layer(h: np.ndarray, layer: dict, threads: int = 1) -> dict:
+    """One layer of the linear stack: every BitLinear input is quantised on
+    entry and the residual addition stays in float ("1.58-bit 大模型极限量化实战"
+    §6.1).  The pages give no wiring between the seven linears, so the reading
+    is: q, k, v, gate and up consume quant(h); o consumes quant(y_v); down
+    consumes quant(y_up); the next layer's input is y_o + y_down, added in
+    binary32.  `layer` maps each name in STACK_MATRICES to (codes, alpha);
+    h is float32 [M][hidden].  Returns every product's output and h_next."""
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    out = {}
+    for name in ("q", "k", "v", "gate", "up"):
+        codes, alpha = layer[name]
+        out[name] = forward(h, codes, alpha, threads=threads)[3]
+    codes, alpha = layer["o"]
+    out["o"] = forward(out["v"], codes, alpha, threads=threads)[3]
+    codes, alpha = layer["down"]
+    out["down"] = forward(out["up"], codes, alpha, threads=threads)[3]
+    out["h_next"] = np.add(out["o"], out["down"], dtype=np.float32)
+    return out
+
+
+def stack_forward(h0: np.ndarray, layers: list, threads: int = 1) -> list:
+    """stack_layer applied layer after layer from h0; returns each layer's outputs."""
+    outs, h = [], h0
+    for layer in layers:
+        o = stack_layer(h, layer, threads=threads)
+        outs.append(o)
+        h = o["h_next"]
+    return outs

@@ -115,3 +115,31 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         bl.lib()
+
+
+def test_linear_block_argument_errors(L):
+    assert ctypes.sizeof(bl.ActSumProblem) == 7 * 8
+    acts = (bl.ActSumProblem * 2)()
+    fwd = (bl.ForwardProblem * 1)()
+    blk = L.bitlinear_linear_block
+    assert blk(None, 1, None, 0, 0, None) == NULL
+    assert blk(acts, 0, None, 0, 0, None) == COUNT          # nothing to do
+    assert blk(acts, 17, None, 0, 0, None) == COUNT
+    assert blk(acts, -1, None, 0, 0, None) == COUNT
+    acts[0] = bl.ActSumProblem(P, P, None, P, P, 1, 64)
+    assert blk(acts, 1, None, 0, 2, None) == FLAGS
+    acts[0] = bl.ActSumProblem(None, P, None, P, P, 1, 64)
+    assert blk(acts, 1, None, 0, 0, None) == NULL
+    acts[0] = bl.ActSumProblem(P, P, None, None, P, 1, 64)
+    assert blk(acts, 1, None, 0, 0, None) == NULL
+    acts[0] = bl.ActSumProblem(P, P, None, P, P, 0, 64)
+    assert blk(acts, 1, None, 0, 0, None) == SHAPE
+    acts[0] = bl.ActSumProblem(P + 2, P, None, P, P, 1, 64)
+    assert blk(acts, 1, None, 0, 0, None) == ALIGN
+    acts[0] = bl.ActSumProblem(P, P + 2, None, P, P, 1, 64)
+    assert blk(acts, 1, None, 0, 0, None) == ALIGN
+    acts[0] = bl.ActSumProblem(P, None, P + 1, P, P, 1, 64)
+    assert blk(acts, 1, None, 0, 0, None) == ALIGN
+    acts[0] = bl.ActSumProblem(P, None, None, P, P, 1, 64)
+    assert blk(acts, 1, fwd, 1, 0, None) == NULL             # forward problem left empty
+    assert blk(None, 0, fwd, 1, 0, None) == NULL
