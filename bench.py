@@ -51,6 +51,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMV HBM GB/s (% of 8 TB/s); prefill int8 TOPS (% of peak)"
+GEMV_SOURCES = ("gemv_ternary.cu", "bl_ptx.cuh", "bl_common.cuh")
+GEMM_SOURCES = ("gemm_tcgen05.cu", "bl_ptx.cuh", "bl_common.cuh")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -91,15 +93,24 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def recorded_traffic(kernel_tag: str, source: str):
+def kernel_sources_sha256(sources) -> str | None:
+    """sha256 over the kernel's source file and the device headers it includes,
+    in the order given (the key a recorded ncu traffic figure is valid for)."""
+    m = hashlib.sha256()
+    for name in sources:
+        src = os.path.join(ROOT, "bitlinear_w1_a8_03_b200", "csrc", name)
+        if not os.path.exists(src):
+            return None
+        m.update(open(src, "rb").read())
+    return m.hexdigest()
+
+
+def recorded_traffic(kernel_tag: str, sources):
     """DRAM bytes per launch recorded from an ncu capture in profiles/, valid
-    only while the kernel source is unchanged (sha256 recorded beside it)."""
-    src = os.path.join(ROOT, "bitlinear_w1_a8_03_b200", "csrc", source)
-    if not os.path.exists(src):
-        return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    only while the kernel's sources are unchanged (sha256 recorded beside it)."""
+    sha = kernel_sources_sha256(sources)
     pdir = os.path.join(ROOT, "profiles")
-    if not os.path.isdir(pdir):
+    if sha is None or not os.path.isdir(pdir):
         return None
     pat = re.compile(rf"^traffic\[{re.escape(kernel_tag)}\]:\s*(\d+)\s+bytes/launch\s+source_sha256:\s*([0-9a-f]+)", re.M)
     for name in sorted(os.listdir(pdir)):
@@ -109,6 +120,24 @@ def recorded_traffic(kernel_tag: str, source: str):
             if m.group(2) == sha:
                 return int(m.group(1))
     return None
+
+
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(values, device, world: int):
+    """Element-wise max of per-rank timings (ms) over all ranks; identity at N=1."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def replica_throughput(units_per_rank: float, max_ms: float, world: int) -> float:
+    """Whole-job units per second: every rank runs its own replica of the same
+    work (weak scaling), timed as the slowest rank."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -282,14 +311,11 @@ def run_native(args, rank, world, local_rank):
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev, world)
 
     bps = bytes_per_step(specs)
-    value = world * bps * K / (elapsed_ms * 1e-3) / 1e9
-    e2e_value = world * bps * K / (e2e_ms * 1e-3) / 1e9
+    value = replica_throughput(bps * K, elapsed_ms, world) / 1e9
+    e2e_value = replica_throughput(bps * K, e2e_ms, world) / 1e9
     # the GEMV and the quantisation of one step overlap (PDL) and consecutive
     # steps overlap too, so the kernel's share of a step is the step: the
     # per-launch duration is the timed region over K (an upper bound)
@@ -297,7 +323,7 @@ def run_native(args, rank, world, local_rank):
     achieved = bps / (kavg * 1e-3) / 1e9
     peaks, peak_src = load_peaks()
     peak = float(peaks["hbm_gbs"])
-    traffic = recorded_traffic("linear_pair:decode7b", "gemv_ternary.cu")
+    traffic = recorded_traffic("gemv_stream:decode7b", GEMV_SOURCES)
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -405,7 +431,7 @@ def run_prefill(args, world, local_rank):
     t1.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms = t0.elapsed_time(t1) / K
+    step_ms = max_over_ranks([t0.elapsed_time(t1) / K], dev, world)[0]
 
     # the GEMM alone, launch by launch (x̃ ready), the three shapes rotating so
     # consecutive launches touch different data (together 3x the L2)
@@ -484,7 +510,7 @@ def run_prefill(args, world, local_rank):
                             "int8/bf16 dense ratio (4.5/2.25 PFLOP/s)"),
             "unit": "TOPS",
             "frac": round(achieved / peak, 4),
-            "traffic": recorded_traffic("gemm:prefill", "gemm_tcgen05.cu"),
+            "traffic": recorded_traffic("gemm_tc:prefill_2048x4096x11008", GEMM_SOURCES),
             "avg_launch_us": {f"{s.M}x{s.K}x{s.N}": round(t * 1e3, 2) for s, t in zip(specs, gemm_ms)},
             "tops_by_shape": {f"{s.M}x{s.K}x{s.N}": round(o / (t * 1e-3) / 1e12, 1)
                               for s, o, t in zip(specs, ops, gemm_ms)},
@@ -545,7 +571,7 @@ def run_stack(args, world, local_rank):
             gr.replay()
             t1.record()
         t1.synchronize()
-        ms = t0.elapsed_time(t1) / K
+        ms = max_over_ranks([t0.elapsed_time(t1) / K], dev, world)[0]
         # per token and layer: quant(y_o + y_down) 8H in, H out; x_h read once, y_q,k,v 12H and y_gate,up
         # 8F out; quant(y_v, y_up) 4H + 4F in, H + F out; x_v + x_up read, y_o + y_down 8H out
         act_bytes = L * M * (36 * hidden + 14 * ffn)
