@@ -194,7 +194,14 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     bitlinear_status st = check_device();
     if (st != BL_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    st = from_cuda(bl::launch_quantize_act(act, count, dtype, s, true, (flags & BL_LINEAR_WEIGHTS_STATIC) != 0));
+    const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    // few tokens: one launch that quantises in the product kernel's prologue
+    bl::FusedInput fin[BITLINEAR_MAX_GROUP];
+    for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
+    bool launched = false;
+    st = from_cuda(bl::launch_linear_fused(fwd, fin, count, dtype, s, weights_static, &launched));
+    if (st != BL_OK || launched) return st;
+    st = from_cuda(bl::launch_quantize_act(act, count, dtype, s, true, weights_static));
     if (st != BL_OK) return st;
     return from_cuda(bl::launch_forward(fwd, count, s, true));
 }
@@ -226,6 +233,32 @@ bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, i
     if (st != BL_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    // Fused single launch when every product reads one of this call's inputs
+    // and every input feeds a product: each product quantises its input in its
+    // prologue; the first product of each input writes that input's outputs.
+    if (n_acts > 0 && n_fwd > 0) {
+        bl::FusedInput fin[BITLINEAR_MAX_GROUP];
+        bool used[BITLINEAR_MAX_GROUP] = {};
+        bool ok = true;
+        for (int i = 0; i < n_fwd && ok; ++i) {
+            int j = 0;
+            while (j < n_acts && !(acts[j].x_q == fwd[i].x_q && acts[j].beta == fwd[i].beta && acts[j].M == fwd[i].M &&
+                                   acts[j].K == fwd[i].K))
+                ++j;
+            if (j == n_acts) {
+                ok = false;
+                break;
+            }
+            fin[i] = bl::FusedInput{acts[j].a, acts[j].b, used[j] ? nullptr : acts[j].x_sum, !used[j]};
+            used[j] = true;
+        }
+        for (int j = 0; j < n_acts && ok; ++j) ok = used[j];
+        if (ok) {
+            bool launched = false;
+            st = from_cuda(bl::launch_linear_fused(fwd, fin, n_fwd, BL_F32, s, weights_static, &launched));
+            if (st != BL_OK || launched) return st;
+        }
+    }
     if (n_acts > 0) {
         st = from_cuda(bl::launch_quantize_act_jobs(jobs, n_acts, BL_F32, s, true, weights_static));
         if (st != BL_OK) return st;

@@ -66,4 +66,20 @@ __device__ __forceinline__ float dequant_scale(float alpha, float beta) {
     return __double2float_rn(s);
 }
 
+// clip(rint(RN(RN(127·v) / β)), -127, 127), exactly (the per-token int8
+// quantisation of "1.58-bit 大模型极限量化实战" §2.4).  With a = RN(127·v) and
+// |v| <= β, |a/β| <= 127·(1 + 2^-24), so q = RN(a·RN(1/β)) is within
+// 127·2^-23 < 1.6e-5 of a/β, and RN(a/β) within 127·2^-24 of it.  When q is
+// farther than 1e-4 from every half-integer, both lie on the same side of it
+// and round to the same integer; otherwise (rare, and for non-finite q) the
+// correctly rounded quotient is taken.  rbeta = RN(1/β).
+__device__ __forceinline__ int8_t quantize_one(float v, float beta, float rbeta) {
+    const float a = __fmul_rn(v, 127.0f);
+    const float q = __fmul_rn(a, rbeta);
+    float r = rintf(q);  // round half to even
+    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) r = rintf(__fdiv_rn(a, beta));
+    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    return (int8_t)__float2int_rn(r);
+}
+
 }  // namespace bl

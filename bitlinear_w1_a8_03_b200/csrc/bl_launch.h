@@ -49,6 +49,21 @@ cudaError_t launch_quantize_weights_static(const void* W, bitlinear_dtype dtype,
 // stream starts before the dependency wait).
 cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl);
 
+// Fused linear for at most four tokens: the streaming GEMV quantises its own
+// activations (x, or x + x2 in float32) into shared memory, so the pair of
+// kernels becomes one launch.  One entry per problem; x_sum (nullable) and the
+// problem's x_q / beta receive x, x̃ and β when write_outputs is set.
+struct FusedInput {
+    const void* x;
+    const float* x2;
+    float* x_sum;
+    bool write_outputs;
+};
+// *launched = false (and nothing enqueued) when the problems do not fit the
+// fused kernel; the caller then runs the quantisation and product separately.
+cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
+                                bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched);
+
 // Tensor-core GEMM for many tokens (tcgen05, int8): one problem per launch.
 bool gemm_tc_supported(const bitlinear_forward_problem& p);
 cudaError_t launch_gemm_tc(const bitlinear_forward_problem& p, cudaStream_t stream, bool pdl);

@@ -31,6 +31,10 @@
 // before griddepcontrol.wait (programmatic dependent launch).
 #include <mutex>
 
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+
 #include "bl_common.cuh"
 #include "bl_launch.h"
 #include "bl_ptx.cuh"
@@ -53,10 +57,14 @@ constexpr int kWarps = BL_GEMV_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = BL_GEMV_STAGES;         // private stages per warp
 constexpr int kRG = 8;                          // rows per row group
-constexpr int kSegChunks = 64;                  // 16-byte chunks per row per segment
+#ifndef BL_GEMV_SEG_CHUNKS
+#define BL_GEMV_SEG_CHUNKS 64
+#endif
+constexpr int kSegChunks = BL_GEMV_SEG_CHUNKS;  // 16-byte chunks per row per segment (multiple of 32)
 constexpr int kIt = kSegChunks / 32;            // chunks per lane per row per segment
 constexpr int kRowStride = kSegChunks * 16;     // bytes per staged row
-constexpr int kStageBytes = kRG * kRowStride;   // 8 KiB
+constexpr int kStageBytes = kRG * kRowStride;   // 8 KiB at 64 chunks
+static_assert(kSegChunks % 32 == 0, "whole chunks per lane");
 constexpr int kSlots = kWarps;                  // row groups shared between warps
 constexpr int kMaxMT = 4;
 constexpr int kGemvMaxTokens = 4;  // more tokens go to the tensor-core GEMM
@@ -76,13 +84,24 @@ struct SProblem {
     int32_t rgn;          // row groups of kRG rows
     int32_t tgn;          // token groups of MT tokens
     int64_t unit_begin;   // first unit (token group, row group, chunk) of this problem
+    // fused quantisation (x̃ made in shared memory from x, see below):
+    const void* x;        // activations, float32 or bfloat16 [M][K]
+    const float* x2;      // nullable float32 second addend
+    float* x_sum;         // nullable: stores x (+ x2)
+    int32_t write_outputs;  // the owner CTA writes x̃ to xq and β to beta (and x_sum)
 };
 
 struct SParams {
     SProblem p[kMaxGroup];
     int count;
     int64_t total_units;
+    int x_bf16;         // fused: activation dtype
+    int32_t slot_row;   // fused: bytes per token row of a shared x̃ slot (64·ceil(K/64) of the widest problem)
 };
+
+// Fused quantisation keeps two problems' x̃ (up to kMaxMT token rows each) in
+// shared memory after SharedLayout.
+constexpr int kFuseSlotBytes = 45056;
 
 struct SharedLayout {
     alignas(128) uint8_t stage[kWarps][kStages][kStageBytes];
@@ -90,6 +109,8 @@ struct SharedLayout {
     int64_t bound[kWarps + 1];  // warp unit ranges inside the CTA
     int slot_acc[kSlots][kRG * kMaxMT];
     int slot_count[kSlots];
+    float xbeta[2][kMaxMT];  // fused: β of each slot's tokens
+    float red[kWarps];       // fused: block reduction scratch
 };
 
 // Position in the unit sequence: problem, (token group, row group), chunk.
@@ -132,7 +153,7 @@ __device__ __forceinline__ void cursor_advance(const SParams& P, Cursor& cur, in
 }
 
 // Start of the row group containing unit t, rounded to the nearer boundary.
-__device__ int64_t snap_to_row_group(const SParams& P, int64_t t) {
+__host__ __device__ int64_t snap_to_row_group(const SParams& P, int64_t t) {
     if (t >= P.total_units) return P.total_units;
     int p = 0;
     while (p + 1 < P.count && t >= P.p[p + 1].unit_begin) ++p;
@@ -176,6 +197,159 @@ __device__ __forceinline__ void load_act_chunk(const int8_t* xrow, int K, int ch
 #pragma unroll
         for (int q = 0; q < 16; ++q) a[q] = 0u;
     }
+}
+
+// Shared x̃ slot layout: the four 16-byte pieces of 64-byte chunk c are
+// rotated by (c >> 1), so the 16-byte reads of 8 lanes on consecutive chunks
+// fall in distinct banks.
+__device__ __forceinline__ uint32_t xs_offset(int k) {
+    const int c = k >> 6, v = (k >> 4) & 3;
+    return (uint32_t)(64 * c + 16 * ((v + (c >> 1)) & 3) + (k & 15));
+}
+
+__device__ __forceinline__ void lds_act_chunk(uint32_t row, int chunk, uint32_t (&a)[16]) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const uint4 u = lds128(row + 64 * chunk + 16 * ((v + (chunk >> 1)) & 3));
+        a[4 * v + 0] = u.x;
+        a[4 * v + 1] = u.y;
+        a[4 * v + 2] = u.z;
+        a[4 * v + 3] = u.w;
+    }
+}
+
+__device__ __forceinline__ float block_max_fused(float mx, float* red) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    __syncthreads();  // red[] free from any previous use
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = red[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, red[w]);
+    return mx;
+}
+
+// 16 bytes of x (+ x2) as binary32 values: 8 bfloat16 or 4 float32 elements.
+template <typename T>
+struct FusedVec;
+template <>
+struct FusedVec<uint16_t> {
+    static constexpr int n = 8;
+    __device__ static void load(const SProblem& pr, int64_t e, float (&f)[8]) {
+        const uint4 u = ld_shared_ro16(static_cast<const uint16_t*>(pr.x) + e);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <>
+struct FusedVec<float> {
+    static constexpr int n = 4;
+    __device__ static void load(const SProblem& pr, int64_t e, float (&f)[4]) {
+        const uint4 u = ld_shared_ro16(static_cast<const float*>(pr.x) + e);
+        f[0] = __uint_as_float(u.x);
+        f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z);
+        f[3] = __uint_as_float(u.w);
+        if (pr.x2) {
+            const uint4 v = ld_shared_ro16(pr.x2 + e);
+            f[0] = __fadd_rn(f[0], __uint_as_float(v.x));
+            f[1] = __fadd_rn(f[1], __uint_as_float(v.y));
+            f[2] = __fadd_rn(f[2], __uint_as_float(v.z));
+            f[3] = __fadd_rn(f[3], __uint_as_float(v.w));
+        }
+    }
+};
+
+constexpr int kFuseVec = 8;  // 16-byte vectors per thread held in registers
+
+// Quantises V consecutive values into the slot (and, for the owner, global).
+template <int V>
+__device__ __forceinline__ void fused_store(const SProblem& pr, const float (&f)[V], int64_t base, int k,
+                                            uint8_t* dst_row, float beta, float rbeta, bool out) {
+    uint32_t w[V / 4];
+#pragma unroll
+    for (int j = 0; j < V / 4; ++j) {
+        uint32_t x = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) x |= (uint32_t)(uint8_t)quantize_one(f[4 * j + b], beta, rbeta) << (8 * b);
+        w[j] = x;
+    }
+#pragma unroll
+    for (int j = 0; j < V / 4; ++j) *reinterpret_cast<uint32_t*>(dst_row + xs_offset(k + 4 * j)) = w[j];
+    if (out) {
+        int8_t* q = const_cast<int8_t*>(pr.xq) + base + k;
+        if constexpr (V == 8)
+            *reinterpret_cast<uint2*>(q) = make_uint2(w[0], w[1]);
+        else
+            *reinterpret_cast<uint32_t*>(q) = w[0];
+        if (pr.x_sum) {
+#pragma unroll
+            for (int j = 0; j < V; ++j) pr.x_sum[base + k + j] = f[j];
+        }
+    }
+}
+
+// Per-token quantisation of one activation row into a shared slot row (the
+// same arithmetic as act_quant_kernel: β = max|x| + 1e-8, x̃ = quantize_one),
+// zero past K.  Rows of up to kThreads·kFuseVec vectors are read once into
+// registers; longer rows are read twice.  The owner also writes x̃, β (and x)
+// to global memory.  K is a multiple of 16 and x, x2 are 16-byte aligned.
+template <typename T>
+__device__ void fused_quantize_row(const SProblem& pr, int m, uint8_t* dst_row, int32_t row_bytes, float* beta_slot,
+                                   float* red, bool owner) {
+    constexpr int V = FusedVec<T>::n;
+    const int64_t base = (int64_t)m * pr.K;
+    const int nvec = pr.K / V;
+    const bool out = owner && pr.write_outputs;
+    float mx = 0.0f;
+    if (nvec <= kThreads * kFuseVec) {
+        float f[kFuseVec][V];
+#pragma unroll
+        for (int j = 0; j < kFuseVec; ++j) {
+            const int i = threadIdx.x + j * kThreads;
+            if (i < nvec) {
+                FusedVec<T>::load(pr, base + (int64_t)i * V, f[j]);
+#pragma unroll
+                for (int e = 0; e < V; ++e) mx = fmaxf(mx, fabsf(f[j][e]));
+            }
+        }
+        const float beta = __fadd_rn(block_max_fused(mx, red), 1e-8f);
+        const float rbeta = __frcp_rn(beta);
+#pragma unroll
+        for (int j = 0; j < kFuseVec; ++j) {
+            const int i = threadIdx.x + j * kThreads;
+            if (i < nvec) fused_store<V>(pr, f[j], base, i * V, dst_row, beta, rbeta, out);
+        }
+        if (threadIdx.x == 0) {
+            *beta_slot = beta;
+            if (out) const_cast<float*>(pr.beta)[m] = beta;
+        }
+    } else {
+        for (int i = threadIdx.x; i < nvec; i += kThreads) {
+            float f[V];
+            FusedVec<T>::load(pr, base + (int64_t)i * V, f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) mx = fmaxf(mx, fabsf(f[e]));
+        }
+        const float beta = __fadd_rn(block_max_fused(mx, red), 1e-8f);
+        const float rbeta = __frcp_rn(beta);
+        for (int i = threadIdx.x; i < nvec; i += kThreads) {
+            float f[V];
+            FusedVec<T>::load(pr, base + (int64_t)i * V, f);
+            fused_store<V>(pr, f, base, i * V, dst_row, beta, rbeta, out);
+        }
+        if (threadIdx.x == 0) {
+            *beta_slot = beta;
+            if (out) const_cast<float*>(pr.beta)[m] = beta;
+        }
+    }
+    for (int k = pr.K + 4 * threadIdx.x; k < row_bytes; k += 4 * kThreads)
+        *reinterpret_cast<uint32_t*>(dst_row + xs_offset(k)) = 0u;
 }
 
 // Issues the bulk copies of one segment (rows of one row group, chunks
@@ -227,7 +401,7 @@ __device__ __forceinline__ int lane_token(int lane) {
     return idx / kRG;
 }
 
-template <int MT>
+template <int MT, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_constant__ SParams P) {
     constexpr bool kMask = MT <= 2;  // one accumulator per code field (no shifts)
     constexpr int NS = kMask ? 4 : 1;
@@ -268,6 +442,43 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
         cursor_advance(P, prod, n);
     }
     griddep_wait();  // x̃, β (and α) may come from the preceding kernels
+
+    // ---- fused quantisation: x̃ of the (at most two) problems of this CTA
+    int p_first = 0;
+    int second_slot = 1;  // slot of the CTA's second problem (0 when it shares the first one's input)
+    uint32_t xs_base = 0;
+    if constexpr (FUSE) {
+        uint8_t* xs = smem_raw + sizeof(SharedLayout);
+        xs_base = smem_addr(xs);
+        Cursor c0, c1;
+        cursor_seek(P, c0, a, b);
+        cursor_seek(P, c1, b > a ? b - 1 : a, b);
+        p_first = c0.p;
+        for (int slot = 0; slot < 2 && a < b; ++slot) {
+            const int p = p_first + slot;
+            if (p > c1.p) break;
+            const SProblem& pr = P.p[p];
+            const bool owner = a <= pr.unit_begin && pr.unit_begin < b;
+            if (slot == 1) {
+                const SProblem& p0 = P.p[p_first];
+                if (pr.x == p0.x && pr.x2 == p0.x2 && pr.K == p0.K && pr.M == p0.M) {
+                    // same input as slot 0: reuse it (the owner still publishes x̃, β)
+                    second_slot = 0;
+                    if (owner && pr.write_outputs && (pr.xq != p0.xq || pr.beta != p0.beta || pr.x_sum != p0.x_sum))
+                        second_slot = 1;  // distinct output buffers: quantise again to write them
+                    if (second_slot == 0) break;
+                }
+            }
+            for (int m = 0; m < pr.M && m < MT; ++m) {
+                uint8_t* row = xs + (slot * MT + m) * P.slot_row;
+                if (P.x_bf16)
+                    fused_quantize_row<uint16_t>(pr, m, row, P.slot_row, &S.xbeta[slot][m], S.red, owner);
+                else
+                    fused_quantize_row<float>(pr, m, row, P.slot_row, &S.xbeta[slot][m], S.red, owner);
+            }
+        }
+        __syncthreads();
+    }
 
     // ---- main loop over this warp's segments
     Cursor cons;
@@ -311,7 +522,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
         if (scale_p != cons.p || scale_tg != tg) {  // start the α, β loads early
             const int tok = m0 + my_tok;
             alpha_v = *pr.alpha;
-            beta_v = tok < pr.M ? pr.beta[tok] : 0.0f;
+            if constexpr (FUSE)
+                beta_v = tok < pr.M ? S.xbeta[cons.p == p_first ? 0 : second_slot][tok] : 0.0f;
+            else
+                beta_v = tok < pr.M ? pr.beta[tok] : 0.0f;
         }
 
         // This segment's activations do not depend on the stage: load them
@@ -322,8 +536,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
 #pragma unroll
             for (int it = 0; it < kIt; ++it) {
                 const int chunk = cons.c + it * 32 + lane;
-                load_act_chunk(pr.xq + (int64_t)m0 * pr.K, pr.K, chunk, chunk < pr.full_chunks,
-                               it * 32 + lane < n && m0 < pr.M, pre[it]);
+                if constexpr (FUSE) {
+                    if (it * 32 + lane < n) {
+                        lds_act_chunk(xs_base + (uint32_t)((cons.p == p_first ? 0 : second_slot) * MT) * P.slot_row, chunk, pre[it]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) pre[it][q] = 0u;
+                    }
+                } else {
+                    load_act_chunk(pr.xq + (int64_t)m0 * pr.K, pr.K, chunk, chunk < pr.full_chunks,
+                                   it * 32 + lane < n && m0 < pr.M, pre[it]);
+                }
             }
         }
 
@@ -347,6 +570,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
                     if constexpr (kPreload) {
 #pragma unroll
                         for (int q = 0; q < 16; ++q) av[m][q] = pre[it][q];
+                    } else if constexpr (FUSE) {
+                        if (m0 + m < pr.M) {
+                            lds_act_chunk(xs_base + (uint32_t)((cons.p == p_first ? 0 : second_slot) * MT + m) * P.slot_row, chunk,
+                                          av[m]);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) av[m][q] = 0u;
+                        }
                     } else {
                         load_act_chunk(pr.xq + (int64_t)(m0 + m) * pr.K, pr.K, chunk, chunk < pr.full_chunks,
                                        m0 + m < pr.M, av[m]);
@@ -531,9 +762,20 @@ __global__ void wait_timeout_selftest_kernel(uint32_t polls) {
     if (!ok && threadIdx.x == 0) atomicCAS(&g_device_error, 0, (int)BL_ERR_TIMEOUT);
 }
 
+int problem_of(const SParams& P, int64_t u) {
+    int p = 0;
+    while (p + 1 < P.count && u >= P.p[p + 1].unit_begin) ++p;
+    return p;
+}
+
+// launches the streaming kernel; with `fused` (one entry per problem) the
+// kernel quantises x itself, if every CTA's range meets at most two problems
+// and a slot holds the widest row (else *launched = false and nothing runs)
 template <int MT>
 cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
-                          cudaStream_t stream, bool pdl) {
+                          cudaStream_t stream, bool pdl, const FusedInput* fused = nullptr, bool x_bf16 = false,
+                          bool* launched = nullptr, bool fuse_always = false) {
+    if (launched) *launched = true;
     SParams P{};
     P.count = count;
     int64_t total = 0, row_groups = 0;
@@ -560,26 +802,73 @@ cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, 
         row_groups += (int64_t)q.tgn * q.rgn;
     }
     P.total_units = total;
+    int64_t grid = dev.sm_count;
+    if (grid > row_groups) grid = row_groups;
+    size_t smem = sizeof(SharedLayout);
+    if (fused) {
+        int32_t slot_row = 0;
+        for (int i = 0; i < count; ++i) {
+            SProblem& q = P.p[i];
+            if (q.M > MT) {
+                *launched = false;
+                return cudaSuccess;
+            }
+            q.x = fused[i].x;
+            q.x2 = fused[i].x2;
+            q.x_sum = fused[i].x_sum;
+            q.write_outputs = fused[i].write_outputs ? 1 : 0;
+            slot_row = std::max(slot_row, 64 * q.C);
+        }
+        P.x_bf16 = x_bf16 ? 1 : 0;
+        P.slot_row = slot_row;
+        bool fits = (int64_t)MT * slot_row <= kFuseSlotBytes;
+        // Every CTA reads its problems' whole input rows before its main loop;
+        // that pays off only while those reads are small next to the weights.
+        int64_t prologue_bytes = 0, weight_bytes = 0;
+        for (int i = 0; i < count; ++i) weight_bytes += (int64_t)P.p[i].N * P.p[i].row_bytes;
+        auto input_bytes = [&](const SProblem& q) {
+            return (int64_t)q.M * q.K * (x_bf16 ? 2 : 4) * (q.x2 ? 2 : 1);
+        };
+        for (int64_t c = 0; c < grid && fits; ++c) {
+            const int64_t a = snap_to_row_group(P, (total * c) / grid);
+            const int64_t b = snap_to_row_group(P, (total * (c + 1)) / grid);
+            if (a >= b) continue;
+            const int pa = problem_of(P, a), pb = problem_of(P, b - 1);
+            fits = pb - pa <= 1;
+            prologue_bytes += input_bytes(P.p[pa]);
+            if (pb != pa && !(P.p[pb].x == P.p[pa].x && P.p[pb].x2 == P.p[pa].x2)) prologue_bytes += input_bytes(P.p[pb]);
+        }
+        if (!fuse_always && 8 * prologue_bytes > weight_bytes) fits = false;
+        if (!fits) {
+            *launched = false;
+            return cudaSuccess;
+        }
+        smem += (size_t)2 * MT * slot_row;
+    }
+    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, true>)
+                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, false>);
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<MT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)sizeof(SharedLayout));
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gemv_stream_kernel<MT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)(sizeof(SharedLayout) + 2 * kFuseSlotBytes));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    int64_t grid = dev.sm_count;
-    if (grid > row_groups) grid = row_groups;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = sizeof(SharedLayout);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MT>, P);
+    void* args[] = {&P};
+    return cudaLaunchKernelExC(&cfg, kernel, args);
 }
 
 cudaError_t launch_generic(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
@@ -643,6 +932,34 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
     if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl);
     if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl);
     return launch_stream<4>(problems, count, dev, stream, pdl);
+}
+
+cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
+                                bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched) {
+    *launched = false;
+    // BITLINEAR_LINEAR_FUSION=off never fuses, =on fuses whenever the
+    // problems fit the kernel (skipping the byte-ratio rule); default: auto
+    const char* mode = std::getenv("BITLINEAR_LINEAR_FUSION");
+    if (mode && std::strcmp(mode, "off") == 0) return cudaSuccess;
+    const bool always = mode && std::strcmp(mode, "on") == 0;
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    int64_t max_m = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_forward_problem& s = problems[i];
+        if (s.K % 16 != 0 || (reinterpret_cast<uintptr_t>(s.x_q) & 15) != 0) return cudaSuccess;
+        // the fused prologue reads x (and x2) in 16-byte vectors
+        if ((reinterpret_cast<uintptr_t>(in[i].x) & 15) != 0 || (reinterpret_cast<uintptr_t>(in[i].x2) & 15) != 0)
+            return cudaSuccess;
+        if (((s.M + 3) / 4) * ((s.N + kRG - 1) / kRG) >= ((int64_t)1 << 30)) return cudaSuccess;
+        if (s.M > max_m) max_m = s.M;
+    }
+    const bool bf16 = dtype == BL_BF16;
+    if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl, in, bf16, launched, always);
+    if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl, in, bf16, launched, always);
+    if (max_m <= 4) return launch_stream<4>(problems, count, dev, stream, pdl, in, bf16, launched, always);
+    return cudaSuccess;
 }
 
 cudaError_t read_device_error(int* code) {

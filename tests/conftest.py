@@ -31,3 +31,12 @@ def read_golden(name: str) -> dict:
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+@pytest.fixture(params=["on", "off", "auto"])
+def fusion(request, monkeypatch):
+    """Runs a test with the few-token fused linear (the product kernel
+    quantising its own input) forced on, off, or chosen by the library
+    (BITLINEAR_LINEAR_FUSION, read on every call)."""
+    monkeypatch.setenv("BITLINEAR_LINEAR_FUSION", request.param)
+    return request.param

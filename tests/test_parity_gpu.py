@@ -344,3 +344,76 @@ def test_act_quant_rounding_boundaries(rows, beta_target):
         xq_r, beta_r = oracle.quantize_act(xo)
         assert np.array_equal(np_(beta), beta_r)
         assert np.array_equal(np_(xq), xq_r)
+
+
+def _grouped_linear_case(shapes, M, dtype, seed, flags=0):
+    """Grouped linear over `shapes` [(K, N)] at M tokens: x̃, β, acc and y of
+    every problem bit-exact against the oracle."""
+    probs, refs = [], []
+    for i, (K, N) in enumerate(shapes):
+        W = synth.weights(seed + 17 * i, N, K, 0.02)
+        x = synth.activations(seed + 17 * i + 1, M, K, outliers=True)
+        packed, alpha, codes, a_ref = check_weights(W, "f32")
+        xd, xo = as_input(x, dtype)
+        pr = dict(x=xd, x_q=torch.empty((M, K), dtype=torch.int8, device="cuda"),
+                  beta=torch.empty(M, dtype=torch.float32, device="cuda"), W_packed=packed, alpha=alpha, N=N,
+                  y=torch.empty((M, N), dtype=torch.float32, device="cuda"),
+                  acc_out=torch.empty((M, N), dtype=torch.int32, device="cuda"))
+        probs.append(pr)
+        refs.append(oracle.forward(xo, codes, a_ref))
+    bl.bitlinear_linear_grouped(probs, flags=flags)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    for pr, (xq_r, beta_r, acc_r, y_r) in zip(probs, refs):
+        assert np.array_equal(np_(pr["x_q"]), xq_r)
+        assert np.array_equal(np_(pr["beta"]), beta_r)
+        assert np.array_equal(np_(pr["acc_out"]), acc_r)
+        assert_y_close(np_(pr["y"]), y_r)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fused_linear_grouped(M, dtype, fusion):
+    """Few tokens: the product kernel quantises x itself (one launch) when
+    fused; the same results either way."""
+    # 11008-wide float32 rows take the prologue's two-pass branch
+    _grouped_linear_case([(4096, 300), (1024, 700), (4096 + 64, 129), (11008, 200)], M, dtype, seed=9100 + M)
+
+
+def test_linear_grouped_many_small_problems(fusion):
+    """Sixteen tiny problems: some CTA ranges meet more than two problems, so
+    even forced fusion falls back to the separate quantisation kernel."""
+    _grouped_linear_case([(256 + 64 * (i % 3), 24 + 8 * i) for i in range(16)], 1, "bf16", seed=9200)
+
+
+def test_linear_rows_wider_than_a_fused_slot(fusion):
+    """Two tokens of a 28672-wide row exceed the fused slot: separate kernels."""
+    _grouped_linear_case([(28672, 96)], 2, "bf16", seed=9300, flags=1)
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_linear_block_fused_and_not(M, fusion):
+    """bitlinear_linear_block with shared and summed inputs (x = a + b), the
+    stack's first call shape, against the oracle."""
+    K, N = 1024, [512, 256, 768]
+    a = synth.activations(9400 + M, M, K, outliers=True)
+    b = synth.activations(9500 + M, M, K, outliers=False)
+    x = (a + b).astype(np.float32)
+    xs = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    beta = torch.empty(M, dtype=torch.float32, device="cuda")
+    fwds, refs = [], []
+    for i, n in enumerate(N):
+        W = synth.weights(9600 + i, n, K, 0.02)
+        packed, alpha, codes, a_ref = check_weights(W, "f32")
+        fwds.append(dict(x_q=xq, beta=beta, W_packed=packed, alpha=alpha, N=n,
+                         y=torch.empty((M, n), dtype=torch.float32, device="cuda")))
+        refs.append(oracle.forward(x, codes, a_ref))
+    bl.bitlinear_linear_block([dict(a=dev_f32(a), b=dev_f32(b), x_sum=xs, x_q=xq, beta=beta)], fwds,
+                              flags=bl.BL_LINEAR_WEIGHTS_STATIC)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    assert np.array_equal(np_(xs), x)
+    assert np.array_equal(np_(xq), refs[0][0]) and np.array_equal(np_(beta), refs[0][1])
+    for f, (_, _, _, y_r) in zip(fwds, refs):
+        assert_y_close(np_(f["y"]), y_r)

@@ -59,9 +59,9 @@ def _check(hidden, ffn, L, M, base_seed):
 
 
 @pytest.mark.parametrize("M", [1, 3, 16])
-def test_small_stack_bitexact(M):
-    """Three layers at hidden 256 / FFN 512: GEMV path (1, 3 tokens) and
-    tensor-core path (16 tokens)."""
+def test_small_stack_bitexact(M, fusion):
+    """Three layers at hidden 256 / FFN 512: GEMV path (1, 3 tokens, fused or
+    not) and tensor-core path (16 tokens)."""
     _check(256, 512, 3, M, base_seed=5100 + M)
 
 
