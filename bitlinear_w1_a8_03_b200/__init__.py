@@ -17,6 +17,7 @@ import threading
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+LIB_PATH = os.environ.get("BITLINEAR_LIB", LIB_PATH)  # a build elsewhere (same ABI)
 MAX_GROUP = 16
 MAX_K = 1 << 20
 

@@ -64,9 +64,9 @@ struct FusedInput {
 cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
                                 bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched);
 
-// Tensor-core GEMM for many tokens (tcgen05, int8): one problem per launch.
+// Tensor-core GEMM for many tokens (tcgen05, int8): all problems in one launch.
 bool gemm_tc_supported(const bitlinear_forward_problem& p);
-cudaError_t launch_gemm_tc(const bitlinear_forward_problem& p, cudaStream_t stream, bool pdl);
+cudaError_t launch_gemm_tc(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl);
 cudaError_t read_gemm_error(int* code);
 
 // Device-side error word (bounded waits that expired): read and clear.

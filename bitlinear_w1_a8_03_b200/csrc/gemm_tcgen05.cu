@@ -29,6 +29,7 @@
 // (bounded) and the tensor memory is freed.
 #include <cuda.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "bl_common.cuh"
@@ -89,7 +90,7 @@ struct Cfg {
     static_assert(kSA >= 2 && kSB >= 2, "rings of at least two slots");
 };
 
-struct GemmParams {
+struct GemmProblem {
     const float* alpha;
     const float* beta;
     const float* bias;
@@ -97,8 +98,31 @@ struct GemmParams {
     int32_t* acc_out;
     int M, N;
     int kblocks;
-    int tiles_m, tiles;
+    int tiles_m;     // token tiles
+    int tile_begin;  // first tile of this problem in the launch
 };
+
+// Several independent problems in one persistent launch: tiles are numbered
+// problem after problem and dealt round-robin to the CTAs.
+struct GemmParams {
+    CUtensorMap xmap[kMaxGroup];  // x̃ [M][K] of each problem
+    CUtensorMap wmap[kMaxGroup];  // packed codes [N][row bytes] of each problem
+    GemmProblem p[kMaxGroup];
+    int count;
+    int tiles;
+};
+
+struct TileRef {
+    int p, m0, n0, kblocks;
+};
+
+template <int NT>
+__device__ __forceinline__ TileRef locate(const GemmParams& P, int tile) {
+    int p = 0;
+    while (p + 1 < P.count && tile >= P.p[p + 1].tile_begin) ++p;
+    const int local = tile - P.p[p].tile_begin;
+    return TileRef{p, (local % P.p[p].tiles_m) * NT, (local / P.p[p].tiles_m) * kRowsTile, P.p[p].kblocks};
+}
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(
@@ -197,16 +221,17 @@ __device__ __forceinline__ bool operands_ready(uint32_t bar_a, uint32_t par_a, u
 // ring of S slots, each reused once the consumer frees it.  On the way out it
 // waits (bounded) for the copies it issued, so no copy lands after the CTA
 // has exited.
-template <int S, typename Coord>
-__device__ void tma_producer(const CUtensorMap* map, uint8_t* ring, uint32_t slot_bytes, uint64_t* full,
-                             uint64_t* empty, const GemmParams& P, volatile int* abort_flag, Coord coord) {
+template <int NT, int S, typename Coord>
+__device__ void tma_producer(uint8_t* ring, uint32_t slot_bytes, uint64_t* full, uint64_t* empty,
+                             const GemmParams& P, volatile int* abort_flag, Coord coord) {
     int it = 0;
     for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
-        for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
+        const TileRef tr = locate<NT>(P, tile);
+        for (int kb = 0; kb < tr.kblocks; ++kb, ++it) {
             const int s = it % S;
             if (it >= S && !wait_or_abort(smem_addr(&empty[s]), ((it / S) - 1) & 1, abort_flag)) goto drain;
             int x, y;
-            coord(tile, kb, x, y);
+            const CUtensorMap* map = coord(tr, kb, x, y);
             mbar_arrive_expect_tx(smem_addr(&full[s]), slot_bytes);
             tma_load_2d(smem_addr(ring + (size_t)s * slot_bytes), map, x, y, smem_addr(&full[s]));
         }
@@ -217,9 +242,7 @@ drain:
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
-                   const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
     using C = Cfg<NT>;
     constexpr int SA = C::kSA, SB = C::kSB, SW = C::kSW;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -277,32 +300,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- x̃ tiles (written by the preceding kernel under PDL: wait for it first)
         if (lane == 0) {
             griddep_wait();
-            tma_producer<SB>(&xmap, ringB, C::kBBytes, fullB, emptyB, P, abort_flag,
-                             [&](int tile, int kb, int& x, int& y) {
-                                 x = kb * kKB;
-                                 y = (tile % P.tiles_m) * NT;
-                             });
+            tma_producer<NT, SB>(ringB, C::kBBytes, fullB, emptyB, P, abort_flag,
+                                 [&](const TileRef& tr, int kb, int& x, int& y) {
+                                     x = kb * kKB;
+                                     y = tr.m0;
+                                     return &P.xmap[tr.p];
+                                 });
         }
     } else if (warp == kWarpTmaW) {
         // ---- packed codes (weights are not written by a kernel this launch may overlap)
         if (lane == 0)
-            tma_producer<SW>(&wmap, ringW, C::kWBytes, fullW, emptyW, P, abort_flag,
-                             [&](int tile, int kb, int& x, int& y) {
-                                 x = kb * kWB;
-                                 y = (tile / P.tiles_m) * kRowsTile;
-                             });
+            tma_producer<NT, SW>(ringW, C::kWBytes, fullW, emptyW, P, abort_flag,
+                                 [&](const TileRef& tr, int kb, int& x, int& y) {
+                                     x = kb * kWB;
+                                     y = tr.n0;
+                                     return &P.wmap[tr.p];
+                                 });
     } else if (warp == kWarpMma) {
         // ---- MMA issue
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc_i8<NT>();
             int it = 0, j = 0;
             for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+                const int kblocks = locate<NT>(P, tile).kblocks;
                 const int b = j & 1;
                 if (j >= 2 && !wait_or_abort(smem_addr(&accEmpty[b]), ((j >> 1) - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_d + (uint32_t)(b * NT);
                 bool ok = true;
-                for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int sa = it % SA, sb = it % SB;
                     ok = operands_ready(smem_addr(&fullA[sa]), (it / SA) & 1, smem_addr(&fullB[sb]), (it / SB) & 1,
                                         abort_flag);
@@ -331,8 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_row = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128);
         int it = 0;
         for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+            const int kblocks = locate<NT>(P, tile).kblocks;
             bool ok = true;
-            for (int kb = 0; kb < P.kblocks; ++kb, ++it) {
+            for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 const int sw = it % SW, sa = it % SA;
                 if (!(ok = wait_or_abort(smem_addr(&fullW[sw]), (it / SW) & 1, abort_flag))) break;
                 const uint32_t wsrc = smem_addr(ringW + (size_t)sw * C::kWBytes) + w_off;
@@ -364,21 +391,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         const int t = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const float alpha = *P.alpha;
         int j = 0;
         for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+            const TileRef tr = locate<NT>(P, tile);
+            // this tile's problem, copied out of the parameter block once
+            // (dynamically indexed parameter reads inside the store loop are slow)
+            const int M = P.p[tr.p].M, N = P.p[tr.p].N;
+            const float* beta_p = P.p[tr.p].beta;
+            const float* bias_p = P.p[tr.p].bias;
+            float* y = P.p[tr.p].y;
+            int32_t* acc_out = P.p[tr.p].acc_out;
+            const float alpha = *P.p[tr.p].alpha;
             const int b = j & 1;
-            const int m0 = (tile % P.tiles_m) * NT;
-            const int row = (tile / P.tiles_m) * kRowsTile + t;
-            const bool row_ok = row < P.N;
-            const float bias = (row_ok && P.bias) ? P.bias[row] : 0.0f;
+            const int m0 = tr.m0;
+            const int row = tr.n0 + t;
+            const bool row_ok = row < N;
+            const float bias = (row_ok && bias_p) ? bias_p[row] : 0.0f;
             if (!wait_or_abort(smem_addr(&accFull[b]), (j >> 1) & 1, abort_flag)) break;
             tc_fence_after();
 #pragma unroll 1
             for (int c0 = 0; c0 < NT; c0 += 32) {
                 // lane l holds the scale of token m0 + c0 + l; shuffled to the writers below
                 const int my_tok = m0 + c0 + lane;
-                const float my_scale = my_tok < P.M ? dequant_scale(alpha, P.beta[my_tok]) : 0.0f;
+                const float my_scale = my_tok < M ? dequant_scale(alpha, beta_p[my_tok]) : 0.0f;
 #pragma unroll
                 for (int h = 0; h < 2 && c0 + 16 * h < NT; ++h) {
                     uint32_t r[16];
@@ -387,12 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 16; ++i) {
                         const float sc = __shfl_sync(0xffffffffu, my_scale, 16 * h + i);
                         const int tok = m0 + c0 + 16 * h + i;
-                        if (row_ok && tok < P.M) {
+                        if (row_ok && tok < M) {
                             const int acc = (int)r[i];
                             float out = __fmul_rn((float)acc, sc);
-                            if (P.bias) out = __fadd_rn(out, bias);
-                            P.y[(int64_t)tok * P.N + row] = out;
-                            if (P.acc_out) P.acc_out[(int64_t)tok * P.N + row] = acc;
+                            if (bias_p) out = __fadd_rn(out, bias);
+                            y[(int64_t)tok * N + row] = out;
+                            if (acc_out) acc_out[(int64_t)tok * N + row] = acc;
                         }
                     }
                 }
@@ -443,31 +478,45 @@ cudaError_t encode_u8(CUtensorMap* map, const void* base, int64_t cols, int64_t 
 }
 
 template <int NT>
-cudaError_t launch_nt(const bitlinear_forward_problem& pr, cudaStream_t stream, bool pdl) {
+cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl) {
     using C = Cfg<NT>;
-    // Out-of-range boxes read zeros: a zero x̃ beyond K or beyond M, and code
-    // 00 (-1) beyond a row's packed bytes or beyond N, which only ever meets a
-    // zero x̃ or lands in a row that is not stored.
-    CUtensorMap xmap, wmap;
-    cudaError_t err = encode_u8(&xmap, pr.x_q, pr.K, pr.M, kKB, NT, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (err != cudaSuccess) return err;
-    const int64_t row_bytes = (int64_t)bitlinear_packed_row_bytes(pr.K);
-    err = encode_u8(&wmap, pr.W_packed, row_bytes, pr.N, kWB, kRowsTile, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (err != cudaSuccess) return err;
     DeviceInfo dev;
-    if ((err = device_info(&dev)) != cudaSuccess) return err;
-
-    GemmParams P{};
-    P.alpha = pr.alpha;
-    P.beta = pr.beta;
-    P.bias = pr.bias;
-    P.y = pr.y;
-    P.acc_out = pr.acc_out;
-    P.M = (int)pr.M;
-    P.N = (int)pr.N;
-    P.kblocks = (int)((pr.K + kKB - 1) / kKB);
-    P.tiles_m = (int)((pr.M + NT - 1) / NT);
-    P.tiles = P.tiles_m * (int)((pr.N + kRowsTile - 1) / kRowsTile);
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    // params are large (two tensor maps per problem): build them off the stack
+    static thread_local GemmParams P;
+    P = GemmParams{};
+    P.count = count;
+    // Tiles are numbered longest K first, so the round-robin deal hands out
+    // the long tiles early and the short ones even out the end.
+    int order[kMaxGroup];
+    for (int i = 0; i < count; ++i) order[i] = i;
+    std::stable_sort(order, order + count, [&](int a, int b) { return problems[a].K > problems[b].K; });
+    int tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_forward_problem& pr = problems[order[i]];
+        // Out-of-range boxes read zeros: a zero x̃ beyond K or beyond M, and
+        // code 00 (-1) beyond a row's packed bytes or beyond N, which only
+        // ever meets a zero x̃ or lands in a row that is not stored.
+        err = encode_u8(&P.xmap[i], pr.x_q, pr.K, pr.M, kKB, NT, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (err != cudaSuccess) return err;
+        const int64_t row_bytes = (int64_t)bitlinear_packed_row_bytes(pr.K);
+        err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, kWB, kRowsTile, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (err != cudaSuccess) return err;
+        GemmProblem& q = P.p[i];
+        q.alpha = pr.alpha;
+        q.beta = pr.beta;
+        q.bias = pr.bias;
+        q.y = pr.y;
+        q.acc_out = pr.acc_out;
+        q.M = (int)pr.M;
+        q.N = (int)pr.N;
+        q.kblocks = (int)((pr.K + kKB - 1) / kKB);
+        q.tiles_m = (int)((pr.M + NT - 1) / NT);
+        q.tile_begin = tiles;
+        tiles += q.tiles_m * (int)((pr.N + kRowsTile - 1) / kRowsTile);
+    }
+    P.tiles = tiles;
 
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -476,7 +525,7 @@ cudaError_t launch_nt(const bitlinear_forward_problem& pr, cudaStream_t stream, 
     });
     if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)(P.tiles < dev.sm_count ? P.tiles : dev.sm_count));
+    cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = stream;
@@ -485,7 +534,7 @@ cudaError_t launch_nt(const bitlinear_forward_problem& pr, cudaStream_t stream, 
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<NT>, xmap, wmap, P);
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<NT>, P);
 }
 
 }  // namespace
@@ -494,16 +543,22 @@ bool gemm_tc_supported(const bitlinear_forward_problem& p) {
     // TMA: x̃ rows (K bytes apart) and the x̃ base 16-byte aligned; tile counts in int
     return p.K % 16 == 0 && (reinterpret_cast<uintptr_t>(p.x_q) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(p.W_packed) & 15) == 0 && p.M <= ((int64_t)1 << 30) &&
-           p.N <= ((int64_t)1 << 30) && ((p.M + 15) / 16) * ((p.N + kRowsTile - 1) / kRowsTile) < ((int64_t)1 << 31) &&
+           p.N <= ((int64_t)1 << 30) && ((p.M + 15) / 16) * ((p.N + kRowsTile - 1) / kRowsTile) < ((int64_t)1 << 26) &&
            encode_fn() != nullptr;
 }
 
-cudaError_t launch_gemm_tc(const bitlinear_forward_problem& p, cudaStream_t stream, bool pdl) {
-    if (p.M <= 16) return launch_nt<16>(p, stream, pdl);
-    if (p.M <= 32) return launch_nt<32>(p, stream, pdl);
-    if (p.M <= 64) return launch_nt<64>(p, stream, pdl);
-    if (p.M <= 128) return launch_nt<128>(p, stream, pdl);
-    return launch_nt<256>(p, stream, pdl);
+cudaError_t launch_gemm_tc(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl) {
+    int64_t max_m = 0, tiles16 = 0;
+    for (int i = 0; i < count; ++i) {
+        max_m = problems[i].M > max_m ? problems[i].M : max_m;
+        tiles16 += ((problems[i].M + 15) / 16) * ((problems[i].N + kRowsTile - 1) / kRowsTile);
+    }
+    if (tiles16 >= ((int64_t)1 << 30)) return cudaErrorInvalidValue;  // tile numbers are int
+    if (max_m <= 16) return launch_nt<16>(problems, count, stream, pdl);
+    if (max_m <= 32) return launch_nt<32>(problems, count, stream, pdl);
+    if (max_m <= 64) return launch_nt<64>(problems, count, stream, pdl);
+    if (max_m <= 128) return launch_nt<128>(problems, count, stream, pdl);
+    return launch_nt<256>(problems, count, stream, pdl);
 }
 
 cudaError_t read_gemm_error(int* code) {

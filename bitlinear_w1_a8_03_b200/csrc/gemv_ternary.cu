@@ -918,16 +918,10 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
     }
     if (!fast) return launch_generic(problems, count, dev, stream);
     if (max_m > kGemvMaxTokens) {
-        // many tokens: the int8 tensor cores, one launch per problem
+        // many tokens: the int8 tensor cores, all problems in one launch
         bool tc = true;
         for (int i = 0; i < count; ++i) tc = tc && gemm_tc_supported(problems[i]);
-        if (tc) {
-            for (int i = 0; i < count; ++i) {
-                err = launch_gemm_tc(problems[i], stream, pdl && i == 0);
-                if (err != cudaSuccess) return err;
-            }
-            return cudaSuccess;
-        }
+        if (tc) return launch_gemm_tc(problems, count, stream, pdl);
     }
     if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl);
     if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl);

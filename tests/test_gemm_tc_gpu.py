@@ -47,3 +47,30 @@ def test_gemm_ragged_k_and_rows(K, N):
 def test_gemm_prefill_shape_small_rows():
     """2048 tokens (the prefill token count) on a few hundred rows."""
     run_case(2048, 1024, 256, seed=800, dtype="f32")
+
+
+@pytest.mark.parametrize("M", [16, 37, 300])
+def test_gemm_grouped_problems(M):
+    """Several problems of different K and N in one tensor-core launch."""
+    shapes = [(256, 200), (1024, 384), (4096 + 64, 130), (128, 16)]
+    probs, refs = [], []
+    for i, (K, N) in enumerate(shapes):
+        W = synth.weights(7000 + 13 * i + M, N, K, 0.02)
+        x = synth.activations(7100 + 13 * i + M, M, K, outliers=True)
+        Wd, Wo = as_input(W, "f32")
+        packed, alpha = bl.bitlinear_quantize_weights(Wd)
+        p_ref, a_ref, codes = oracle.quantize_weights(Wo)
+        xd, xo = as_input(x, "bf16")
+        xq, beta = bl.bitlinear_quantize_act(xd)
+        pr = dict(x_q=xq, beta=beta, W_packed=packed, alpha=alpha, N=N,
+                  y=torch.empty((M, N), dtype=torch.float32, device="cuda"),
+                  acc_out=torch.empty((M, N), dtype=torch.int32, device="cuda"))
+        probs.append(pr)
+        refs.append(oracle.forward(xo, codes, a_ref, threads=8))
+    bl.bitlinear_forward_grouped(probs)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    for pr, (xq_r, beta_r, acc_r, y_r) in zip(probs, refs):
+        assert np.array_equal(np_(pr["acc_out"]), acc_r)
+        err = np.abs(np_(pr["y"]).astype(np.float64) - y_r)
+        assert np.all(err <= 1e-5 * np.abs(y_r) + 1e-37)
