@@ -347,9 +347,8 @@ def run_native(args, rank, world, local_rank):
     bps = bytes_per_step(specs)
     value = replica_throughput(bps * K, elapsed_ms, world) / 1e9
     e2e_value = replica_throughput(bps * K, e2e_ms, world) / 1e9
-    # the GEMV and the quantisation of one step overlap (PDL) and consecutive
-    # steps overlap too, so the kernel's share of a step is the step: the
-    # per-launch duration is the timed region over K (an upper bound)
+    # one launch per step (the fused GEMV; consecutive steps overlap by PDL),
+    # so the per-launch duration is the timed region over K (an upper bound)
     kavg = elapsed_ms / K
     achieved = bps / (kavg * 1e-3) / 1e9
     peaks, peak_src = load_peaks()
@@ -375,14 +374,14 @@ def run_native(args, rank, world, local_rank):
             "l2": f"inputs larger than L2: {replicas} rotating weight replicas, {replicas * set_bytes / 1e6:.0f} MB "
                   f"(L2 {props.L2_cache_size / 1e6:.0f} MB)",
             "launch": "K steps captured in one CUDA graph; per step one bitlinear_linear_grouped call "
-                      "(BL_LINEAR_WEIGHTS_STATIC) = grouped act-quant kernel + grouped GEMV kernel, chained by PDL",
+                      "(BL_LINEAR_WEIGHTS_STATIC) = one fused quantise + GEMV launch, steps chained by PDL",
             "parallelism": f"replicas x{world}",
             "pct_of_8TBps": round(100 * value / world / 8000.0, 2),
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "act_quant_kernel + gemv_stream_kernel<1> (one bitlinear_linear_grouped call over the 7 "
-                      "matrices; the GEMV overlaps the quantisation by programmatic dependent launch)",
+            "kernel": "gemv_stream_kernel<1, fused> (one bitlinear_linear_grouped call over the 7 matrices = one "
+                      "launch that quantises its inputs in its prologue; consecutive steps chained by PDL)",
             "achieved": round(achieved, 2),
             "peak": peak,
             "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json copy bandwidth)" if peak_src == "measured"
@@ -401,7 +400,7 @@ def run_native(args, rank, world, local_rank):
             "how": "public binding per step: pinned x -> device, bitlinear_linear_grouped, y -> pinned host; "
                    "double-buffered on two copy streams so copies overlap the neighbouring steps' kernels",
         },
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clocks,
     }
     return result
@@ -465,9 +464,21 @@ def run_prefill(args, world, local_rank):
         dist.barrier()
     step_ms = max_over_ranks([t0.elapsed_time(t1) / K], dev, world)[0]
 
-    # the GEMM alone, launch by launch (x̃ ready), the three shapes rotating so
-    # consecutive launches touch different data (together 3x the L2)
+    # the product alone: one grouped tcgen05 launch over the three matrices
+    # (x̃ ready), as in the step; and each shape on its own for context
     reps = max(5, min(50, K // 4))
+    fwd_arr = bl.make_forward_problems([dict(x_q=pr["x_q"], beta=pr["beta"], W_packed=pr["W_packed"],
+                                             alpha=pr["alpha"], N=pr["N"], y=pr["y"]) for pr in probs])
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            bl.check(L.bitlinear_forward_grouped(fwd_arr, len(specs), sh), "forward_grouped")
+        g0.record()
+        for _ in range(reps):
+            bl.check(L.bitlinear_forward_grouped(fwd_arr, len(specs), sh), "forward_grouped")
+        g1.record()
+    stream.synchronize()
+    grouped_ms = g0.elapsed_time(g1) / reps
     gemm_ms = [0.0] * len(specs)
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in specs]
            for _ in range(reps)]
@@ -499,6 +510,29 @@ def run_prefill(args, world, local_rank):
     aq_ms = q0.elapsed_time(q1) / reps
     aq_bytes = sum(s.M * s.K * 3 + 4 * s.M for s in specs)
 
+    # the one-off weight quantisation (absmean + ternarise + pack) of the
+    # prefill matrices, fp32 W: algorithmic bytes = 2 reads of W + packed write
+    wq_bytes, wq_ms = 0, 0.0
+    for s in specs:
+        W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+        ws = torch.empty(L.bitlinear_quantize_weights_workspace_bytes(s.N, s.K), dtype=torch.uint8, device=dev)
+        pk = torch.empty((s.N, int(L.bitlinear_packed_row_bytes(s.K))), dtype=torch.uint8, device=dev)
+        al = torch.empty(1, dtype=torch.float32, device=dev)
+        def wq():
+            bl.check(L.bitlinear_quantize_weights(bl._ptr(W), bl.BL_F32, s.N, s.K, bl._ptr(pk), bl._ptr(al),
+                                                  bl._ptr(ws), ws.numel(), sh), "quantize_weights")
+        with torch.cuda.stream(stream):
+            wq()
+            w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            w0.record()
+            for _ in range(5):
+                wq()
+            w1.record()
+        w1.synchronize()
+        wq_ms += w0.elapsed_time(w1) / 5
+        wq_bytes += 2 * s.N * s.K * 4 + pk.numel()
+        del W, ws, pk
+
     # context: cuBLAS int8 GEMM (torch._int_mm) on int8 operands of the same shapes
     cublas = {}
     try:
@@ -520,8 +554,7 @@ def run_prefill(args, world, local_rank):
 
     peaks, peak_src = load_peaks()
     peak = 2.0 * float(peaks["bf16_tflops"])
-    gemm_total_ms = sum(gemm_ms)
-    achieved = sum(ops) / (gemm_total_ms * 1e-3) / 1e12
+    achieved = sum(ops) / (grouped_ms * 1e-3) / 1e12
     value = world * sum(ops) / (step_ms * 1e-3) / 1e12
     return {
         "metric": "prefill int8 TOPS",
@@ -535,22 +568,27 @@ def run_prefill(args, world, local_rank):
         "l2": "per step the three problems hold x 79 MB, x_q 39 MB, packed W 27 MB, y 157 MB (>2x the L2)",
         "roofline": {
             "bound": "tensor",
-            "kernel": "gemm_tc_kernel<256> (tcgen05.mma kind::i8, persistent, one CTA per SM)",
+            "kernel": "gemm_tc_kernel<256> (tcgen05.mma kind::i8, persistent, one CTA per SM), one grouped launch "
+                      "over the three matrices",
             "achieved": round(achieved, 1),
             "peak": round(peak, 1),
             "peak_source": (f"{peak_src} bf16_tflops {peaks['bf16_tflops']} (cuBLAS bf16 burst) x 2, the nominal "
                             "int8/bf16 dense ratio (4.5/2.25 PFLOP/s)"),
             "unit": "TOPS",
             "frac": round(achieved / peak, 4),
-            "traffic": recorded_traffic("gemm_tc:prefill_2048x4096x11008", GEMM_SOURCES),
-            "avg_launch_us": {f"{s.M}x{s.K}x{s.N}": round(t * 1e3, 2) for s, t in zip(specs, gemm_ms)},
+            "traffic": recorded_traffic("gemm_tc:prefill_grouped", GEMM_SOURCES),
+            "avg_launch_us": round(grouped_ms * 1e3, 2),
+            "single_launch_us": {f"{s.M}x{s.K}x{s.N}": round(t * 1e3, 2) for s, t in zip(specs, gemm_ms)},
             "tops_by_shape": {f"{s.M}x{s.K}x{s.N}": round(o / (t * 1e-3) / 1e12, 1)
                               for s, o, t in zip(specs, ops, gemm_ms)},
         },
         "act_quant": {"us_per_step": round(aq_ms * 1e3, 2), "GB/s": round(aq_bytes / (aq_ms * 1e-3) / 1e9, 1),
                       "bytes_per_step": aq_bytes},
+        "weight_quant": {"us_for_3_matrices": round(wq_ms * 1e3, 1), "GB/s": round(wq_bytes / (wq_ms * 1e-3) / 1e9, 1),
+                         "bytes": wq_bytes, "what": "absmean (exact sum) + ternarise + 2-bit pack of the three fp32 "
+                                                   "prefill matrices, once per matrix (not on the step path)"},
         "cublas_int8_tops_context": cublas,
-        "gpu_launches": (1 + len(specs)) * K,
+        "gpu_launches": 2 * K,  # grouped act quant + one grouped GEMM per step
         "clocks": clocks,
     }
 

@@ -57,6 +57,11 @@ constexpr int kWarps = BL_GEMV_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = BL_GEMV_STAGES;         // private stages per warp
 constexpr int kRG = 8;                          // rows per row group
+// CTAs per SM the streaming kernel is compiled for: 2 lets the next launch's
+// CTAs start streaming weights beside the current ones (needs small stages)
+#ifndef BL_GEMV_MIN_BLOCKS
+#define BL_GEMV_MIN_BLOCKS 1
+#endif
 #ifndef BL_GEMV_SEG_CHUNKS
 #define BL_GEMV_SEG_CHUNKS 64
 #endif
@@ -402,7 +407,7 @@ __device__ __forceinline__ int lane_token(int lane) {
 }
 
 template <int MT, bool FUSE>
-__global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_constant__ SParams P) {
+__global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kernel(const __grid_constant__ SParams P) {
     constexpr bool kMask = MT <= 2;  // one accumulator per code field (no shifts)
     constexpr int NS = kMask ? 4 : 1;
     constexpr int V = kRG * MT;

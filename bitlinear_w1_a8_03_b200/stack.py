@@ -75,15 +75,11 @@ class LinearStack:
         return dict(x_q=self.xq[src], beta=self.beta[src], W_packed=W, alpha=alpha, N=y[name].shape[1], y=y[name])
 
     def launches(self) -> int:
-        """Kernel launches of one run (the token-count-dependent product path
-        launches one tensor-core GEMM per matrix above four tokens)."""
-        per_fwd = 1 if self.M <= 4 else None
-        n = 0
-        for _, n_a, _, n_f in self.calls:
-            n += 1 if n_a else 0
-            if n_f:
-                n += per_fwd if per_fwd else n_f
-        return n
+        """Kernel launches of one run when each call runs its quantisation and
+        its products as separate launches (the products of a call always share
+        one launch).  For at most four tokens a call may instead run as one
+        fused launch, which only lowers this count."""
+        return sum((1 if n_a else 0) + (1 if n_f else 0) for _, n_a, _, n_f in self.calls)
 
     def run(self, stream=None, flags: int = bl.BL_LINEAR_WEIGHTS_STATIC) -> None:
         """One pass of the whole stack from h0 to h_final (asynchronous)."""

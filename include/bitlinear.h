@@ -173,7 +173,8 @@ typedef struct bitlinear_act_problem {
 BITLINEAR_API bitlinear_status bitlinear_quantize_act_grouped(const bitlinear_act_problem* problems, int count,
                                                 bitlinear_dtype dtype, bitlinear_stream_t stream);
 
-/* One problem of a grouped forward; fields as in bitlinear_forward. */
+/* One problem of a grouped forward; fields as in bitlinear_forward.  Above
+ * four tokens all problems of a call share one tensor-core launch. */
 typedef struct bitlinear_forward_problem {
     const int8_t* x_q;
     const float* beta;
@@ -229,6 +230,11 @@ BITLINEAR_API bitlinear_status bitlinear_linear(const void* x, bitlinear_dtype d
 /* bitlinear_linear on `count` independent problems of one input dtype: one
  * grouped quantisation launch and one grouped product launch.  `problems` is a
  * HOST array.  flags: 0 or BL_LINEAR_WEIGHTS_STATIC.
+ * With at most four tokens per problem the quantisation may instead run in
+ * the product kernel's prologue (one launch; x_q and beta are still written),
+ * when the problems fit it and the input rows are small next to the weights;
+ * the environment variable BITLINEAR_LINEAR_FUSION=on|off forces the choice.
+ * Results are identical either way.
  * Errors: as bitlinear_linear, plus BL_ERR_COUNT, BL_ERR_FLAGS. */
 BITLINEAR_API bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* problems, int count,
                                                         bitlinear_dtype dtype, uint32_t flags,
@@ -258,7 +264,10 @@ typedef struct bitlinear_act_sum_problem {
  * any other), chained by programmatic dependent launch exactly as in
  * bitlinear_linear_grouped.  Either count may be 0, not both; each is at most
  * BITLINEAR_MAX_GROUP.  Both arrays are HOST arrays, reusable on return.
- * flags: 0 or BL_LINEAR_WEIGHTS_STATIC.
+ * flags: 0 or BL_LINEAR_WEIGHTS_STATIC.  As in bitlinear_linear_grouped, with
+ * at most four tokens the quantisation may run inside the product kernel when
+ * every product reads one of this call's inputs and every input feeds one;
+ * the first product of each input then writes its x_q, beta and x_sum.
  * Errors: as bitlinear_quantize_act (per input) and bitlinear_forward (per
  * problem), plus BL_ERR_COUNT and BL_ERR_FLAGS; nothing is launched then. */
 BITLINEAR_API bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, int n_acts,
