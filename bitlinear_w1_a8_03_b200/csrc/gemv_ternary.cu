@@ -29,6 +29,14 @@
 //    each row's sum in one lane.
 // The weight stream does not depend on the previous kernel, so it starts
 // before griddepcontrol.wait (programmatic dependent launch).
+//
+// Fused mode (at most four tokens, chosen by the host): the kernel also does
+// the per-token activation quantisation.  Right after its dependency wait each
+// CTA quantises the input rows of the (at most two) problems its range covers
+// into shared-memory slots with the same arithmetic as the activation kernel,
+// and the main loop reads x̃ and β from there; the CTA owning a problem's first
+// unit writes x̃ and β (and a residual sum) out.  One launch then replaces the
+// quantisation kernel and the product kernel.
 #include <mutex>
 
 #include <algorithm>
@@ -543,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
                 const int chunk = cons.c + it * 32 + lane;
                 if constexpr (FUSE) {
                     if (it * 32 + lane < n) {
-                        lds_act_chunk(xs_base + (uint32_t)((cons.p == p_first ? 0 : second_slot) * MT) * P.slot_row, chunk, pre[it]);
+                        lds_act_chunk(xs_base + (uint32_t)((cons.p == p_first ? 0 : second_slot) * MT) * P.slot_row,
+                                      chunk, pre[it]);
                     } else {
 #pragma unroll
                         for (int q = 0; q < 16; ++q) pre[it][q] = 0u;
@@ -577,8 +586,9 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
                         for (int q = 0; q < 16; ++q) av[m][q] = pre[it][q];
                     } else if constexpr (FUSE) {
                         if (m0 + m < pr.M) {
-                            lds_act_chunk(xs_base + (uint32_t)((cons.p == p_first ? 0 : second_slot) * MT + m) * P.slot_row, chunk,
-                                          av[m]);
+                            lds_act_chunk(xs_base + (uint32_t)((cons.p == p_first ? 0 : second_slot) * MT + m) *
+                                                        P.slot_row,
+                                          chunk, av[m]);
                         } else {
 #pragma unroll
                             for (int q = 0; q < 16; ++q) av[m][q] = 0u;
@@ -841,7 +851,8 @@ cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, 
             const int pa = problem_of(P, a), pb = problem_of(P, b - 1);
             fits = pb - pa <= 1;
             prologue_bytes += input_bytes(P.p[pa]);
-            if (pb != pa && !(P.p[pb].x == P.p[pa].x && P.p[pb].x2 == P.p[pa].x2)) prologue_bytes += input_bytes(P.p[pb]);
+            if (pb != pa && !(P.p[pb].x == P.p[pa].x && P.p[pb].x2 == P.p[pa].x2))
+                prologue_bytes += input_bytes(P.p[pb]);
         }
         if (!fuse_always && 8 * prologue_bytes > weight_bytes) fits = false;
         if (!fits) {
