@@ -1,0 +1,88 @@
+"""Host-side logic without a GPU: the layer stack's call wiring, the binding's
+problem arrays, and the benchmark's byte accounting.  Tensors live on the
+CPU; nothing here calls into the CUDA library."""
+import ctypes
+
+import torch
+
+import bitlinear_w1_a8_03_b200 as bl
+from bitlinear_w1_a8_03_b200.stack import MATRICES, LinearStack, shapes
+
+
+def _cpu_layers(hidden, ffn, L):
+    sh = shapes(hidden, ffn)
+    layers = []
+    for _ in range(L):
+        layers.append({n: (torch.zeros((sh[n][0], 16 * ((sh[n][1] + 63) // 64)), dtype=torch.uint8),
+                           torch.zeros(1, dtype=torch.float32)) for n in MATRICES})
+    return layers
+
+
+def test_stack_wiring():
+    """Per layer: call 1 quantises h (layer 0: h0; later: y_o + y_down of the
+    previous layer) for q, k, v, gate, up; call 2 quantises y_v and y_up for o
+    and down; a last call materialises y_o + y_down into h_final."""
+    hidden, ffn, L, M = 64, 128, 3, 2
+    layers = _cpu_layers(hidden, ffn, L)
+    st = LinearStack(layers, hidden, ffn, M, torch.device("cpu"), keep_all=True)
+    assert len(st.calls) == 2 * L + 1
+    assert st.launches() == 4 * L + 1
+    ptr = lambda t: t.data_ptr()
+    for l in range(L):
+        acts1, n_a1, fwd1, n_f1 = st.calls[2 * l]
+        acts2, n_a2, fwd2, n_f2 = st.calls[2 * l + 1]
+        assert (n_a1, n_f1, n_a2, n_f2) == (1, 5, 2, 2)
+        a = acts1[0]
+        if l == 0:
+            assert a.a == ptr(st.h0) and a.b is None
+        else:
+            assert a.a == ptr(st.y[l - 1]["o"]) and a.b == ptr(st.y[l - 1]["down"])
+        assert a.x_sum == ptr(st.h_in[l]) and a.x_q == ptr(st.xq["h"]) and a.M == M and a.K == hidden
+        for f, n in zip(fwd1, ("q", "k", "v", "gate", "up")):
+            assert f.x_q == ptr(st.xq["h"]) and f.y == ptr(st.y[l][n])
+            assert f.W_packed == ptr(layers[l][n][0]) and f.N == shapes(hidden, ffn)[n][0] and f.K == hidden
+        assert acts2[0].a == ptr(st.y[l]["v"]) and acts2[0].x_q == ptr(st.xq["v"]) and acts2[0].K == hidden
+        assert acts2[1].a == ptr(st.y[l]["up"]) and acts2[1].x_q == ptr(st.xq["up"]) and acts2[1].K == ffn
+        assert fwd2[0].x_q == ptr(st.xq["v"]) and fwd2[0].y == ptr(st.y[l]["o"]) and fwd2[0].K == hidden
+        assert fwd2[1].x_q == ptr(st.xq["up"]) and fwd2[1].y == ptr(st.y[l]["down"]) and fwd2[1].K == ffn
+    acts, n_a, fwd, n_f = st.calls[-1]
+    assert (n_a, n_f, fwd) == (1, 0, None)
+    assert acts[0].a == ptr(st.y[L - 1]["o"]) and acts[0].b == ptr(st.y[L - 1]["down"])
+    assert acts[0].x_sum == ptr(st.h_final)
+    assert st.weight_bytes == L * sum(16 * ((shapes(hidden, ffn)[n][1] + 63) // 64) * shapes(hidden, ffn)[n][0]
+                                      for n in MATRICES)
+
+
+def test_stack_without_keep_all_reuses_buffers():
+    st = LinearStack(_cpu_layers(64, 128, 2), 64, 128, 1, torch.device("cpu"))
+    assert len(st.y) == 1 and st.h_in is None
+    acts, _, _, _ = st.calls[2]  # layer 1 reads the shared y_o / y_down
+    assert acts[0].a == st.y[0]["o"].data_ptr() and acts[0].x_sum is None
+
+
+def test_problem_arrays_carry_shapes_and_pointers():
+    x = torch.zeros((3, 128), dtype=torch.bfloat16)
+    xq = torch.zeros((3, 128), dtype=torch.int8)
+    beta = torch.zeros(3)
+    W = torch.zeros((40, 32), dtype=torch.uint8)
+    alpha = torch.zeros(1)
+    y = torch.zeros((3, 40))
+    lin = bl.make_linear_problems([dict(x=x, x_q=xq, beta=beta, W_packed=W, alpha=alpha, N=40, y=y)])
+    assert (lin[0].M, lin[0].N, lin[0].K) == (3, 40, 128)
+    assert lin[0].x == x.data_ptr() and lin[0].y == y.data_ptr() and lin[0].bias is None
+    fwd = bl.make_forward_problems([dict(x_q=xq, beta=beta, W_packed=W, alpha=alpha, N=40, y=y)])
+    assert (fwd[0].M, fwd[0].N, fwd[0].K) == (3, 40, 128) and fwd[0].acc_out is None
+    acts = bl.make_act_sum_problems([dict(a=y, b=y, x_q=xq, beta=beta)])
+    assert (acts[0].M, acts[0].K) == (3, 40) and acts[0].b == y.data_ptr() and acts[0].x_sum is None
+    assert isinstance(acts, ctypes.Array) and len(acts) == 1
+
+
+def test_decode_bytes_per_step():
+    """The decode leg's algorithmic bytes: packed weights once, plus per matrix
+    the act quant (bf16 x in, x̃ and β out) and the product (x̃, β in; y out)."""
+    import bench
+    specs = bench.workload_specs()
+    w = sum(s.N * 16 * ((s.K + 63) // 64) for s in specs)
+    assert w == 50_593_792
+    acts = sum(2 * s.K + s.K + 4 + s.K + 4 + 4 * s.N for s in specs)
+    assert bench.bytes_per_step(specs) == w + acts == 50_906_168
