@@ -122,8 +122,15 @@ struct SharedLayout {
     int64_t bound[kWarps + 1];  // warp unit ranges inside the CTA
     int slot_acc[kSlots][kRG * kMaxMT];
     int slot_count[kSlots];
+    SProblem prob[kMaxGroup];  // copy of the problem table (indexed reads of it are cheap here)
     float xbeta[2][kMaxMT];  // fused: β of each slot's tokens
     float red[kWarps];       // fused: block reduction scratch
+};
+
+// The problem table as the kernel reads it after copying it to shared memory.
+struct ProbTable {
+    const SProblem* p;
+    int count;
 };
 
 // Position in the unit sequence: problem, (token group, row group), chunk.
@@ -134,7 +141,8 @@ struct Cursor {
     int64_t u, end;
 };
 
-__device__ __forceinline__ void cursor_seek(const SParams& P, Cursor& cur, int64_t u, int64_t end) {
+template <typename Tab>
+__device__ __forceinline__ void cursor_seek(const Tab& P, Cursor& cur, int64_t u, int64_t end) {
     int p = 0;
     while (p + 1 < P.count && u >= P.p[p + 1].unit_begin) ++p;
     const int64_t local = u - P.p[p].unit_begin;
@@ -146,14 +154,16 @@ __device__ __forceinline__ void cursor_seek(const SParams& P, Cursor& cur, int64
 }
 
 // Length (chunks) of the segment starting at the cursor.
-__device__ __forceinline__ int cursor_len(const SParams& P, const Cursor& cur) {
+template <typename Tab>
+__device__ __forceinline__ int cursor_len(const Tab& P, const Cursor& cur) {
     int64_t n = P.p[cur.p].C - cur.c;
     if (n > kSegChunks) n = kSegChunks;
     if (n > cur.end - cur.u) n = (int)(cur.end - cur.u);
     return (int)n;
 }
 
-__device__ __forceinline__ void cursor_advance(const SParams& P, Cursor& cur, int n) {
+template <typename Tab>
+__device__ __forceinline__ void cursor_advance(const Tab& P, Cursor& cur, int n) {
     cur.u += n;
     cur.c += n;
     if (cur.c == P.p[cur.p].C) {
@@ -436,8 +446,10 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
     for (int i = threadIdx.x; i < kSlots * kRG * kMaxMT; i += kThreads) (&S.slot_acc[0][0])[i] = 0;
     if (threadIdx.x < kSlots) S.slot_count[threadIdx.x] = 0;
     if (threadIdx.x < kWarps * kStages) mbar_init(smem_addr(&S.full[0][0] + threadIdx.x), 1);
+    for (int i = threadIdx.x; i < P.count; i += kThreads) S.prob[i] = P.p[i];
     fence_mbar_init();
     __syncthreads();
+    const ProbTable T{S.prob, P.count};
 
     const int64_t wu0 = S.bound[warp], wu1 = S.bound[warp + 1];
     const uint64_t policy = policy_evict_first();
@@ -446,13 +458,13 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
 
     // ---- prologue: weights do not depend on the previous kernel
     Cursor prod;
-    cursor_seek(P, prod, wu0, wu1);
+    cursor_seek(T, prod, wu0, wu1);
     int issued = 0;  // segments whose copies this warp has issued
     for (int st = 0; st < kStages && prod.u < prod.end; ++st, ++issued) {
-        const int n = cursor_len(P, prod);
-        const SProblem& pr = P.p[prod.p];
+        const int n = cursor_len(T, prod);
+        const SProblem& pr = S.prob[prod.p];
         issue_segment(pr, prod.tgrg % pr.rgn, prod.c, n, stage0 + st * kStageBytes, bar0 + 8 * st, policy, lane);
-        cursor_advance(P, prod, n);
+        cursor_advance(T, prod, n);
     }
     griddep_wait();  // x̃, β (and α) may come from the preceding kernels
 
@@ -464,16 +476,16 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
         uint8_t* xs = smem_raw + sizeof(SharedLayout);
         xs_base = smem_addr(xs);
         Cursor c0, c1;
-        cursor_seek(P, c0, a, b);
-        cursor_seek(P, c1, b > a ? b - 1 : a, b);
+        cursor_seek(T, c0, a, b);
+        cursor_seek(T, c1, b > a ? b - 1 : a, b);
         p_first = c0.p;
         for (int slot = 0; slot < 2 && a < b; ++slot) {
             const int p = p_first + slot;
             if (p > c1.p) break;
-            const SProblem& pr = P.p[p];
+            const SProblem& pr = S.prob[p];
             const bool owner = a <= pr.unit_begin && pr.unit_begin < b;
             if (slot == 1) {
-                const SProblem& p0 = P.p[p_first];
+                const SProblem& p0 = S.prob[p_first];
                 if (pr.x == p0.x && pr.x2 == p0.x2 && pr.K == p0.K && pr.M == p0.M) {
                     // same input as slot 0: reuse it (the owner still publishes x̃, β)
                     second_slot = 0;
@@ -495,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
 
     // ---- main loop over this warp's segments
     Cursor cons;
-    cursor_seek(P, cons, wu0, wu1);
+    cursor_seek(T, cons, wu0, wu1);
     const int my_tok = lane_token<MT>(lane);
     int acc[kRG][MT][NS];
     int sx[MT];
@@ -512,8 +524,8 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
     for (int seg = 0; cons.u < cons.end; ++seg) {
         const int st = seg % kStages;
         const uint32_t phase = (uint32_t)((seg / kStages) & 1);
-        const SProblem& pr = P.p[cons.p];
-        const int n = cursor_len(P, cons);
+        const SProblem& pr = S.prob[cons.p];
+        const int n = cursor_len(T, cons);
         const int tg = cons.tgrg / pr.rgn;
         const int rg = cons.tgrg - tg * pr.rgn;
         const int m0 = tg * MT;
@@ -635,13 +647,13 @@ __global__ void __launch_bounds__(kThreads, BL_GEMV_MIN_BLOCKS) gemv_stream_kern
         // refill this stage with the segment kStages ahead
         __syncwarp();
         if (prod.u < prod.end) {
-            const int pn = cursor_len(P, prod);
-            const SProblem& pp = P.p[prod.p];
+            const int pn = cursor_len(T, prod);
+            const SProblem& pp = S.prob[prod.p];
             issue_segment(pp, prod.tgrg % pp.rgn, prod.c, pn, sbase, bar0 + 8 * st, policy, lane);
-            cursor_advance(P, prod, pn);
+            cursor_advance(T, prod, pn);
             ++issued;
         }
-        cursor_advance(P, cons, n);
+        cursor_advance(T, cons, n);
 
         if (rg_done) {
             if (rg_whole && !sx_from_cache) {
