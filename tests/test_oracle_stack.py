@@ -81,3 +81,46 @@ def test_stack_output_depends_on_v_o_up_down_only():
     for n in ("v", "o", "up", "down"):
         changed = dict(layer, **{n: other[n]})
         assert not np.array_equal(oracle.stack_layer(h, changed)["h_next"], ref), n
+
+
+def _mutant_layer(kind):
+    """A stack layer with one plausible wiring mistake planted."""
+    def layer_fn(h, layer):
+        h = np.ascontiguousarray(h, dtype=np.float32)
+        out = {n: oracle.forward(h, *layer[n])[3] for n in ("q", "k", "v", "gate", "up")}
+        src_o = out["k"] if kind == "o_reads_k" else out["v"]
+        src_down = out["gate"] if kind == "down_reads_gate" else out["up"]
+        out["o"] = oracle.forward(src_o, *layer["o"])[3]
+        out["down"] = oracle.forward(src_down, *layer["down"])[3]
+        if kind == "no_residual_down":
+            out["h_next"] = out["o"].copy()
+        elif kind == "sum_after_quant_of_parts":
+            # quantising y_o and y_down separately and adding the dequantised
+            # codes instead of quantising their float sum
+            xo, bo = oracle.quantize_act(out["o"])
+            xd, bd = oracle.quantize_act(out["down"])
+            out["h_next"] = (xo * (bo[:, None] / np.float32(127)) + xd * (bd[:, None] / np.float32(127))
+                             ).astype(np.float32)
+        else:
+            out["h_next"] = np.add(out["o"], out["down"], dtype=np.float32)
+        return out
+    return layer_fn
+
+
+@pytest.mark.parametrize("kind", ["o_reads_k", "down_reads_gate", "no_residual_down", "sum_after_quant_of_parts"])
+def test_stack_pins_reject_planted_wiring_mistakes(kind):
+    """Each mutant disagrees with the independent float64 recomposition
+    (the pin the real stack_layer passes)."""
+    layer = _layer(40)
+    h = _h0(3, seed=9)
+    mutant = _mutant_layer(kind)(h, layer)
+    ys = {n: _product_f64(h, *layer[n]) for n in ("q", "k", "v", "gate", "up")}
+    ys["o"] = _product_f64(ys["v"], *layer["o"])
+    ys["down"] = _product_f64(ys["up"], *layer["down"])
+    h_next = (ys["o"] + ys["down"]).astype(np.float32)
+    agree = all(np.array_equal(mutant[n], ys[n]) for n in oracle.STACK_MATRICES) and \
+        np.array_equal(mutant["h_next"], h_next)
+    assert not agree
+    real = oracle.stack_layer(h, layer)
+    assert all(np.array_equal(real[n], ys[n]) for n in oracle.STACK_MATRICES)
+    assert np.array_equal(real["h_next"], h_next)
