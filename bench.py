@@ -122,6 +122,17 @@ def recorded_traffic(kernel_tag: str, sources):
     return None
 
 
+def decode_config(specs) -> dict:
+    """The decode workload's config, identical in the native and reference arms."""
+    return {
+        "workload": "7B decode layer set, M=1: q,k,v,o 4096->4096; gate,up 4096->11008; down 11008->4096",
+        "bytes_per_step": bytes_per_step(specs),
+        "weight_bytes_per_step": sum(s.N * 16 * ((s.K + 63) // 64) for s in specs),
+        "l2": "inputs larger than L2: weight replicas rotate across steps, together more than 4x the L2",
+        "parallelism": "replicas (one independent replica of the workload per GPU, weak scaling)",
+    }
+
+
 # ----------------------------------------------------------------------------- ranks
 def max_over_ranks(values, device, world: int):
     """Element-wise max of per-rank timings (ms) over all ranks; identity at N=1."""
@@ -182,6 +193,24 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
                 "samples": len(sms)}
+
+
+def gpu_id(props, local_rank) -> str:
+    return "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local_rank)
+
+
+def settle(stream, replay, props, local_rank, seconds: float = 1.0) -> ClockSampler:
+    """Starts the clock sampler, then runs about `seconds` of identical replays
+    so the timed region that follows runs at settled clocks; the caller stops
+    the sampler after its timed region (and a few more replays)."""
+    import torch
+    sampler = ClockSampler(gpu_id(props, local_rank))
+    t_end = time.time() + seconds
+    with torch.cuda.stream(stream):
+        while time.time() < t_end:
+            replay()
+            stream.synchronize()
+    return sampler
 
 
 # ----------------------------------------------------------------------------- native arm
@@ -257,13 +286,7 @@ def run_native(args, rank, world, local_rank):
         for _ in range(max(1, math.ceil(args.warmup / replicas))):
             g_warm.replay()
     stream.synchronize()
-    gpu_id = "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local_rank)
-    sampler = ClockSampler(gpu_id)
-    t_end = time.time() + 1.0
-    with torch.cuda.stream(stream):
-        while time.time() < t_end:
-            g_warm.replay()
-            stream.synchronize()
+    sampler = settle(stream, g_warm.replay, props, local_rank)
 
     import torch.distributed as dist
     if world > 1:
@@ -367,15 +390,12 @@ def run_native(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "int8 x ternary(2-bit) -> int32, fp32 dequant",
         "data": "synthetic (seeded SplitMix64/Box-Muller; W ~ N(0,0.02) ternarised once, x bf16 ~ N(0,1) + 0.1% x20 outliers)",
-        "config": {
-            "workload": "7B decode layer set, M=1: q,k,v,o 4096->4096; gate,up 4096->11008; down 11008->4096",
-            "bytes_per_step": bps,
-            "weight_bytes_per_step": set_bytes,
-            "l2": f"inputs larger than L2: {replicas} rotating weight replicas, {replicas * set_bytes / 1e6:.0f} MB "
+        "config": decode_config(specs),
+        "timing": {
+            "l2": f"{replicas} rotating weight replicas, {replicas * set_bytes / 1e6:.0f} MB "
                   f"(L2 {props.L2_cache_size / 1e6:.0f} MB)",
             "launch": "K steps captured in one CUDA graph; per step one bitlinear_linear_grouped call "
                       "(BL_LINEAR_WEIGHTS_STATIC) = one fused quantise + GEMV launch, steps chained by PDL",
-            "parallelism": f"replicas x{world}",
             "pct_of_8TBps": round(100 * value / world / 8000.0, 2),
         },
         "roofline": {
@@ -448,8 +468,7 @@ def run_prefill(args, world, local_rank):
     with torch.cuda.stream(stream):
         g.replay()  # warm replay (W steps already ran eagerly)
     stream.synchronize()
-    gpu_id = "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local_rank)
-    sampler = ClockSampler(gpu_id)
+    sampler = settle(stream, g.replay, props, local_rank)  # ≈1 s of identical steps under the clock sampler
     import torch.distributed as dist
     if world > 1:
         dist.barrier()
@@ -593,6 +612,145 @@ def run_prefill(args, world, local_rank):
     }
 
 
+# ----------------------------------------------------------------------------- 100B batched-decode leg
+def run_batched_100b(args, world, local_rank):
+    """The 100B-shaped batched decode sweep: (K, N) = (8192, 28672) and
+    (28672, 8192), M in {1, 2, 4, 8, 16, 32, 64}.  One step is one
+    bitlinear_linear_grouped call on one matrix (act quant + product, flagged
+    BL_LINEAR_WEIGHTS_STATIC); K steps per M in one CUDA graph over weight
+    replicas that together exceed 4x the L2.  GB/s = algorithmic bytes per
+    step (as for the decode leg) / time per step."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth, workloads
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    peak = float(load_peaks()[0]["hbm_gbs"])
+    L = bl.lib()
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    Ms = (1, 2, 4, 8, 16, 32, 64)
+    K_steps = max(12, args.steps)
+    out, sampler, graphs = {}, None, []
+    for (K, N) in ((8192, 28672), (28672, 8192)):
+        spec0 = workloads.batched_decode_100b(K, N, 1)
+        W = torch.from_numpy(synth.weights(spec0.seed, N, K, spec0.w_std)).to(dev)
+        p0, alpha = bl.bitlinear_quantize_weights(W)
+        del W
+        wbytes = p0.numel()
+        replicas = max(2, math.ceil(4 * props.L2_cache_size / wbytes) + 1)
+        packed = [p0] + [p0.clone() for _ in range(replicas - 1)]
+        per_m = {}
+        for M in Ms:
+            spec = workloads.batched_decode_100b(K, N, M)
+            xb = synth.f32_to_bf16_bits(synth.activations(spec.x_seed, M, K))
+            x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+            xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+            beta = torch.empty(M, dtype=torch.float32, device=dev)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            arrs = [bl.make_linear_problems([dict(x=x, x_q=xq, beta=beta, W_packed=packed[r], alpha=alpha, N=N, y=y)])
+                    for r in range(replicas)]
+
+            def step(i):
+                bl.check(L.bitlinear_linear_grouped(arrs[i % replicas], 1, bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
+                                                    sh), "linear")
+
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    step(i)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(K_steps):
+                    step(i)
+            graphs.append(g)
+            if sampler is None:
+                sampler = settle(stream, g.replay, props, local_rank)
+            with torch.cuda.stream(stream):
+                g.replay()
+            stream.synchronize()
+            if world > 1:
+                import torch.distributed as dist
+                dist.barrier()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                t0.record()
+                g.replay()
+                t1.record()
+            t1.synchronize()
+            ms = max_over_ranks([t0.elapsed_time(t1) / K_steps], dev, world)[0]
+            bps = bytes_per_step([spec])
+            gbs = bps / (ms * 1e-3) / 1e9
+            per_m[f"M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
+                              "frac": round(gbs / peak, 4), "pct_of_8TBps": round(100 * gbs / 8000.0, 2),
+                              "kernel": "gemv_stream_kernel (CUDA cores)" if M <= 4 else "gemm_tc_kernel (tcgen05 i8)"}
+        out[f"K{K}_N{N}"] = {"weight_bytes": wbytes, "replicas": replicas, **per_m}
+        del packed, p0
+    with torch.cuda.stream(stream):
+        graphs[-1].replay()
+    stream.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
+    del graphs
+    worst = min((v["frac"], k, m) for k, d in out.items() for m, v in d.items() if isinstance(v, dict))
+    return {
+        "metric": "ternary GEMV/GEMM HBM GB/s, 100B-shaped batched decode",
+        "workload": "100B-shaped batched decode: (K,N) = (8192,28672) and (28672,8192), M in {1,2,4,8,16,32,64}; "
+                    "W ~ N(0,0.015) ternarised once, x bf16 ~ N(0,1); per step one bitlinear_linear_grouped call "
+                    "(act quant + product + dequant), K steps in one CUDA graph",
+        "l2": "weight replicas rotate across steps, together more than 4x the L2",
+        "steps": K_steps,
+        "peak": peak,
+        "unit": "GB/s",
+        **out,
+        "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peak,
+                     "achieved_M1": {k: d["M1"]["GB/s"] for k, d in out.items()},
+                     "frac_M1": {k: d["M1"]["frac"] for k, d in out.items()},
+                     "lowest_frac": {"frac": worst[0], "shape": worst[1], "M": worst[2]}},
+        "clocks": clocks,
+    }
+
+
+# ----------------------------------------------------------------------------- tiny leg
+def run_tiny(args, world, local_rank):
+    """Config 1: M = 1, K = N = 256, float32 x and W (seed 0).  A latency line:
+    each bitlinear_linear call timed alone with CUDA events, an L2 flush (a
+    write larger than the L2) between calls outside the timed events."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth, workloads
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    s = workloads.tiny()
+    packed, alpha = bl.bitlinear_quantize_weights(torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev))
+    x = torch.from_numpy(synth.activations(s.x_seed, s.M, s.K)).to(dev)
+    xq = torch.empty((s.M, s.K), dtype=torch.int8, device=dev)
+    beta = torch.empty(s.M, dtype=torch.float32, device=dev)
+    y = torch.empty((s.M, s.N), dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * props.L2_cache_size // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    reps = max(20, args.steps)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            bl.bitlinear_linear(x, packed, alpha, s.N, x_q=xq, beta=beta, y=y, stream=stream)
+        for e0, e1 in evs:
+            flush.fill_(1.0)
+            e0.record()
+            bl.bitlinear_linear(x, packed, alpha, s.N, x_q=xq, beta=beta, y=y, stream=stream)
+            e1.record()
+    stream.synchronize()
+    us = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
+    med = statistics.median(us)
+    bytes_call = s.N * 16 * ((s.K + 63) // 64) + s.M * s.K * 4 + s.M * s.K + 4 * s.M + s.M * s.K + 4 * s.M + 4 * s.M * s.N
+    us = max_over_ranks([med], dev, world)[0]
+    return {"metric": "latency of one bitlinear_linear call (act quant + GEMV + dequant), L2 flushed between calls",
+            "workload": "tiny: M=1, K=N=256, fp32 x ~ N(0,1), W ~ N(0,0.02), seed 0",
+            "us_per_call_median": round(us, 3), "GB/s": round(bytes_call / (us * 1e-6) / 1e9, 2),
+            "bytes_per_call": bytes_call, "calls": reps}
+
+
 # ----------------------------------------------------------------------------- stack leg
 def run_stack(args, world, local_rank):
     """The 32-layer 7B-shaped linear stack per decode step (M = 1 and 16)."""
@@ -602,6 +760,7 @@ def run_stack(args, world, local_rank):
     from bitlinear_w1_a8_03_b200.stack import MATRICES, LinearStack, shapes
 
     dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
     hidden, ffn, L = 4096, 11008, 32
     sh = shapes(hidden, ffn)
     g = torch.Generator(device=dev)
@@ -632,6 +791,7 @@ def run_stack(args, world, local_rank):
         with torch.cuda.stream(stream):
             gr.replay()
         stream.synchronize()
+        sampler = settle(stream, gr.replay, props, local_rank)
         import torch.distributed as dist
         if world > 1:
             dist.barrier()
@@ -641,6 +801,10 @@ def run_stack(args, world, local_rank):
             gr.replay()
             t1.record()
         t1.synchronize()
+        with torch.cuda.stream(stream):
+            gr.replay()
+        stream.synchronize()
+        clocks = sampler.stop()
         ms = max_over_ranks([t0.elapsed_time(t1) / K], dev, world)[0]
         # per token and layer: quant(y_o + y_down) 8H in, H out; x_h read once, y_q,k,v 12H and y_gate,up
         # 8F out; quant(y_v, y_up) 4H + 4F in, H + F out; x_v + x_up read, y_o + y_down 8H out
@@ -656,6 +820,7 @@ def run_stack(args, world, local_rank):
             "steps": K,
             "gpu_launches_per_step": st.launches(),
             "device_error": err,
+            "clocks": clocks,
         }
         del gr, st
     return {
@@ -762,8 +927,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "int8 x ternary -> int64 (checked into int32), fp32 dequant",
         "data": "synthetic (same seeds as the native arm)",
-        "config": {"workload": "7B decode layer set, M=1: q,k,v,o 4096->4096; gate,up 4096->11008; down 11008->4096",
-                   "parallelism": "host cores"},
+        "config": decode_config(workload_specs()),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -777,8 +941,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--legs", default="decode,prefill,stack",
-                    help="comma list: decode (the headline line), prefill and stack (added under their keys)")
+    ap.add_argument("--legs", default="decode,tiny,batched_100b,prefill,stack",
+                    help="comma list: decode (the headline line); tiny, batched_100b, prefill and stack are added "
+                         "under their own keys")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     args = ap.parse_args()
     legs = [x for x in args.legs.split(",") if x]
@@ -809,6 +974,10 @@ def main():
             result.update({"value": pre["value"], "unit": pre["unit"], "n_gpus": world, "steps": args.steps,
                            "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True,
                            "scaling": "weak", "vs_baseline": None})
+    if "tiny" in legs:
+        result["tiny"] = run_tiny(args, world, local_rank)
+    if "batched_100b" in legs:
+        result["batched_100b"] = run_batched_100b(args, world, local_rank)
     if "stack" in legs:
         result["stack"] = run_stack(args, world, local_rank)
     if rank == 0:

@@ -5,6 +5,7 @@
 // compute capability 10.0, then enqueues kernels on the caller's stream.
 #include <mutex>
 
+#include "bl_attr.h"
 #include "bl_launch.h"
 
 namespace bl {
@@ -29,6 +30,17 @@ cudaError_t device_info(DeviceInfo* out) {
     }
     *out = cache[dev];
     return cudaSuccess;
+}
+
+cudaError_t set_max_dynamic_smem(const void* func, int bytes) {
+    static AttrOnce once;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    const int rc = once.ensure(func, dev, [&] {
+        return (int)cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+    return rc < 0 ? cudaErrorInvalidDevice : static_cast<cudaError_t>(rc);
 }
 
 }  // namespace bl
@@ -75,6 +87,28 @@ bitlinear_status check_forward(const bitlinear_forward_problem& p) {
 }
 
 bool valid_dtype(bitlinear_dtype d) { return d == BL_F32 || d == BL_BF16; }
+
+// Byte ranges [p, p + n) and [q, q + m) intersect.
+bool ranges_overlap(const void* p, int64_t n, const void* q, int64_t m) {
+    if (!p || !q) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + (uintptr_t)m && b < a + (uintptr_t)n;
+}
+
+// Some x_sum of the call overlaps some a or b of the call.
+bool sums_overlap_inputs(const bitlinear_act_sum_problem* acts, int n) {
+    for (int i = 0; i < n; ++i) {
+        if (!acts[i].x_sum) continue;
+        const int64_t bytes_i = acts[i].M * acts[i].K * 4;
+        for (int j = 0; j < n; ++j) {
+            const int64_t bytes_j = acts[j].M * acts[j].K * 4;
+            if (ranges_overlap(acts[i].x_sum, bytes_i, acts[j].a, bytes_j) ||
+                ranges_overlap(acts[i].x_sum, bytes_i, acts[j].b, bytes_j))
+                return true;
+        }
+    }
+    return false;
+}
 
 }  // namespace
 
@@ -239,7 +273,9 @@ bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, i
     if (n_acts > 0 && n_fwd > 0) {
         bl::FusedInput fin[BITLINEAR_MAX_GROUP];
         bool used[BITLINEAR_MAX_GROUP] = {};
-        bool ok = true;
+        // In the fused form other CTAs still read a and b while the owner of an
+        // input writes its x_sum, so an x_sum that overlaps any input rules it out.
+        bool ok = !sums_overlap_inputs(acts, n_acts);
         for (int i = 0; i < n_fwd && ok; ++i) {
             int j = 0;
             while (j < n_acts && !(acts[j].x_q == fwd[i].x_q && acts[j].beta == fwd[i].beta && acts[j].M == fwd[i].M &&

@@ -15,6 +15,10 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// Opts `func` in to `bytes` of dynamic shared memory on the current device,
+// once per (kernel, device) for the life of the process (thread-safe).
+cudaError_t set_max_dynamic_smem(const void* func, int bytes);
+
 // One activation-quantisation job: x = a, or a + b (float32 only) when b is
 // set; x_sum (nullable) receives x.
 struct ActJob {

@@ -518,12 +518,9 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
     }
     P.tiles = tiles;
 
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
+    // the opt-in is per device: set once on each device that launches the kernel
+    err = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tc_kernel<NT>), (int)C::kSmem);
+    if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count));
     cfg.blockDim = dim3(kThreads);

@@ -37,7 +37,6 @@
 // and the main loop reads x̃ and β from there; the CTA owning a problem's first
 // unit writes x̃ and β (and a residual sum) out.  One launch then replaces the
 // quantisation kernel and the product kernel.
-#include <mutex>
 
 #include <algorithm>
 #include <cstdlib>
@@ -875,15 +874,9 @@ cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, 
     }
     const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, true>)
                                : reinterpret_cast<const void*>(gemv_stream_kernel<MT, false>);
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemv_stream_kernel<MT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)sizeof(SharedLayout));
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(gemv_stream_kernel<MT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)(sizeof(SharedLayout) + 2 * kFuseSlotBytes));
-    });
+    // the opt-in is per device: set once on each device that launches the kernel
+    cudaError_t attr_err = set_max_dynamic_smem(
+        kernel, fused ? (int)(sizeof(SharedLayout) + 2 * kFuseSlotBytes) : (int)sizeof(SharedLayout));
     if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);

@@ -281,6 +281,8 @@ cudaError_t launch_quantize_weights(const void* W, bitlinear_dtype dtype, int64_
 // that device's first call; that first call should therefore come before any
 // stream capture.
 static __device__ __align__(256) unsigned long long g_static_partials[kMaxPartials * kLimbs];
+static_assert(sizeof(g_static_partials) == (size_t)kMaxPartials * kLimbs * sizeof(unsigned long long),
+              "the static scratch holds the largest partial-sum grid (partial_blocks never exceeds kMaxPartials)");
 
 namespace {
 

@@ -114,7 +114,9 @@ BITLINEAR_API bitlinear_status bitlinear_quantize_weights(const void* W, bitline
  * overwrites what it reads, so calls that overlap on the GPU (e.g. on two
  * unordered streams) race and give wrong results; order them on one stream.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) and so should come before any stream capture.
+ * (cudaGetSymbolAddress) and so should come before any stream capture.  The
+ * address is kept for the life of the process: resetting a device
+ * (cudaDeviceReset) after that first call is not supported.
  * Arguments, layouts and errors are those of bitlinear_quantize_weights; the
  * maximum size is the same (N·K <= 2^40, K <= BITLINEAR_MAX_K), and larger
  * sizes return BL_ERR_SHAPE. */
@@ -247,7 +249,11 @@ BITLINEAR_API bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_p
  * chenxutan.com/d/5049.html §6.1).  x is quantised exactly as by
  * bitlinear_quantize_act into x_q [M][K] and beta [M]; x_sum (nullable,
  * [M][K] float32) receives x itself.  a, b and x_sum are float32 [M][K]
- * row-major, 4-byte aligned; x_q as in bitlinear_quantize_act. */
+ * row-major, 4-byte aligned; x_q as in bitlinear_quantize_act.
+ * x_sum may be exactly a or exactly b (an in-place residual update h += y);
+ * otherwise it must not overlap any a or b of the call (a partial overlap
+ * gives undefined results).  When an x_sum overlaps an input, the call does
+ * not take the single-launch fused form described below. */
 typedef struct bitlinear_act_sum_problem {
     const float* a;
     const float* b;

@@ -86,3 +86,18 @@ def test_decode_bytes_per_step():
     assert w == 50_593_792
     acts = sum(2 * s.K + s.K + 4 + s.K + 4 + 4 * s.N for s in specs)
     assert bench.bytes_per_step(specs) == w + acts == 50_906_168
+
+
+def test_kernel_attribute_set_once_per_device(tmp_path):
+    """The opt-in shared-memory attribute is per device: the bookkeeping in
+    csrc/bl_attr.h must run the setting once for each (kernel, device) pair,
+    retry a failed setting, and refuse devices outside its table.  Compiled
+    with the host compiler only (no CUDA)."""
+    import os
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "attr_once_check")
+    subprocess.check_call(["g++", "-std=c++17", "-O1", "-I", os.path.join(root, "bitlinear_w1_a8_03_b200", "csrc"),
+                           os.path.join(root, "tests", "native", "attr_once_check.cpp"), "-o", exe, "-pthread"])
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout

@@ -108,3 +108,43 @@ def test_prefill_2048(K, N):
     acc = torch.empty((spec.M, N), dtype=torch.int32, device="cuda")
     y = bl.bitlinear_forward(xq, beta, packed, alpha, N, acc_out=acc)
     check_sampled(xq, beta, acc, y, xo, codes, a_ref, sample_rows(N, K, n=48))
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 32, 64])
+def test_100b_bench_call_graph_rotating_replicas(weights_100b, M):
+    """The call the benchmark times for the 100B sweep: one
+    bitlinear_linear_grouped problem flagged BL_LINEAR_WEIGHTS_STATIC, two
+    steps in one CUDA graph over two weight replicas, a new input per step."""
+    K, N, packed, alpha, codes, a_ref = weights_100b
+    spec = workloads.batched_decode_100b(K, N, M)
+    replicas = [packed, packed.clone()]
+    steps = []
+    for st in range(2):
+        xb = synth.f32_to_bf16_bits(synth.activations(spec.x_seed + 1000 * st, M, K))
+        xd = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+        p = dict(x=xd, x_q=torch.empty((M, K), dtype=torch.int8, device="cuda"),
+                 beta=torch.empty(M, dtype=torch.float32, device="cuda"), W_packed=replicas[st], alpha=alpha, N=N,
+                 y=torch.empty((M, N), dtype=torch.float32, device="cuda"),
+                 acc_out=torch.empty((M, N), dtype=torch.int32, device="cuda"))
+        steps.append((xb, p, bl.make_linear_problems([p])))
+    L = bl.lib()
+    stream = torch.cuda.Stream()
+
+    def call(st):
+        bl.check(L.bitlinear_linear_grouped(steps[st][2], 1, bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
+                                            stream.cuda_stream), "bitlinear_linear_grouped")
+
+    with torch.cuda.stream(stream):
+        call(0)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        call(0)
+        call(1)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    for st, (xb, p, _) in enumerate(steps):
+        check_sampled(p["x_q"], p["beta"], p["acc_out"], p["y"], xb, codes, a_ref, sample_rows(N, 31 * M + st))
+    del g

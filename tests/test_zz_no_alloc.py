@@ -40,7 +40,11 @@ def test_static_scratch_matches_workspace_entry_point_twice():
         assert np.array_equal(p_static.cpu().numpy(), p_ref.cpu().numpy())
 
 
-def test_static_rejects_oversize_before_launch():
+def test_static_rejects_shapes_beyond_the_shared_limit():
+    """N·K above 2^40 is refused before anything is launched.  The static
+    entry point shares this limit with the workspace one; its own scratch-size
+    check cannot fire for accepted shapes (the partial-sum grid is capped at
+    the scratch size, pinned by a static_assert in the library)."""
     L = bl.lib()
     P = 0x7F0000000000
     assert L.bitlinear_quantize_weights_static(P, 0, 1 << 30, 1 << 20, P, P, None) == 2  # BL_ERR_SHAPE
