@@ -4,10 +4,15 @@ TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, the smoke check in
 ``__graft_entry__`` and the benchmark's CPU-baseline / reference arm may import
 this package.  It shares no code with the CUDA library and never imports it.
 
-Pinned functions (the pins live in ``tests/test_oracle_pins.py`` and, for the
-layer stack, ``tests/test_oracle_stack.py``): ``absmean``, ``ternarize``,
-``pack``, ``quantize_act``, ``ternary_matmul``, ``dequant``, ``forward``,
-``stack_layer``, ``stack_forward``.  No function here is "parity unpinned".
+Pinned functions (the pins live in ``tests/test_oracle_pins.py``, for the
+layer stack ``tests/test_oracle_stack.py``, and for the rotation, the finer
+scale granularities and the 4-bit activations ``tests/test_oracle_variants.py``):
+``absmean``, ``ternarize``, ``pack``, ``quantize_act``, ``ternary_matmul``,
+``dequant``, ``forward``, ``stack_layer``, ``stack_forward``, ``hadamard``,
+``hadamard_block``, ``quantize_weights_rotated``, ``quantize_act_rotated``,
+``absmean_groups``, ``ternarize_groups``, ``forward_groups``,
+``quantize_act_a4``, ``unpack_a4``, ``dequant_a4``, ``forward_a4``.  No
+function here is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -53,6 +58,15 @@ def configure(lib):
     lib.orc_dequant.argtypes = [p, p, f32, p, i64, i64, p]
     lib.orc_dequant.restype = None
     lib.orc_forward.argtypes = [p, i32, i64, i64, p, f32, p, i64, p, p, p, p, i32]
+    lib.orc_hadamard.argtypes = [p, i32, i64, i64, i64, f32, p]
+    lib.orc_absmean_groups.argtypes = [p, i32, i64, i64, i64, p]
+    lib.orc_ternarize_groups.argtypes = [p, i32, i64, i64, i64, p, p]
+    lib.orc_forward_groups.argtypes = [p, p, i64, i64, p, p, i64, p, i64, p, i32]
+    lib.orc_quantize_act_a4.argtypes = [p, i32, i64, i64, p, p]
+    lib.orc_unpack_a4.argtypes = [p, i64, i64, p]
+    lib.orc_unpack_a4.restype = None
+    lib.orc_dequant_a4.argtypes = [p, p, f32, p, i64, i64, p]
+    lib.orc_dequant_a4.restype = None
     return lib
 
 
@@ -211,3 +225,127 @@ def stack_forward(h0: np.ndarray, layers: list, threads: int = 1) -> list:
         outs.append(o)
         h = o["h_next"]
     return outs
+
+
+# ----------------------------------------------------------------------------- rotation
+def hadamard_block(K: int, cap: int = 8192) -> int:
+    """Block order used when a rotation is asked for without one: the largest
+    power of two dividing K, at most `cap` (4096 for K = 4096, 256 for 11008)."""
+    b = 1
+    while K % (2 * b) == 0 and 2 * b <= cap:
+        b *= 2
+    return b
+
+
+def hadamard(x: np.ndarray, block: int, scale: float = 1.0) -> np.ndarray:
+    """x·H per row, H block-diagonal Sylvester Hadamard of order `block`, by the
+    binary32 butterfly (stages h = 1, 2, 4, …), outputs times `scale`
+    ([BitNet 三值权重实战] §6.2)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    out = np.empty((M, K), dtype=np.float32)
+    if _load().orc_hadamard(_ptr(x), dt, M, K, block, ctypes.c_float(float(np.float32(scale))), _ptr(out)) != 0:
+        raise ValueError("block must be a power of two dividing K")
+    return out
+
+
+def quantize_weights_rotated(W: np.ndarray, block: int):
+    """(packed, α, codes, W') of W' = W·H/block: the weight side of the rotation,
+    so that (x·H)·W'ᵀ = x·Wᵀ in exact arithmetic."""
+    Wr = hadamard(W, block, 1.0 / block)
+    packed, alpha, codes = quantize_weights(Wr)
+    return packed, alpha, codes, Wr
+
+
+def quantize_act_rotated(x: np.ndarray, block: int):
+    """(x̃, β, x·H): the absmax int8 quantisation of the rotated activations."""
+    xr = hadamard(x, block)
+    xq, beta = quantize_act(xr)
+    return xq, beta, xr
+
+
+# ----------------------------------------------------------------------------- scale granularity
+def absmean_groups(W: np.ndarray, group: int) -> np.ndarray:
+    """α [N][ceil(K/group)]: exact mean of |W| over each group of `group`
+    consecutive elements of a row, RN32(RN64(·)) (per row: group >= K)."""
+    W, dt = _as_input(W)
+    N, K = W.shape
+    G = -(-K // group)
+    out = np.empty((N, G), dtype=np.float32)
+    if _load().orc_absmean_groups(_ptr(W), dt, N, K, group, _ptr(out)) != 0:
+        raise ValueError("non-finite weight or bad group")
+    return out
+
+
+def ternarize_groups(W: np.ndarray, alpha: np.ndarray, group: int) -> np.ndarray:
+    """Codes ŵ = clip(round(W/α_group), -1, 1)."""
+    W, dt = _as_input(W)
+    N, K = W.shape
+    alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+    out = np.empty((N, K), dtype=np.int8)
+    _load().orc_ternarize_groups(_ptr(W), dt, N, K, group, _ptr(alpha), _ptr(out))
+    return out
+
+
+def quantize_weights_groups(W: np.ndarray, group: int):
+    """(packed, α [N][G], codes) with one α per group of each row."""
+    alpha = absmean_groups(W, group)
+    codes = ternarize_groups(W, alpha, group)
+    return pack(codes), alpha, codes
+
+
+def forward_groups(xq: np.ndarray, beta: np.ndarray, codes: np.ndarray, alpha: np.ndarray, group: int,
+                   bias: np.ndarray | None = None, threads: int = 1) -> np.ndarray:
+    """y with one α per group: S = Σ_b α_b·acc_b (binary64, groups in order),
+    y = RN32(RN32(S)·RN32(RN64(β/127))) (+ bias)."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    beta = np.ascontiguousarray(beta, dtype=np.float32)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+    M, K = xq.shape
+    N = codes.shape[0]
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((M, N), dtype=np.float32)
+    _load().orc_forward_groups(_ptr(xq), _ptr(beta), M, K, _ptr(codes), _ptr(alpha), group, _ptr(bias), N, _ptr(y),
+                               threads)
+    return y
+
+
+# ----------------------------------------------------------------------------- 4-bit activations
+def quantize_act_a4(x: np.ndarray):
+    """(x̃ packed 4-bit [M][ceil(K/2)] uint8, β [M]): clip(round(7x/β), -7, 7)."""
+    x, dt = _as_input(x)
+    M, K = x.shape
+    xq4 = np.empty((M, (K + 1) // 2), dtype=np.uint8)
+    beta = np.empty(M, dtype=np.float32)
+    _load().orc_quantize_act_a4(_ptr(x), dt, M, K, _ptr(xq4), _ptr(beta))
+    return xq4, beta
+
+
+def unpack_a4(xq4: np.ndarray, K: int) -> np.ndarray:
+    xq4 = np.ascontiguousarray(xq4, dtype=np.uint8)
+    M = xq4.shape[0]
+    out = np.empty((M, K), dtype=np.int8)
+    _load().orc_unpack_a4(_ptr(xq4), M, K, _ptr(out))
+    return out
+
+
+def dequant_a4(acc: np.ndarray, beta: np.ndarray, alpha, bias: np.ndarray | None = None) -> np.ndarray:
+    """y = fp32(acc)·fp32(α·β/7) (+ bias)."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    beta = np.ascontiguousarray(beta, dtype=np.float32)
+    M, N = acc.shape
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((M, N), dtype=np.float32)
+    _load().orc_dequant_a4(_ptr(acc), _ptr(beta), ctypes.c_float(float(np.float32(alpha))), _ptr(bias), M, N, _ptr(y))
+    return y
+
+
+def forward_a4(x: np.ndarray, codes: np.ndarray, alpha, bias: np.ndarray | None = None, threads: int = 1):
+    """4-bit-activation forward on cached codes: returns (x̃ packed, β, acc, y)."""
+    xq4, beta = quantize_act_a4(x)
+    K = codes.shape[1]
+    acc = ternary_matmul(unpack_a4(xq4, K), codes, threads=threads)
+    return xq4, beta, acc, dequant_a4(acc, beta, alpha, bias)

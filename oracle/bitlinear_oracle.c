@@ -169,3 +169,236 @@ int orc_forward(const void* x, int dtype, int64_t M, int64_t K, const int8_t* co
     orc_dequant(acc, beta, alpha, bias, M, N, y);
     return rc;
 }
+
+/* ------------------------------------------------------------------------
+ * Rotation before the absmax quantisation ([BitNet 三值权重实战] §6.2: an
+ * orthogonal (Hadamard) rotation of the activations spreads an outlier's
+ * energy over all dimensions before absmax quantisation).
+ *
+ * out[m][·] = x[m][·]·H, H block-diagonal with Sylvester Hadamard blocks of
+ * order `block` (a power of two dividing K): inside a block,
+ * out[j] = Σ_i x[i]·(-1)^popcount(i & j).  Evaluated by the fast
+ * Walsh–Hadamard butterfly network in binary32 with the stages in a fixed
+ * order, h = 1, 2, 4, …, block/2: each butterfly replaces the pair at
+ * positions (i, i + h), i & h == 0, by (a + b, a - b).  Every output is then
+ * multiplied by `scale` (1 for activations; 1/block, a power of two, for the
+ * weights, so that (x·H)·(W·H/block)ᵀ = x·Wᵀ in exact arithmetic). */
+int orc_hadamard(const void* x, int dtype, int64_t M, int64_t K, int64_t block, float scale, float* out) {
+    if (block < 1 || (block & (block - 1)) != 0 || K % block != 0) return -1;
+    for (int64_t m = 0; m < M; ++m) {
+        float* v = out + m * K;
+        for (int64_t k = 0; k < K; ++k) v[k] = orc_load(x, dtype, m * K + k);
+        for (int64_t s = 0; s < K; s += block) {
+            float* b = v + s;
+            for (int64_t h = 1; h < block; h <<= 1) {
+                for (int64_t i = 0; i < block; ++i) {
+                    if (i & h) continue;
+                    float p = b[i], q = b[i + h];
+                    b[i] = p + q;
+                    b[i + h] = p - q;
+                }
+            }
+        }
+        if (scale != 1.0f)
+            for (int64_t k = 0; k < K; ++k) v[k] = v[k] * scale;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Scale granularity finer than the tensor: per output row ([1.58 位大模型]
+ * §3.1, §4.2: alpha = mean(|w|, axis=-1)) and per block of consecutive input
+ * features within a row ([硬件协同优化] §2.3, §4.2: one scale per 128
+ * elements, scale[C_out][C_in/128]).  Both are groups of `group` consecutive
+ * elements of a row (group >= K: one group per row); the last group of a row
+ * may be shorter.  Each α is the exact mean rounded once to binary64 and once
+ * to binary32, as for the tensor. */
+
+/* RN64(S / count) where S·2^149 = limbs (little-endian 32-bit digits). */
+static double orc_exact_mean(const uint64_t* limbs_in, int nlimbs, uint64_t count) {
+    enum { EXTRA = 4 };                /* 128 more bits below the sum for the quotient */
+    uint32_t num[32], q[32];
+    int n = nlimbs + EXTRA;
+    for (int j = 0; j < EXTRA; ++j) num[j] = 0;
+    for (int j = 0; j < nlimbs; ++j) num[EXTRA + j] = (uint32_t)limbs_in[j];
+    /* long division by count, most significant digit first */
+    unsigned __int128 rem = 0;
+    for (int j = n - 1; j >= 0; --j) {
+        unsigned __int128 cur = (rem << 32) | num[j];
+        q[j] = (uint32_t)(cur / count);
+        rem = cur % count;
+    }
+    int top = -1;
+    for (int j = n - 1; j >= 0 && top < 0; --j)
+        for (int b = 31; b >= 0; --b)
+            if ((q[j] >> b) & 1u) {
+                top = 32 * j + b;
+                break;
+            }
+    if (top < 0) return 0.0;
+    /* quotient Q = S·2^(149+128)/count; keep 53 bits below and including the top */
+    uint64_t mant = 0;
+    for (int b = 0; b < 53; ++b) {
+        int pos = top - 52 + b;
+        if (pos >= 0 && ((q[pos >> 5] >> (pos & 31)) & 1u)) mant |= 1ull << b;
+    }
+    int round_pos = top - 53;
+    int round_bit = round_pos >= 0 && ((q[round_pos >> 5] >> (round_pos & 31)) & 1u);
+    int sticky = rem != 0;
+    for (int pos = 0; pos < round_pos && !sticky; ++pos)
+        if ((q[pos >> 5] >> (pos & 31)) & 1u) sticky = 1;
+    int e = top - 52 - 149 - 128;
+    if (round_bit && (sticky || (mant & 1ull))) {
+        ++mant;
+        if (mant == (1ull << 53)) {
+            mant >>= 1;
+            ++e;
+        }
+    }
+    return ldexp((double)mant, e);
+}
+
+int orc_absmean_groups(const void* W, int dtype, int64_t N, int64_t K, int64_t group, float* alpha) {
+    if (group < 1) return -1;
+    const int64_t G = (K + group - 1) / group;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            int64_t k0 = g * group, k1 = k0 + group < K ? k0 + group : K;
+            uint64_t limbs[10] = {0};
+            for (int64_t k = k0; k < k1; ++k) {
+                float w = orc_load(W, dtype, n * K + k);
+                uint32_t bits;
+                memcpy(&bits, &w, 4);
+                bits &= 0x7FFFFFFFu;
+                uint32_t e = bits >> 23, sig = bits & 0x7FFFFFu;
+                if (e == 255) return -1;
+                if (e != 0) sig = sig | 0x800000u;
+                /* |w|·2^149 = sig·2^(max(e,1)-1) */
+                uint32_t p = (e != 0 ? e : 1u) - 1u;
+                uint64_t v = (uint64_t)sig << (p & 31u);
+                limbs[p >> 5] += v & 0xFFFFFFFFull;
+                limbs[(p >> 5) + 1] += v >> 32;
+            }
+            for (int j = 0; j + 1 < 10; ++j) {
+                limbs[j + 1] += limbs[j] >> 32;
+                limbs[j] &= 0xFFFFFFFFull;
+            }
+            alpha[n * G + g] = (float)orc_exact_mean(limbs, 10, (uint64_t)(k1 - k0));
+        }
+    }
+    return 0;
+}
+
+/* Codes with one α per group: ŵ = clip(round(W/α_g), -1, 1), as orc_ternarize. */
+int orc_ternarize_groups(const void* W, int dtype, int64_t N, int64_t K, int64_t group, const float* alpha,
+                         int8_t* codes) {
+    const int64_t G = (K + group - 1) / group;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            float qg = orc_load(W, dtype, n * K + k) / alpha[n * G + k / group];
+            if (qg != qg) {
+                codes[n * K + k] = 0;
+                continue;
+            }
+            float rg = rintf(qg);
+            if (rg > 1.0f) rg = 1.0f;
+            if (rg < -1.0f) rg = -1.0f;
+            codes[n * K + k] = (int8_t)rg;
+        }
+    return 0;
+}
+
+/* Product and dequantisation with one α per group: for each group b the
+ * integer sum acc_b = Σ_{k in b} x̃·ŵ (add / subtract / skip), then
+ * S = Σ_b α_b·acc_b in binary64, groups in order (each product is exact);
+ * y = RN32( RN32(S)·s_m ) (+ bias[n]) with s_m = RN32(RN64(β_m / 127)): the
+ * per-token dequantisation of the activations, then the weights' scale, as
+ * [1.58 位大模型] §4.3 scales the product by alpha afterwards. */
+int orc_forward_groups(const int8_t* xq, const float* beta, int64_t M, int64_t K, const int8_t* codes,
+                       const float* alpha, int64_t group, const float* bias, int64_t N, float* y, int threads) {
+    const int64_t G = (K + group - 1) / group;
+    (void)threads;
+#ifdef _OPENMP
+    int nt = threads > 0 ? threads : 1;
+#pragma omp parallel for collapse(2) schedule(static) num_threads(nt)
+#endif
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double sd = (double)beta[m] / 127.0;
+            float s = (float)sd;
+            double S = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t k0 = g * group, k1 = k0 + group < K ? k0 + group : K;
+                int64_t a = 0;
+                for (int64_t k = k0; k < k1; ++k) {
+                    int8_t w = codes[n * K + k];
+                    if (w == 1) a += xq[m * K + k];
+                    else if (w == -1) a -= xq[m * K + k];
+                }
+                S += (double)alpha[n * G + g] * (double)a;
+            }
+            float v = (float)S;
+            v = v * s;
+            if (bias) v = v + bias[n];
+            y[m * N + n] = v;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * 4-bit activations ([BitNet CPU 实测] §2.1: later variants quantise the
+ * activations to 4 bits; §6.2).  The absmax rule of [BitNet 三值权重实战] §2.4
+ * with the 4-bit signed range: β = max|x| + 1e-8, x̃ = clip(round((x·7)/β),
+ * -7, 7).  Stored two per byte: element k in byte k/2, the low nibble for even
+ * k, two's complement; the high nibble of the last byte of an odd-K row is 0.
+ * The dequantisation scale is RN32(RN64(α·β/7)). */
+int orc_quantize_act_a4(const void* x, int dtype, int64_t M, int64_t K, uint8_t* xq4, float* beta) {
+    const int64_t rb = (K + 1) / 2;
+    for (int64_t m = 0; m < M; ++m) {
+        float mx = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(orc_load(x, dtype, m * K + k));
+            if (a > mx) mx = a;
+        }
+        float b4 = mx + 1e-8f;
+        beta[m] = b4;
+        for (int64_t j = 0; j < rb; ++j) xq4[m * rb + j] = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = orc_load(x, dtype, m * K + k) * 7.0f;
+            t = t / b4;
+            float r4 = rintf(t);
+            if (r4 > 7.0f) r4 = 7.0f;
+            if (r4 < -7.0f) r4 = -7.0f;
+            uint8_t nib = (uint8_t)((int)r4 & 0xF);
+            xq4[m * rb + k / 2] |= (uint8_t)(nib << (4 * (k % 2)));
+        }
+    }
+    return 0;
+}
+
+/* Unpacks 4-bit activations [M][ceil(K/2)] into int8 [M][K]. */
+void orc_unpack_a4(const uint8_t* xq4, int64_t M, int64_t K, int8_t* xq) {
+    const int64_t rb = (K + 1) / 2;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            int nib = (xq4[m * rb + k / 2] >> (4 * (k % 2))) & 0xF;
+            xq[m * K + k] = (int8_t)(nib >= 8 ? nib - 16 : nib);
+        }
+}
+
+/* y = fp32(acc)·fp32(α·β_m/7) (+ bias[n]), as orc_dequant with 7 for 127. */
+void orc_dequant_a4(const int32_t* acc, const float* beta, float alpha, const float* bias, int64_t M, int64_t N,
+                    float* y) {
+    for (int64_t m = 0; m < M; ++m) {
+        double s4 = (double)alpha * (double)beta[m];
+        s4 = s4 / 7.0;
+        float s = (float)s4;
+        for (int64_t n = 0; n < N; ++n) {
+            float v = (float)acc[m * N + n];
+            v = v * s;
+            if (bias) v = v + bias[n];
+            y[m * N + n] = v;
+        }
+    }
+}

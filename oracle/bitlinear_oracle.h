@@ -56,6 +56,32 @@ int orc_forward(const void* x, int dtype, int64_t M, int64_t K, const int8_t* co
                 const float* bias, int64_t N, int8_t* xq, float* beta, int32_t* acc, float* y,
                 int threads);
 
+/* Block-diagonal Hadamard rotation of each row (blocks of `block`, a power of
+ * two dividing K) by the binary32 butterfly network, outputs times `scale`. */
+int orc_hadamard(const void* x, int dtype, int64_t M, int64_t K, int64_t block, float scale, float* out);
+
+/* One α per group of `group` consecutive elements of each row of W [N][K]:
+ * alpha[N][ceil(K/group)], exact mean rounded to binary64 then binary32. */
+int orc_absmean_groups(const void* W, int dtype, int64_t N, int64_t K, int64_t group, float* alpha);
+
+/* Ternary codes with one α per group. */
+int orc_ternarize_groups(const void* W, int dtype, int64_t N, int64_t K, int64_t group, const float* alpha,
+                         int8_t* codes);
+
+/* Product and dequantisation with one α per group (see the source). */
+int orc_forward_groups(const int8_t* xq, const float* beta, int64_t M, int64_t K, const int8_t* codes,
+                       const float* alpha, int64_t group, const float* bias, int64_t N, float* y, int threads);
+
+/* Per-token absmax 4-bit quantisation, packed two per byte: xq4[M][ceil(K/2)]. */
+int orc_quantize_act_a4(const void* x, int dtype, int64_t M, int64_t K, uint8_t* xq4, float* beta);
+
+/* Unpacks 4-bit activations into int8 [M][K]. */
+void orc_unpack_a4(const uint8_t* xq4, int64_t M, int64_t K, int8_t* xq);
+
+/* y = fp32(acc)·fp32(α·β_m/7) (+ bias[n]). */
+void orc_dequant_a4(const int32_t* acc, const float* beta, float alpha, const float* bias, int64_t M, int64_t N,
+                    float* y);
+
 #ifdef __cplusplus
 }
 #endif
