@@ -11,7 +11,8 @@ scale granularities and the 4-bit activations ``tests/test_oracle_variants.py``)
 ``dequant``, ``forward``, ``stack_layer``, ``stack_forward``, ``hadamard``,
 ``hadamard_block``, ``quantize_weights_rotated``, ``quantize_act_rotated``,
 ``absmean_groups``, ``ternarize_groups``, ``forward_groups``,
-``quantize_act_a4``, ``unpack_a4``, ``dequant_a4``, ``forward_a4``.  No
+``quantize_act_a4``, ``unpack_a4``, ``dequant_a4``, ``forward_a4``,
+``ste_grad_x``, ``ste_grad_w`` (pins in ``tests/test_oracle_train.py``).  No
 function here is "parity unpinned".
 """
 from __future__ import annotations
@@ -67,6 +68,8 @@ def configure(lib):
     lib.orc_unpack_a4.restype = None
     lib.orc_dequant_a4.argtypes = [p, p, f32, p, i64, i64, p]
     lib.orc_dequant_a4.restype = None
+    lib.orc_ste_grad_x.argtypes = [p, i64, i64, p, i64, f32, p, i32]
+    lib.orc_ste_grad_w.argtypes = [p, i64, i64, p, p, i64, p, i32, f32, p, i32]
     return lib
 
 
@@ -349,3 +352,42 @@ def forward_a4(x: np.ndarray, codes: np.ndarray, alpha, bias: np.ndarray | None 
     K = codes.shape[1]
     acc = ternary_matmul(unpack_a4(xq4, K), codes, threads=threads)
     return xq4, beta, acc, dequant_a4(acc, beta, alpha, bias)
+
+
+# ----------------------------------------------------------------------------- training (STE)
+def ste_grad_x(g: np.ndarray, codes: np.ndarray, alpha, threads: int = 1) -> np.ndarray:
+    """∂L/∂x [M][K] = α·Σ_n g[m][n]·ŵ[n][k] (binary64 sum, one binary32 rounding)
+    ([BitNet 三值权重实战] §3.3: the quantisers pass the gradient straight through)."""
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    M, N = g.shape
+    K = codes.shape[1]
+    out = np.empty((M, K), dtype=np.float32)
+    _load().orc_ste_grad_x(_ptr(g), M, N, _ptr(codes), K, ctypes.c_float(float(np.float32(alpha))), _ptr(out), threads)
+    return out
+
+
+def ste_grad_w(g: np.ndarray, xq: np.ndarray, beta: np.ndarray, W: np.ndarray, alpha, threads: int = 1) -> np.ndarray:
+    """∂L/∂W [N][K] = [|W/α| <= 1]·Σ_m RN32(g[m][n]·s_m)·x̃[m][k] (§3.3, §6.3:
+    no gradient outside the clip range), s_m = RN32(RN64(β_m/127))."""
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    beta = np.ascontiguousarray(beta, dtype=np.float32)
+    W, dt = _as_input(W)
+    M, N = g.shape
+    K = xq.shape[1]
+    out = np.empty((N, K), dtype=np.float32)
+    _load().orc_ste_grad_w(_ptr(g), M, N, _ptr(xq), _ptr(beta), K, _ptr(W), dt,
+                           ctypes.c_float(float(np.float32(alpha))), _ptr(out), threads)
+    return out
+
+
+def train_step(W: np.ndarray, x: np.ndarray, g: np.ndarray, threads: int = 1):
+    """One training step of the layer on latent weights W: the forward with
+    the weights quantised afresh (§4.2, training branch) and the STE backward
+    for the upstream gradient g.  Returns (y, grad_x, grad_W, α, codes, x̃, β)."""
+    alpha = absmean(W)
+    codes = ternarize(W, alpha)
+    xq, beta, acc, y = forward(x, codes, alpha, threads=threads)
+    return (y, ste_grad_x(g, codes, alpha, threads), ste_grad_w(g, xq, beta, W, alpha, threads), alpha, codes,
+            xq, beta)

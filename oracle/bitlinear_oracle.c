@@ -402,3 +402,61 @@ void orc_dequant_a4(const int32_t* acc, const float* beta, float alpha, const fl
         }
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Training with the straight-through estimator ([BitNet 三值权重实战] §3.3,
+ * §6.3; [1.58 位大模型] §3.4).  The forward is the inference arithmetic with
+ * the weights quantised afresh from the latent float weights every step (§4.2,
+ * the training branch).  The backward of y = (x̃·β/127)·(Ŵ·α)ᵀ treats both
+ * quantisers as the identity ("前向量化、反向恒等"), except that a weight
+ * outside the clip range gets no gradient (§6.3): with g = ∂L/∂y,
+ *   ∂L/∂x[m][k] = α · Σ_n g[m][n]·ŵ[n][k]
+ *   ∂L/∂W[n][k] = [ |W[n][k]/α| <= 1 ] · Σ_m g[m][n]·(x̃[m][k]·β_m/127)
+ * with α and β treated as constants.  Arithmetic: the sums in binary64 in
+ * index order, each result rounded once to binary32; W/α is the forward's
+ * binary32 quotient; β_m/127 is s_m = RN32(RN64(β_m/127)) and each product
+ * g·s_m is rounded to binary32 before it multiplies x̃ (exact in binary64). */
+int orc_ste_grad_x(const float* g, int64_t M, int64_t N, const int8_t* codes, int64_t K, float alpha, float* gx,
+                   int threads) {
+    (void)threads;
+#ifdef _OPENMP
+    int nt = threads > 0 ? threads : 1;
+#pragma omp parallel for collapse(2) schedule(static) num_threads(nt)
+#endif
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                int8_t w = codes[n * K + k];
+                if (w == 1) s += (double)g[m * N + n];
+                else if (w == -1) s -= (double)g[m * N + n];
+            }
+            gx[m * K + k] = (float)((double)alpha * s);
+        }
+    return 0;
+}
+
+int orc_ste_grad_w(const float* g, int64_t M, int64_t N, const int8_t* xq, const float* beta, int64_t K,
+                   const void* W, int dtype, float alpha, float* gw, int threads) {
+    (void)threads;
+#ifdef _OPENMP
+    int nt = threads > 0 ? threads : 1;
+#pragma omp parallel for collapse(2) schedule(static) num_threads(nt)
+#endif
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            float q = orc_load(W, dtype, n * K + k) / alpha;
+            if (!(fabsf(q) <= 1.0f)) {  /* outside the clip range (or 0/0): no gradient */
+                gw[n * K + k] = 0.0f;
+                continue;
+            }
+            double s = 0.0;
+            for (int64_t m = 0; m < M; ++m) {
+                double sm = (double)beta[m] / 127.0;
+                float gs = g[m * N + n] * (float)sm;
+                s += (double)gs * (double)xq[m * K + k];
+            }
+            gw[n * K + k] = (float)s;
+        }
+    return 0;
+}

@@ -82,6 +82,13 @@ void orc_unpack_a4(const uint8_t* xq4, int64_t M, int64_t K, int8_t* xq);
 void orc_dequant_a4(const int32_t* acc, const float* beta, float alpha, const float* bias, int64_t M, int64_t N,
                     float* y);
 
+/* Straight-through backward of the BitLinear layer (see the source):
+ * gx[M][K] = α·(g·Ŵ), gw[N][K] = mask ⊙ (gᵀ·x̃·β/127). */
+int orc_ste_grad_x(const float* g, int64_t M, int64_t N, const int8_t* codes, int64_t K, float alpha, float* gx,
+                   int threads);
+int orc_ste_grad_w(const float* g, int64_t M, int64_t N, const int8_t* xq, const float* beta, int64_t K,
+                   const void* W, int dtype, float alpha, float* gw, int threads);
+
 #ifdef __cplusplus
 }
 #endif
