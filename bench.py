@@ -711,6 +711,200 @@ def run_batched_100b(args, world, local_rank):
     }
 
 
+# ----------------------------------------------------------------------------- shared timing
+def time_steps(step, n_rep: int, K: int, stream, props, local_rank, world, dev):
+    """Captures K calls of step(i) (i = 0..K-1, rotating over n_rep weight
+    replicas inside step) in one CUDA graph, settles the clocks for ≈1 s of
+    replays under the sampler, then times one replay with CUDA events on the
+    replay stream.  Returns (ms per step, max over ranks; clocks)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(K):
+            step(i)
+    sampler = settle(stream, g.replay, props, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    t1.synchronize()
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    clocks = sampler.stop()
+    ms = max_over_ranks([t0.elapsed_time(t1) / K], dev, world)[0]
+    del g
+    return ms, clocks
+
+
+def decode_inputs(specs, dev):
+    """bf16 inputs (with outliers) and output buffers of the 7B decode set."""
+    import torch
+    from bitlinear_w1_a8_03_b200 import synth
+    out = []
+    for s in specs:
+        xb = synth.f32_to_bf16_bits(synth.activations(s.x_seed, s.M, s.K, outliers=s.outliers))
+        out.append(dict(x=torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev).view(s.M, s.K),
+                        x_q=torch.empty((s.M, s.K), dtype=torch.int8, device=dev),
+                        beta=torch.empty(s.M, dtype=torch.float32, device=dev),
+                        y=torch.empty((s.M, s.N), dtype=torch.float32, device=dev), N=s.N))
+    return out
+
+
+# ----------------------------------------------------------------------------- rotation leg
+def run_hadamard(args, world, local_rank):
+    """The 7B decode set with the Hadamard rotation before the absmax
+    quantisation ("1.58-bit 大模型极限量化实战" §6.2): weights quantised once from
+    W·H/b (not timed); one step = one bitlinear_linear_grouped call flagged
+    BL_LINEAR_HADAMARD | BL_LINEAR_WEIGHTS_STATIC (the grouped rotate+quantise
+    kernel, then the GEMV, chained by PDL)."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    specs = workload_specs()
+    packed0, alphas = [], []
+    for s in specs:
+        W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+        p, a = bl.bitlinear_quantize_weights_rotated(W, bl.hadamard_block(s.K))
+        packed0.append(p)
+        alphas.append(a)
+        del W
+    torch.cuda.synchronize()
+    set_bytes = sum(p.numel() for p in packed0)
+    replicas = max(2, math.ceil(4 * props.L2_cache_size / set_bytes) + 1)
+    packed = [packed0] + [[p.clone() for p in packed0] for _ in range(replicas - 1)]
+    ins = decode_inputs(specs, dev)
+    arrs = [bl.make_linear_problems([dict(io, W_packed=packed[r][i], alpha=alphas[i]) for i, io in enumerate(ins)])
+            for r in range(replicas)]
+    L = bl.lib()
+    stream = torch.cuda.Stream(device=dev)
+    flags = bl.BL_LINEAR_HADAMARD | bl.BL_LINEAR_WEIGHTS_STATIC
+
+    def step(i):
+        bl.check(L.bitlinear_linear_grouped(arrs[i % replicas], len(specs), bl.BL_BF16, flags, stream.cuda_stream),
+                 "linear")
+
+    K = max(12, args.steps)
+    ms, clocks = time_steps(step, replicas, K, stream, props, local_rank, world, dev)
+    bps = bytes_per_step(specs)
+    peak = float(load_peaks()[0]["hbm_gbs"])
+    gbs = bps / (ms * 1e-3) / 1e9
+    return {"metric": "decode GB/s with the Hadamard rotation before the act quant",
+            "workload": "7B decode layer set, M=1, bf16 x with 0.1% x20 outliers; weights from W*H/b; block = largest "
+                        "power of two dividing K (4096 for K=4096, 256 for K=11008)",
+            "us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
+            "bytes_per_step": bps, "steps": K, "replicas": replicas,
+            "launches_per_step": 2, "clocks": clocks}
+
+
+# ----------------------------------------------------------------------------- scale-granularity leg
+def run_scales(args, world, local_rank):
+    """The 7B decode set with one α per row and one α per 128-block of a row
+    (bitlinear_linear_scaled: grouped act quant, then the scaled GEMV).  The α
+    table (N·ceil(K/group)·4 bytes) counts as weight traffic."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    specs = workload_specs()
+    peak = float(load_peaks()[0]["hbm_gbs"])
+    L = bl.lib()
+    stream = torch.cuda.Stream(device=dev)
+    out = {}
+    for name, group in (("per_row", 1 << 30), ("per_block128", 128)):
+        packed0, alphas = [], []
+        for s in specs:
+            W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+            p, a = bl.bitlinear_quantize_weights_scaled(W, group)
+            packed0.append(p)
+            alphas.append(a)
+            del W
+        torch.cuda.synchronize()
+        set_bytes = sum(p.numel() + 4 * a.numel() for p, a in zip(packed0, alphas))
+        replicas = max(2, math.ceil(4 * props.L2_cache_size / set_bytes) + 1)
+        reps = [(packed0, alphas)] + [([p.clone() for p in packed0], [a.clone() for a in alphas])
+                                      for _ in range(replicas - 1)]
+        ins = decode_inputs(specs, dev)
+        arrs = [bl.make_scaled_problems([dict(io, W_packed=reps[r][0][i], alpha=reps[r][1][i], group=group)
+                                         for i, io in enumerate(ins)]) for r in range(replicas)]
+
+        def step(i):
+            bl.check(L.bitlinear_linear_scaled(arrs[i % replicas], len(specs), bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
+                                               stream.cuda_stream), "linear_scaled")
+
+        K = max(12, args.steps)
+        ms, clocks = time_steps(step, replicas, K, stream, props, local_rank, world, dev)
+        bps = bytes_per_step(specs) + sum(4 * a.numel() for a in alphas)
+        gbs = bps / (ms * 1e-3) / 1e9
+        out[name] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
+                     "bytes_per_step": bps, "alpha_bytes": sum(4 * a.numel() for a in alphas), "steps": K,
+                     "replicas": replicas, "clocks": clocks}
+        del reps, arrs
+    return {"metric": "decode GB/s with one alpha per row / per 128-block",
+            "workload": "7B decode layer set, M=1, bf16 x with outliers; bitlinear_linear_scaled (act quant + scaled "
+                        "GEMV, 2 launches per step)", **out}
+
+
+# ----------------------------------------------------------------------------- 4-bit activation leg
+def run_a4(args, world, local_rank):
+    """The 7B decode set with 4-bit activations: one step = one
+    bitlinear_linear_a4 call (grouped 4-bit act quant, then the CUDA-core
+    product on packed 4-bit x̃), weights flagged static."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    specs = workload_specs()
+    packed0, alphas = [], []
+    for s in specs:
+        W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+        p, a = bl.bitlinear_quantize_weights(W)
+        packed0.append(p)
+        alphas.append(a)
+        del W
+    torch.cuda.synchronize()
+    set_bytes = sum(p.numel() for p in packed0)
+    replicas = max(2, math.ceil(4 * props.L2_cache_size / set_bytes) + 1)
+    packed = [packed0] + [[p.clone() for p in packed0] for _ in range(replicas - 1)]
+    ins = decode_inputs(specs, dev)
+    for io, s in zip(ins, specs):
+        io["x_q"] = torch.empty((s.M, (s.K + 1) // 2), dtype=torch.uint8, device=dev)
+    arrs = [bl.make_linear_a4_problems([dict(io, W_packed=packed[r][i], alpha=alphas[i]) for i, io in enumerate(ins)])
+            for r in range(replicas)]
+    L = bl.lib()
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        bl.check(L.bitlinear_linear_a4(arrs[i % replicas], len(specs), bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
+                                       stream.cuda_stream), "linear_a4")
+
+    K = max(12, args.steps)
+    ms, clocks = time_steps(step, replicas, K, stream, props, local_rank, world, dev)
+    bps = sum(s.N * 16 * ((s.K + 63) // 64) + s.M * s.K * 2 + 2 * s.M * ((s.K + 1) // 2) + 8 * s.M + 4 * s.M * s.N
+              for s in specs)
+    peak = float(load_peaks()[0]["hbm_gbs"])
+    gbs = bps / (ms * 1e-3) / 1e9
+    return {"metric": "decode GB/s with 4-bit activations",
+            "workload": "7B decode layer set, M=1, bf16 x with outliers; bitlinear_linear_a4 (2 launches per step)",
+            "us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
+            "bytes_per_step": bps, "steps": K, "replicas": replicas, "clocks": clocks}
+
+
 # ----------------------------------------------------------------------------- tiny leg
 def run_tiny(args, world, local_rank):
     """Config 1: M = 1, K = N = 256, float32 x and W (seed 0).  A latency line:
@@ -941,9 +1135,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--legs", default="decode,tiny,batched_100b,prefill,stack",
-                    help="comma list: decode (the headline line); tiny, batched_100b, prefill and stack are added "
-                         "under their own keys")
+    ap.add_argument("--legs", default="decode,tiny,batched_100b,prefill,stack,hadamard,scales,a4",
+                    help="comma list: decode (the headline line); tiny, batched_100b, prefill, stack, hadamard, "
+                         "scales and a4 are added under their own keys")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     args = ap.parse_args()
     legs = [x for x in args.legs.split(",") if x]
@@ -980,6 +1174,12 @@ def main():
         result["batched_100b"] = run_batched_100b(args, world, local_rank)
     if "stack" in legs:
         result["stack"] = run_stack(args, world, local_rank)
+    if "hadamard" in legs:
+        result["hadamard"] = run_hadamard(args, world, local_rank)
+    if "scales" in legs:
+        result["scales"] = run_scales(args, world, local_rank)
+    if "a4" in legs:
+        result["a4"] = run_a4(args, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(args)

@@ -28,6 +28,7 @@ STATUS = {
     10: "BL_ERR_FLAGS",
 }
 BL_LINEAR_WEIGHTS_STATIC = 1
+BL_LINEAR_HADAMARD = 2
 
 _lock = threading.Lock()
 _lib = None
@@ -56,6 +57,13 @@ class LinearProblem(ctypes.Structure):
                 ("W_packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("bias", ctypes.c_void_p),
                 ("y", ctypes.c_void_p), ("acc_out", ctypes.c_void_p), ("M", ctypes.c_int64),
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+class ScaledProblem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("x_q", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("W_packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("acc_out", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("group", ctypes.c_int64)]
 
 
 class ActSumProblem(ctypes.Structure):
@@ -87,6 +95,17 @@ def lib():
             L.bitlinear_linear_grouped.argtypes = [ctypes.POINTER(LinearProblem), i32, i32, ctypes.c_uint32, p]
             L.bitlinear_linear_block.argtypes = [ctypes.POINTER(ActSumProblem), i32, ctypes.POINTER(ForwardProblem), i32,
                                                  ctypes.c_uint32, p]
+            L.bitlinear_hadamard_block.argtypes = [i64]
+            L.bitlinear_hadamard_block.restype = i64
+            L.bitlinear_hadamard.argtypes = [p, i32, i64, i64, i64, ctypes.c_float, p, p]
+            L.bitlinear_quantize_act_hadamard.argtypes = [p, i32, i64, i64, i64, p, p, p]
+            L.bitlinear_quantize_weights_scaled.argtypes = [p, i32, i64, i64, i64, p, p, p]
+            L.bitlinear_linear_scaled.argtypes = [ctypes.POINTER(ScaledProblem), i32, i32, ctypes.c_uint32, p]
+            L.bitlinear_quantize_act_a4.argtypes = [p, i32, i64, i64, p, p, p]
+            L.bitlinear_forward_a4.argtypes = [p, p, i64, i64, p, p, i64, p, p, p, p]
+            L.bitlinear_linear_a4.argtypes = [ctypes.POINTER(LinearProblem), i32, i32, ctypes.c_uint32, p]
+            L.bitlinear_train_forward.argtypes = [p, i32, i64, i64, p, i32, i64, p, p, p, p, p, p, sz, p]
+            L.bitlinear_ste_backward.argtypes = [p, i64, i64, i64, p, p, p, p, p, i32, p, p, p]
             L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
             L.bitlinear_selftest_timeout.argtypes = [ctypes.c_uint32, p]
             L.bitlinear_status_string.argtypes = [i32]
@@ -96,7 +115,10 @@ def lib():
                          "bitlinear_quantize_act", "bitlinear_forward",
                          "bitlinear_quantize_act_grouped", "bitlinear_forward_grouped", "bitlinear_linear",
                          "bitlinear_linear_grouped", "bitlinear_linear_block", "bitlinear_device_error",
-                         "bitlinear_selftest_timeout",
+                         "bitlinear_selftest_timeout", "bitlinear_hadamard", "bitlinear_quantize_act_hadamard",
+                         "bitlinear_quantize_weights_scaled", "bitlinear_linear_scaled",
+                         "bitlinear_quantize_act_a4", "bitlinear_forward_a4", "bitlinear_linear_a4",
+                         "bitlinear_train_forward", "bitlinear_ste_backward",
                          "bitlinear_version"):
                 getattr(L, name).restype = i32
             _lib = L
@@ -279,3 +301,160 @@ def bitlinear_device_error() -> int:
     code = ctypes.c_int(0)
     check(lib().bitlinear_device_error(ctypes.byref(code)), "bitlinear_device_error")
     return code.value
+
+
+# ------------------------------------------------------------------ rotation
+def hadamard_block(K: int) -> int:
+    """The block a BL_LINEAR_HADAMARD linear uses for K input features."""
+    return int(lib().bitlinear_hadamard_block(K))
+
+
+def bitlinear_hadamard(x, block: int, scale: float = 1.0, out=None, stream=None):
+    """(x·H)·scale per row in float32 (H block-diagonal Sylvester Hadamard)."""
+    torch = _torch()
+    _need(x, "x")
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    check(lib().bitlinear_hadamard(_ptr(x), _dtype_code(x), M, K, block, scale, _ptr(out), _stream(stream)),
+          "bitlinear_hadamard")
+    return out
+
+
+def bitlinear_quantize_act_hadamard(x, block: int, x_q=None, beta=None, stream=None):
+    """Per-token int8 quantisation of x·H: (x_q int8 [M][K], beta float32 [M])."""
+    torch = _torch()
+    _need(x, "x")
+    M, K = x.shape
+    if x_q is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if beta is None:
+        beta = torch.empty(M, dtype=torch.float32, device=x.device)
+    check(lib().bitlinear_quantize_act_hadamard(_ptr(x), _dtype_code(x), M, K, block, _ptr(x_q), _ptr(beta),
+                                                _stream(stream)), "bitlinear_quantize_act_hadamard")
+    return x_q, beta
+
+
+def bitlinear_quantize_weights_rotated(W, block: int | None = None, stream=None):
+    """Weights of a rotated layer: W' = W·H/block (float32, on the device), then
+    the absmean quantisation of W'.  Returns (W_packed, alpha)."""
+    K = W.shape[1]
+    block = hadamard_block(K) if block is None else block
+    Wr = bitlinear_hadamard(W, block, 1.0 / block, stream=stream)
+    out = bitlinear_quantize_weights(Wr, stream=stream)
+    del Wr
+    return out
+
+
+# ------------------------------------------------------------------ scale granularity
+def bitlinear_quantize_weights_scaled(W, group: int, W_packed=None, alpha=None, stream=None):
+    """One α per group of `group` input features of each row (group >= K: per
+    row).  Returns (W_packed uint8 [N][16·ceil(K/64)], alpha float32 [N][G])."""
+    torch = _torch()
+    _need(W, "W")
+    N, K = W.shape
+    G = 1 if group >= K else -(-K // group)
+    if W_packed is None:
+        W_packed = torch.empty((N, packed_row_bytes(K)), dtype=torch.uint8, device=W.device)
+    if alpha is None:
+        alpha = torch.empty((N, G), dtype=torch.float32, device=W.device)
+    check(lib().bitlinear_quantize_weights_scaled(_ptr(W), _dtype_code(W), N, K, group, _ptr(W_packed), _ptr(alpha),
+                                                  _stream(stream)), "bitlinear_quantize_weights_scaled")
+    return W_packed, alpha
+
+
+def make_scaled_problems(problems):
+    """ctypes array for bitlinear_linear_scaled from dicts with keys x_q, beta,
+    W_packed, alpha, group, N, y and optional x, bias, acc_out."""
+    arr = (ScaledProblem * len(problems))()
+    for i, p in enumerate(problems):
+        M, K = p["x_q"].shape
+        arr[i] = ScaledProblem(_ptr(p.get("x")), _ptr(p["x_q"]), _ptr(p["beta"]), _ptr(p["W_packed"]),
+                               _ptr(p["alpha"]), _ptr(p.get("bias")), _ptr(p["y"]), _ptr(p.get("acc_out")), M, p["N"],
+                               K, p["group"])
+    return arr
+
+
+def bitlinear_linear_scaled(problems, dtype_code: int = BL_BF16, flags: int = 0, stream=None):
+    """Linears with one α per group (see make_scaled_problems)."""
+    arr = problems if isinstance(problems, ctypes.Array) else make_scaled_problems(problems)
+    check(lib().bitlinear_linear_scaled(arr, len(arr), dtype_code, flags, _stream(stream)), "bitlinear_linear_scaled")
+
+
+# ------------------------------------------------------------------ 4-bit activations
+def bitlinear_quantize_act_a4(x, x_q4=None, beta=None, stream=None):
+    """x [M][K] -> (x_q4 uint8 [M][ceil(K/2)] packed 4-bit, beta float32 [M])."""
+    torch = _torch()
+    _need(x, "x")
+    M, K = x.shape
+    if x_q4 is None:
+        x_q4 = torch.empty((M, (K + 1) // 2), dtype=torch.uint8, device=x.device)
+    if beta is None:
+        beta = torch.empty(M, dtype=torch.float32, device=x.device)
+    check(lib().bitlinear_quantize_act_a4(_ptr(x), _dtype_code(x), M, K, _ptr(x_q4), _ptr(beta), _stream(stream)),
+          "bitlinear_quantize_act_a4")
+    return x_q4, beta
+
+
+def bitlinear_forward_a4(x_q4, beta, K: int, W_packed, alpha, N: int, bias=None, y=None, acc_out=None, stream=None):
+    """y [M][N] = fp32(x̃·Ŵᵀ)·(α·β/7) (+ bias) on packed 4-bit activations."""
+    torch = _torch()
+    M = x_q4.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x_q4.device)
+    check(lib().bitlinear_forward_a4(_ptr(x_q4), _ptr(beta), M, K, _ptr(W_packed), _ptr(alpha), N, _ptr(bias), _ptr(y),
+                                     _ptr(acc_out), _stream(stream)), "bitlinear_forward_a4")
+    return y
+
+
+def make_linear_a4_problems(problems):
+    """ctypes array for bitlinear_linear_a4: dicts as for make_linear_problems,
+    with x_q a packed uint8 [M][ceil(K/2)] buffer."""
+    arr = (LinearProblem * len(problems))()
+    for i, p in enumerate(problems):
+        M, K = p["x"].shape
+        arr[i] = LinearProblem(_ptr(p["x"]), _ptr(p["x_q"]), _ptr(p["beta"]), _ptr(p["W_packed"]), _ptr(p["alpha"]),
+                               _ptr(p.get("bias")), _ptr(p["y"]), _ptr(p.get("acc_out")), M, p["N"], K)
+    return arr
+
+
+def bitlinear_linear_a4(problems, dtype_code: int = BL_BF16, flags: int = 0, stream=None):
+    arr = problems if isinstance(problems, ctypes.Array) else make_linear_a4_problems(problems)
+    check(lib().bitlinear_linear_a4(arr, len(arr), dtype_code, flags, _stream(stream)), "bitlinear_linear_a4")
+
+
+# ------------------------------------------------------------------ training (straight-through estimator)
+def bitlinear_train_forward(W, x, W_packed=None, alpha=None, x_q=None, beta=None, y=None, workspace=None, stream=None):
+    """Forward of a training step on latent weights W [N][K]: quantise W, then
+    the linear on x [M][K].  Returns (y, W_packed, alpha, x_q, beta)."""
+    torch = _torch()
+    _need(W, "W")
+    _need(x, "x")
+    N, K = W.shape
+    M = x.shape[0]
+    dev = W.device
+    W_packed = torch.empty((N, packed_row_bytes(K)), dtype=torch.uint8, device=dev) if W_packed is None else W_packed
+    alpha = torch.empty(1, dtype=torch.float32, device=dev) if alpha is None else alpha
+    x_q = torch.empty((M, K), dtype=torch.int8, device=dev) if x_q is None else x_q
+    beta = torch.empty(M, dtype=torch.float32, device=dev) if beta is None else beta
+    y = torch.empty((M, N), dtype=torch.float32, device=dev) if y is None else y
+    ws = int(lib().bitlinear_quantize_weights_workspace_bytes(N, K))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 8), dtype=torch.uint8, device=dev)
+    check(lib().bitlinear_train_forward(_ptr(W), _dtype_code(W), N, K, _ptr(x), _dtype_code(x), M, _ptr(W_packed),
+                                        _ptr(alpha), _ptr(x_q), _ptr(beta), _ptr(y), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)), "bitlinear_train_forward")
+    return y, W_packed, alpha, x_q, beta
+
+
+def bitlinear_ste_backward(g, W_packed, alpha, x_q, beta, W, grad_x=True, grad_W=True, stream=None):
+    """Straight-through backward for g = ∂L/∂y [M][N]: returns (grad_x [M][K] or
+    None, grad_W [N][K] or None)."""
+    torch = _torch()
+    M, N = g.shape
+    K = W.shape[1]
+    gx = torch.empty((M, K), dtype=torch.float32, device=g.device) if grad_x is True else (grad_x or None)
+    gw = torch.empty((N, K), dtype=torch.float32, device=g.device) if grad_W is True else (grad_W or None)
+    check(lib().bitlinear_ste_backward(_ptr(g), M, N, K, _ptr(W_packed), _ptr(alpha), _ptr(x_q), _ptr(beta), _ptr(W),
+                                       _dtype_code(W), _ptr(gx), _ptr(gw), _stream(stream)), "bitlinear_ste_backward")
+    return gx, gw

@@ -210,7 +210,8 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     if (!problems) return BL_ERR_NULL;
     if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
     if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
-    if (flags & ~(uint32_t)BL_LINEAR_WEIGHTS_STATIC) return BL_ERR_FLAGS;
+    if (flags & ~(uint32_t)(BL_LINEAR_WEIGHTS_STATIC | BL_LINEAR_HADAMARD)) return BL_ERR_FLAGS;
+    const bool rotate = (flags & BL_LINEAR_HADAMARD) != 0;
     bitlinear_act_problem act[BITLINEAR_MAX_GROUP];
     bitlinear_forward_problem fwd[BITLINEAR_MAX_GROUP];
     int64_t rows = 0;
@@ -222,6 +223,7 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
         if (st == BL_OK) st = check_forward(fwd[i]);
         if (st != BL_OK) return st;
         if (misaligned(q.x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+        if (rotate && bitlinear_hadamard_block(q.K) < 2) return BL_ERR_SHAPE;
         rows += q.M;
     }
     if (rows >= kMaxRows) return BL_ERR_SHAPE;
@@ -229,6 +231,17 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     if (st != BL_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    if (rotate) {
+        // rotation + quantisation in one grouped launch, then the product
+        // (the product kernel streams weights early only under the flag)
+        bl::HadJob jobs[BITLINEAR_MAX_GROUP];
+        for (int i = 0; i < count; ++i)
+            jobs[i] = bl::HadJob{problems[i].x, nullptr, problems[i].x_q, problems[i].beta, problems[i].M,
+                                 problems[i].K, (int)bitlinear_hadamard_block(problems[i].K), 1.0f};
+        st = from_cuda(bl::launch_hadamard(jobs, count, dtype, s, true));
+        if (st != BL_OK) return st;
+        return from_cuda(bl::launch_forward(fwd, count, s, true));
+    }
     // few tokens: one launch that quantises in the product kernel's prologue
     bl::FusedInput fin[BITLINEAR_MAX_GROUP];
     for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
@@ -306,6 +319,190 @@ bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, i
     return BL_OK;
 }
 
+int64_t bitlinear_hadamard_block(int64_t K) {
+    if (K < 1) return 0;
+    int64_t b = 1;
+    while (K % (2 * b) == 0 && 2 * b <= BITLINEAR_MAX_HADAMARD_BLOCK) b *= 2;
+    return b;
+}
+
+static bitlinear_status check_hadamard(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K, int64_t block) {
+    if (!x) return BL_ERR_NULL;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (M < 1 || K < 1 || K > BITLINEAR_MAX_K || M > kMaxRows) return BL_ERR_SHAPE;
+    if (block < 1 || (block & (block - 1)) != 0 || block > BITLINEAR_MAX_HADAMARD_BLOCK || K % block != 0)
+        return BL_ERR_SHAPE;
+    if (block > bl::hadamard_max_block()) return BL_ERR_SHAPE;
+    if (misaligned(x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+    return BL_OK;
+}
+
+bitlinear_status bitlinear_hadamard(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K, int64_t block,
+                                    float scale, float* out, bitlinear_stream_t stream) {
+    bitlinear_status st = check_hadamard(x, dtype, M, K, block);
+    if (st != BL_OK) return st;
+    if (!out) return BL_ERR_NULL;
+    if (misaligned(out, 4)) return BL_ERR_ALIGN;
+    st = check_device();
+    if (st != BL_OK) return st;
+    bl::HadJob job{x, out, nullptr, nullptr, M, K, (int)block, scale};
+    return from_cuda(bl::launch_hadamard(&job, 1, dtype, reinterpret_cast<cudaStream_t>(stream), false));
+}
+
+bitlinear_status bitlinear_quantize_act_hadamard(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K,
+                                                 int64_t block, int8_t* x_q, float* beta, bitlinear_stream_t stream) {
+    bitlinear_status st = check_hadamard(x, dtype, M, K, block);
+    if (st != BL_OK) return st;
+    if (!x_q || !beta) return BL_ERR_NULL;
+    if (misaligned(beta, 4)) return BL_ERR_ALIGN;
+    st = check_device();
+    if (st != BL_OK) return st;
+    bl::HadJob job{x, nullptr, x_q, beta, M, K, (int)block, 1.0f};
+    return from_cuda(bl::launch_hadamard(&job, 1, dtype, reinterpret_cast<cudaStream_t>(stream), false));
+}
+
+static bool valid_group(int64_t K, int64_t group) { return group >= K || (group > 0 && group % 64 == 0); }
+
+bitlinear_status bitlinear_quantize_weights_scaled(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K,
+                                                   int64_t group, uint8_t* W_packed, float* alpha,
+                                                   bitlinear_stream_t stream) {
+    if (!W || !W_packed || !alpha) return BL_ERR_NULL;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (N < 1 || K < 1 || K > BITLINEAR_MAX_K || N > kMaxWeights / K || !valid_group(K, group)) return BL_ERR_SHAPE;
+    if (misaligned(W_packed, 16) || misaligned(alpha, 4) || misaligned(W, dtype == BL_F32 ? 4 : 2))
+        return BL_ERR_ALIGN;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_quantize_weights_groups(W, dtype, N, K, group >= K ? K : group, W_packed, alpha,
+                                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bitlinear_status bitlinear_linear_scaled(const bitlinear_scaled_problem* problems, int count, bitlinear_dtype dtype,
+                                         uint32_t flags, bitlinear_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (flags & ~(uint32_t)BL_LINEAR_WEIGHTS_STATIC) return BL_ERR_FLAGS;
+    bitlinear_act_problem act[BITLINEAR_MAX_GROUP];
+    bl::ScaledProblem fwd[BITLINEAR_MAX_GROUP];
+    int nact = 0;
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_scaled_problem& q = problems[i];
+        bitlinear_forward_problem f{q.x_q, q.beta, q.W_packed, q.alpha, q.bias, q.y, q.acc_out, q.M, q.N, q.K};
+        bitlinear_status st = check_forward(f);
+        if (st != BL_OK) return st;
+        if (!valid_group(q.K, q.group) || (q.acc_out && q.group < q.K)) return BL_ERR_SHAPE;
+        if (q.x) {
+            act[nact] = bitlinear_act_problem{q.x, q.x_q, q.beta, q.M, q.K};
+            st = check_act(act[nact]);
+            if (st != BL_OK) return st;
+            if (misaligned(q.x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+            ++nact;
+            rows += q.M;
+        }
+        fwd[i] = bl::ScaledProblem{q.x_q, q.beta, q.W_packed, q.alpha, q.bias, q.y, q.acc_out, q.M, q.N, q.K,
+                                   q.group >= q.K ? q.K : q.group};
+    }
+    if (rows >= kMaxRows) return BL_ERR_SHAPE;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    if (nact > 0) {
+        st = from_cuda(bl::launch_quantize_act(act, nact, dtype, s, true, weights_static));
+        if (st != BL_OK) return st;
+    }
+    return from_cuda(bl::launch_forward_scaled(fwd, count, s, nact > 0 || weights_static));
+}
+
+bitlinear_status bitlinear_quantize_act_a4(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K, uint8_t* x_q4,
+                                           float* beta, bitlinear_stream_t stream) {
+    bitlinear_act_problem p{x, reinterpret_cast<int8_t*>(x_q4), beta, M, K};
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    bitlinear_status st = check_act(p);
+    if (st != BL_OK) return st;
+    if (misaligned(x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+    st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_quantize_act_a4(&p, 1, dtype, reinterpret_cast<cudaStream_t>(stream), false));
+}
+
+bitlinear_status bitlinear_forward_a4(const uint8_t* x_q4, const float* beta, int64_t M, int64_t K,
+                                      const uint8_t* W_packed, const float* alpha, int64_t N, const float* bias,
+                                      float* y, int32_t* acc_out, bitlinear_stream_t stream) {
+    bitlinear_forward_problem p{reinterpret_cast<const int8_t*>(x_q4), beta, W_packed, alpha, bias, y, acc_out, M, N, K};
+    bitlinear_status st = check_forward(p);
+    if (st != BL_OK) return st;
+    st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_forward_a4(&p, 1, reinterpret_cast<cudaStream_t>(stream), false));
+}
+
+bitlinear_status bitlinear_linear_a4(const bitlinear_linear_problem* problems, int count, bitlinear_dtype dtype,
+                                     uint32_t flags, bitlinear_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (flags & ~(uint32_t)BL_LINEAR_WEIGHTS_STATIC) return BL_ERR_FLAGS;
+    bitlinear_act_problem act[BITLINEAR_MAX_GROUP];
+    bitlinear_forward_problem fwd[BITLINEAR_MAX_GROUP];
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_linear_problem& q = problems[i];
+        act[i] = bitlinear_act_problem{q.x, q.x_q, q.beta, q.M, q.K};
+        fwd[i] = bitlinear_forward_problem{q.x_q, q.beta, q.W_packed, q.alpha, q.bias, q.y, q.acc_out, q.M, q.N, q.K};
+        bitlinear_status st = check_act(act[i]);
+        if (st == BL_OK) st = check_forward(fwd[i]);
+        if (st != BL_OK) return st;
+        if (misaligned(q.x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+        rows += q.M;
+    }
+    if (rows >= kMaxRows) return BL_ERR_SHAPE;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = from_cuda(bl::launch_quantize_act_a4(act, count, dtype, s, true));
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_forward_a4(fwd, count, s, true));
+}
+
+bitlinear_status bitlinear_train_forward(const void* W, bitlinear_dtype w_dtype, int64_t N, int64_t K, const void* x,
+                                         bitlinear_dtype x_dtype, int64_t M, uint8_t* W_packed, float* alpha,
+                                         int8_t* x_q, float* beta, float* y, void* workspace, size_t workspace_bytes,
+                                         bitlinear_stream_t stream) {
+    // validate both steps before launching either
+    if (!x || !x_q || !beta || !y) return BL_ERR_NULL;
+    if (!valid_dtype(x_dtype)) return BL_ERR_DTYPE;
+    bitlinear_act_problem a{x, x_q, beta, M, K};
+    bitlinear_status st = check_act(a);
+    if (st != BL_OK) return st;
+    if (misaligned(x, x_dtype == BL_F32 ? 4 : 2) || misaligned(y, 4)) return BL_ERR_ALIGN;
+    st = bitlinear_quantize_weights(W, w_dtype, N, K, W_packed, alpha, workspace, workspace_bytes, stream);
+    if (st != BL_OK) return st;
+    bitlinear_linear_problem p{x, x_q, beta, W_packed, alpha, nullptr, y, nullptr, M, N, K};
+    return bitlinear_linear_grouped(&p, 1, x_dtype, 0u, stream);
+}
+
+bitlinear_status bitlinear_ste_backward(const float* g, int64_t M, int64_t N, int64_t K, const uint8_t* W_packed,
+                                        const float* alpha, const int8_t* x_q, const float* beta, const void* W,
+                                        bitlinear_dtype w_dtype, float* grad_x, float* grad_W,
+                                        bitlinear_stream_t stream) {
+    if (!g || !alpha) return BL_ERR_NULL;
+    if (grad_x && !W_packed) return BL_ERR_NULL;
+    if (grad_W && (!x_q || !beta || !W)) return BL_ERR_NULL;
+    if (grad_W && !valid_dtype(w_dtype)) return BL_ERR_DTYPE;
+    if (M < 1 || N < 1 || K < 1 || K > BITLINEAR_MAX_K || M > kMaxRows || N > kMaxRows || N > kMaxWeights / K)
+        return BL_ERR_SHAPE;
+    if (misaligned(g, 4) || misaligned(alpha, 4) || misaligned(grad_x, 4) || misaligned(grad_W, 4) ||
+        misaligned(beta, 4) || (grad_W && misaligned(W, w_dtype == BL_F32 ? 4 : 2)))
+        return BL_ERR_ALIGN;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    return from_cuda(bl::launch_ste_backward(g, M, N, K, W_packed, alpha, x_q, beta, W, w_dtype, grad_x, grad_W,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
 bitlinear_status bitlinear_device_error(int* code) {
     if (!code) return BL_ERR_NULL;
     bitlinear_status st = check_device();
@@ -340,6 +537,6 @@ const char* bitlinear_status_string(bitlinear_status status) {
     return "unknown status";
 }
 
-int bitlinear_version(void) { return 100; }
+int bitlinear_version(void) { return 101; }
 
 }  // extern "C"

@@ -82,4 +82,38 @@ __device__ __forceinline__ int8_t quantize_one(float v, float beta, float rbeta)
     return (int8_t)__float2int_rn(r);
 }
 
+// clip(rint(RN(RN(7·v) / β)), -7, 7): the 4-bit variant of quantize_one, with
+// the same argument (|a/β| <= 7·(1 + 2^-24), so q = RN(a·RN(1/β)) is within
+// 7·2^-23 of a/β; away from half-integers by more than 1e-4 both round alike,
+// otherwise the correctly rounded quotient is taken).
+__device__ __forceinline__ int quantize_one_a4(float v, float beta, float rbeta) {
+    const float a = __fmul_rn(v, 7.0f);
+    const float q = __fmul_rn(a, rbeta);
+    float r = rintf(q);
+    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) r = rintf(__fdiv_rn(a, beta));
+    r = fminf(fmaxf(r, -7.0f), 7.0f);
+    return __float2int_rn(r);
+}
+
+// Dequantisation scale of one token for 4-bit activations: RN32(RN64(α·β / 7)).
+__device__ __forceinline__ float dequant_scale_a4(float alpha, float beta) {
+    double s = __dmul_rn((double)alpha, (double)beta);
+    s = __ddiv_rn(s, 7.0);
+    return __double2float_rn(s);
+}
+
+// Eight 4-bit activations (two's complement nibbles, element 2i in the low
+// nibble of byte i) as two words of four int8: the nibbles are spread to bytes
+// and sign-extended without borrows between bytes: ((u ^ 8) | 0x80) - 8, then ^ 0x80.
+__device__ __forceinline__ void unpack_a4(uint32_t w, uint32_t& lo4, uint32_t& hi4) {
+    const uint32_t even = w & 0x0F0F0F0Fu;         // elements 0, 2, 4, 6
+    const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;   // elements 1, 3, 5, 7
+    uint32_t a = __byte_perm(even, odd, 0x5140);   // 0, 1, 2, 3
+    uint32_t b = __byte_perm(even, odd, 0x7362);   // 4, 5, 6, 7
+    a = (((a ^ 0x08080808u) | 0x80808080u) - 0x08080808u) ^ 0x80808080u;
+    b = (((b ^ 0x08080808u) | 0x80808080u) - 0x08080808u) ^ 0x80808080u;
+    lo4 = a;
+    hi4 = b;
+}
+
 }  // namespace bl

@@ -39,9 +39,18 @@ cudaError_t launch_quantize_act_jobs(const ActJob* jobs, int count, bitlinear_dt
 cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
                                 cudaStream_t stream, bool pdl = false, bool early_trigger = false);
 
+// 4-bit activations: x_q of each problem is packed [M][ceil(K/2)] (two per byte).
+cudaError_t launch_quantize_act_a4(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
+                                   cudaStream_t stream, bool pdl);
+
 size_t quantize_weights_workspace_bytes(int64_t N, int64_t K);
 cudaError_t launch_quantize_weights(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K, uint8_t* W_packed,
                                     float* alpha, void* workspace, cudaStream_t stream);
+
+// One α per group of `group` consecutive elements of each row (group a
+// multiple of 16, or >= K for one per row): alpha [N][ceil(K/group)].
+cudaError_t launch_quantize_weights_groups(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K, int64_t group,
+                                           uint8_t* W_packed, float* alpha, cudaStream_t stream);
 
 // Allocation-free weight quantisation: scratch in a static device array.
 size_t quantize_weights_static_scratch_bytes();
@@ -67,6 +76,44 @@ struct FusedInput {
 // fused kernel; the caller then runs the quantisation and product separately.
 cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
                                 bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched);
+
+// Hadamard rotation (out = x·H·scale) or rotation + per-token int8
+// quantisation (x_q, beta), one job per problem of a grouped launch; all jobs
+// of a launch are of one kind (x_q set on all, or on none) and one dtype.
+struct HadJob {
+    const void* x;
+    float* out;
+    int8_t* x_q;
+    float* beta;
+    int64_t M, K;
+    int block;    // power of two dividing K, at most hadamard_max_block()
+    float scale;  // rotation only
+};
+int hadamard_max_block();
+cudaError_t launch_hadamard(const HadJob* jobs, int count, bitlinear_dtype dtype, cudaStream_t stream, bool pdl);
+
+// Product with one α per group of `group` input features of a row (group >= K:
+// one per row), alpha [N][ceil(K/group)]; any M (four tokens per pass).
+struct ScaledProblem {
+    const int8_t* x_q;
+    const float* beta;
+    const uint8_t* W_packed;
+    const float* alpha;
+    const float* bias;
+    float* y;
+    int32_t* acc_out;  // one α per row only
+    int64_t M, N, K, group;
+};
+cudaError_t launch_forward_scaled(const ScaledProblem* problems, int count, cudaStream_t stream, bool pdl);
+// Product on 4-bit activations (x_q packed [M][ceil(K/2)]), one α for the
+// tensor: y = fp32(acc)·RN32(RN64(α·β/7)) (+ bias).
+cudaError_t launch_forward_a4(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl);
+
+// Straight-through backward: grad_x [M][K] = α·(g·Ŵ), grad_W [N][K] = clip mask ⊙
+// ((g·s)ᵀ·x̃); either output may be NULL.
+cudaError_t launch_ste_backward(const float* g, int64_t M, int64_t N, int64_t K, const uint8_t* W_packed,
+                                const float* alpha, const int8_t* x_q, const float* beta, const void* W,
+                                bitlinear_dtype w_dtype, float* grad_x, float* grad_W, cudaStream_t stream);
 
 // Tensor-core GEMM for many tokens (tcgen05, int8): all problems in one launch.
 bool gemm_tc_supported(const bitlinear_forward_problem& p);

@@ -218,10 +218,15 @@ cudaError_t launch_hadamard(const HadJob* jobs, int count, bitlinear_dtype dtype
         bmax = jobs[i].block > bmax ? jobs[i].block : bmax;
     }
     P.row_begin[count] = rows;
-    // threads: enough for one tile of the longest row, a multiple of 32
+    // threads: enough for one tile of the longest row, a multiple of 32 and
+    // of bmax / kE, so that a tile holds whole blocks of every problem (the
+    // shared-memory pair passes stay inside the tile); at most kMaxThreads,
+    // whose tile (kTile, a multiple of every block) then takes several passes
+    const int64_t step = bmax / kE > 32 ? bmax / kE : 32;
     int64_t want = (kmax + kE - 1) / kE;
+    want = (want + step - 1) / step * step;
     if (want > kMaxThreads) want = kMaxThreads;
-    const int threads = (int)((want + 31) / 32 * 32);
+    const int threads = (int)want;
     const size_t smem = bmax > 32 * kE ? (size_t)threads * kE * sizeof(float) : 0;
     const bool quant = jobs[0].x_q != nullptr;
     const void* kernel;

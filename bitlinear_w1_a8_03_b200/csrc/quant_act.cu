@@ -207,7 +207,62 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
     }
 }
 
+// Per-token absmax 4-bit quantisation ("BitNet CPU 实测", cf-1.com/news/5800143
+// §2.1: later variants quantise the activations to 4 bits): β = max|x| + 1e-8,
+// x̃ = clip(round((x·7)/β), -7, 7), two per byte (element k in byte k/2, the
+// low nibble for even k; the high nibble of an odd row's last byte is 0).
+// One CTA per row: absmax, then each thread quantises element pairs.
+template <typename T>
+__global__ void __launch_bounds__(kMaxThreads) act_quant_a4_kernel(const __grid_constant__ ActParams P) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int64_t row = blockIdx.x;
+    int pi = 0;
+    while (pi + 1 < P.count && row >= P.row_begin[pi + 1]) ++pi;
+    const ActJob& pr = P.p[pi];
+    const int64_t m = row - P.row_begin[pi];
+    const int64_t K = pr.K;
+    const T* x = static_cast<const T*>(pr.a) + m * K;
+    const int64_t rb = (K + 1) / 2;
+    uint8_t* q = reinterpret_cast<uint8_t*>(pr.x_q) + m * rb;
+    float mx = 0.0f;
+    for (int64_t i = threadIdx.x; i < K; i += blockDim.x) mx = fmaxf(mx, fabsf(load_as_f32(x, i)));
+    const float beta = __fadd_rn(block_max(mx), 1e-8f);
+    const float rbeta = __frcp_rn(beta);
+    if (threadIdx.x == 0) pr.beta[m] = beta;
+    for (int64_t j = threadIdx.x; j < rb; j += blockDim.x) {
+        const int lo = quantize_one_a4(load_as_f32(x, 2 * j), beta, rbeta);
+        const int hi = 2 * j + 1 < K ? quantize_one_a4(load_as_f32(x, 2 * j + 1), beta, rbeta) : 0;
+        q[j] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_act_a4(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
+                                   cudaStream_t stream, bool pdl) {
+    ActParams P{};
+    P.count = count;
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) {
+        P.p[i] = ActJob{problems[i].x, nullptr, nullptr, problems[i].x_q, problems[i].beta, problems[i].M,
+                        problems[i].K};
+        P.row_begin[i] = rows;
+        rows += problems[i].M;
+    }
+    P.row_begin[count] = rows;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)rows);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (dtype == BL_BF16) return cudaLaunchKernelEx(&cfg, act_quant_a4_kernel<uint16_t>, P);
+    return cudaLaunchKernelEx(&cfg, act_quant_a4_kernel<float>, P);
+}
 
 cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count, bitlinear_dtype dtype,
                                 cudaStream_t stream, bool pdl, bool early_trigger) {

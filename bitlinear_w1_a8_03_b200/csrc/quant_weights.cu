@@ -118,20 +118,9 @@ __device__ uint64_t extract_bits(const uint32_t* q, int nlimbs, int lo, int n) {
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads) absmean_finalize_kernel(const unsigned long long* __restrict__ partials,
-                                                                    int nparts, int64_t count,
-                                                                    float* __restrict__ alpha) {
-    uint64_t acc[kLimbs];
-#pragma unroll
-    for (int j = 0; j < kLimbs; ++j) acc[j] = 0;
-    for (int g = threadIdx.x; g < nparts; g += kThreads) {
-#pragma unroll
-        for (int j = 0; j < kLimbs; ++j) acc[j] += partials[(int64_t)g * kLimbs + j];
-    }
-    block_sum(acc);
-    if (threadIdx.x != 0) return;
-
-    // T = S·2^128 (S = 2^149·Σ|W| as 32-bit limbs); Q = floor(T / count), R = T mod count.
+// RN32(RN64(S / count)) for S·2^149 = acc (normalised 32-bit digits in
+// 64-bit lanes).  T = S·2^128; Q = floor(T / count), R = T mod count.
+__device__ float limbs_mean(const uint64_t (&acc)[kLimbs], int64_t count) {
     constexpr int kT = kLimbs + 4;
     uint32_t t[kT], q[kT];
     for (int j = 0; j < 4; ++j) t[j] = 0;
@@ -146,10 +135,7 @@ __global__ void __launch_bounds__(kThreads) absmean_finalize_kernel(const unsign
     int top = -1;
     for (int j = kT - 1; j >= 0 && top < 0; --j)
         if (q[j] != 0) top = 32 * j + 31 - __clz(q[j]);
-    if (top < 0) {  // Σ|W| = 0
-        *alpha = 0.0f;
-        return;
-    }
+    if (top < 0) return 0.0f;  // Σ|W| = 0
     // mean = (Q + R/count)·2^-277.  Round Q to 53 significant bits, half to even;
     // S >= 1 gives Q >= 2^88, so top >= 88 and all shifts below are valid.
     uint64_t mant = extract_bits(q, kT, top - 52, 53);
@@ -166,7 +152,51 @@ __global__ void __launch_bounds__(kThreads) absmean_finalize_kernel(const unsign
         }
     }
     const double mean = ldexp((double)mant, e);  // exact: a normal binary64
-    *alpha = __double2float_rn(mean);
+    return __double2float_rn(mean);
+}
+
+__global__ void __launch_bounds__(kThreads) absmean_finalize_kernel(const unsigned long long* __restrict__ partials,
+                                                                    int nparts, int64_t count,
+                                                                    float* __restrict__ alpha) {
+    uint64_t acc[kLimbs];
+#pragma unroll
+    for (int j = 0; j < kLimbs; ++j) acc[j] = 0;
+    for (int g = threadIdx.x; g < nparts; g += kThreads) {
+#pragma unroll
+        for (int j = 0; j < kLimbs; ++j) acc[j] += partials[(int64_t)g * kLimbs + j];
+    }
+    block_sum(acc);
+    if (threadIdx.x != 0) return;
+    *alpha = limbs_mean(acc, count);
+}
+
+// One α per group of `group` consecutive elements of each row (the last group
+// of a row may be shorter): the same exact mean as for the tensor, one warp
+// per group, the limb vectors of the lanes summed by shuffles.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) absmean_groups_kernel(const T* __restrict__ W, int64_t N, int64_t K,
+                                                                  int64_t group, float* __restrict__ alpha) {
+    const int lane = threadIdx.x & 31;
+    const int64_t G = (K + group - 1) / group;
+    const int64_t warp0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
+    for (int64_t gi = warp0; gi < N * G; gi += nwarps) {
+        const int64_t n = gi / G, g = gi - n * G;
+        const int64_t k0 = g * group, k1 = min(K, k0 + group);
+        uint64_t acc[kLimbs];
+#pragma unroll
+        for (int j = 0; j < kLimbs; ++j) acc[j] = 0;
+        for (int64_t k = k0 + lane; k < k1; k += 32) add_abs(acc, load_as_f32(W + n * K, k));
+        normalize(acc);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int j = 0; j < kLimbs; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        if (lane == 0) {
+            normalize(acc);
+            alpha[gi] = limbs_mean(acc, k1 - k0);
+        }
+    }
 }
 
 __device__ __forceinline__ uint32_t ternary_code(float w, float alpha) {
@@ -179,11 +209,14 @@ __device__ __forceinline__ uint32_t ternary_code(float w, float alpha) {
 
 // One thread per packed 32-bit word (16 weights).  Weight 16g + 4s + b sits
 // in byte b, bits 2s..2s+1 of word g; weights past K carry the zero code 01.
+// group == 0: one α for the tensor; otherwise α[n][k / group] (group a
+// multiple of 16, so a word's 16 weights share one α).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) ternary_pack_kernel(const T* __restrict__ W, int64_t N, int64_t K,
                                                                 int64_t row_words, const float* __restrict__ alpha_p,
-                                                                uint32_t* __restrict__ out) {
-    const float alpha = *alpha_p;
+                                                                int64_t group, uint32_t* __restrict__ out) {
+    const float alpha_t = group == 0 ? *alpha_p : 0.0f;
+    const int64_t G = group == 0 ? 1 : (K + group - 1) / group;
     const int64_t total = N * row_words;
     constexpr int V = 16 / sizeof(T);
     const bool vec_rows = ((reinterpret_cast<uintptr_t>(W) & 15) == 0) && (K % V == 0);
@@ -191,6 +224,7 @@ __global__ void __launch_bounds__(kThreads) ternary_pack_kernel(const T* __restr
         const int64_t n = wi / row_words;
         const int64_t k0 = (wi - n * row_words) * 16;
         const T* row = W + n * K;
+        const float alpha = group == 0 ? alpha_t : alpha_p[n * G + min(k0, K - 1) / group];
         float f[16];
         if (vec_rows && k0 + 16 <= K) {
 #pragma unroll
@@ -250,13 +284,39 @@ cudaError_t launch_quantize_weights(const void* W, bitlinear_dtype dtype, int64_
         absmean_partial_kernel<uint16_t><<<nparts, kThreads, 0, stream>>>(w, count, partials);
         absmean_finalize_kernel<<<1, kThreads, 0, stream>>>(partials, nparts, count, alpha);
         ternary_pack_kernel<uint16_t><<<(unsigned)pack_blocks, kThreads, 0, stream>>>(
-            w, N, K, row_words, alpha, reinterpret_cast<uint32_t*>(W_packed));
+            w, N, K, row_words, alpha, 0, reinterpret_cast<uint32_t*>(W_packed));
     } else {
         const auto* w = static_cast<const float*>(W);
         absmean_partial_kernel<float><<<nparts, kThreads, 0, stream>>>(w, count, partials);
         absmean_finalize_kernel<<<1, kThreads, 0, stream>>>(partials, nparts, count, alpha);
         ternary_pack_kernel<float><<<(unsigned)pack_blocks, kThreads, 0, stream>>>(
-            w, N, K, row_words, alpha, reinterpret_cast<uint32_t*>(W_packed));
+            w, N, K, row_words, alpha, 0, reinterpret_cast<uint32_t*>(W_packed));
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weights_groups(const void* W, bitlinear_dtype dtype, int64_t N, int64_t K, int64_t group,
+                                           uint8_t* W_packed, float* alpha, cudaStream_t stream) {
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    const int64_t G = (K + group - 1) / group;
+    int64_t blocks = (N * G + kThreads / 32 - 1) / (kThreads / 32);
+    const int64_t cap = (int64_t)dev.sm_count * 16;
+    if (blocks > cap) blocks = cap;
+    const int64_t row_words = (int64_t)bitlinear_packed_row_bytes(K) / 4;
+    int64_t pack_blocks = (N * row_words + kThreads - 1) / kThreads;
+    if (pack_blocks > cap) pack_blocks = cap;
+    if (dtype == BL_BF16) {
+        const auto* w = static_cast<const uint16_t*>(W);
+        absmean_groups_kernel<uint16_t><<<(unsigned)blocks, kThreads, 0, stream>>>(w, N, K, group, alpha);
+        ternary_pack_kernel<uint16_t><<<(unsigned)pack_blocks, kThreads, 0, stream>>>(
+            w, N, K, row_words, alpha, group, reinterpret_cast<uint32_t*>(W_packed));
+    } else {
+        const auto* w = static_cast<const float*>(W);
+        absmean_groups_kernel<float><<<(unsigned)blocks, kThreads, 0, stream>>>(w, N, K, group, alpha);
+        ternary_pack_kernel<float><<<(unsigned)pack_blocks, kThreads, 0, stream>>>(
+            w, N, K, row_words, alpha, group, reinterpret_cast<uint32_t*>(W_packed));
     }
     return cudaGetLastError();
 }

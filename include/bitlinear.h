@@ -75,8 +75,9 @@ typedef enum bitlinear_dtype {
  * row is read as little-endian 32-bit words of 16 weights each: weight
  * k = 16g + 4s + b lives in byte b of word g, bits 2s..2s+1.  So masking a word
  * with 0x03030303 << 2s yields the codes of weights 16g+4s .. 16g+4s+3 in the
- * four bytes, in order.  Weights k >= K are padding with code 01 (zero); code
- * 11 is never written and reads as zero. */
+ * four bytes, in order.  Weights k >= K are padding with code 01 (zero).  Code
+ * 11 is never written by bitlinear_quantize_weights; a product over packed
+ * data that contains it gives unspecified results. */
 BITLINEAR_API size_t bitlinear_packed_row_bytes(int64_t K);
 
 /* Device workspace bytes bitlinear_quantize_weights needs for an N×K matrix. */
@@ -229,10 +230,16 @@ BITLINEAR_API bitlinear_status bitlinear_linear(const void* x, bitlinear_dtype d
  * still finishing (e.g. the previous layer's product), instead of after it. */
 #define BL_LINEAR_WEIGHTS_STATIC 1u
 
+/* Flag for bitlinear_linear_grouped: rotate each input x by the Hadamard
+ * matrix of block bitlinear_hadamard_block(K) before quantising it (x_q and
+ * beta then hold the rotated input's quantisation); the weights must have been
+ * quantised from W·H/block.  Each K must have bitlinear_hadamard_block(K) > 1. */
+#define BL_LINEAR_HADAMARD 2u
+
 /* bitlinear_linear on `count` independent problems of one input dtype: one
  * grouped quantisation launch and one grouped product launch.  `problems` is a
- * HOST array.  flags: 0 or BL_LINEAR_WEIGHTS_STATIC.
- * With at most four tokens per problem the quantisation may instead run in
+ * HOST array.  flags: BL_LINEAR_WEIGHTS_STATIC and/or BL_LINEAR_HADAMARD.
+ * With at most four tokens per problem (and no rotation) the quantisation may instead run in
  * the product kernel's prologue (one launch; x_q and beta are still written),
  * when the problems fit it and the input rows are small next to the weights;
  * the environment variable BITLINEAR_LINEAR_FUSION=on|off forces the choice.
@@ -279,6 +286,157 @@ typedef struct bitlinear_act_sum_problem {
 BITLINEAR_API bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, int n_acts,
                                                       const bitlinear_forward_problem* fwd, int n_fwd,
                                                       uint32_t flags, bitlinear_stream_t stream);
+
+/* ---- Hadamard rotation before the absmax quantisation ("1.58-bit 大模型极限
+ * 量化实战", chenxutan.com/d/5049.html §6.2: a few activation dimensions hold
+ * large outliers that inflate β = max|x| and crush every other dimension; an
+ * orthogonal Hadamard rotation of the activations first spreads them out).
+ *
+ * H is block-diagonal with Sylvester blocks of order `block` (a power of two
+ * dividing K, at most BITLINEAR_MAX_HADAMARD_BLOCK): inside a block
+ * out[j] = Σ_i x[i]·(-1)^popcount(i & j), unnormalised.  It is evaluated by
+ * the butterfly network in binary32, stages h = 1, 2, 4, …, block/2 in that
+ * order, each butterfly replacing the pair (i, i+h), i & h == 0, by
+ * (a + b, a - b); so results are reproducible bit for bit.  The product is
+ * unchanged when the weights take the same rotation scaled by 1/block:
+ * (x·H)·(W·H/block)ᵀ = x·Wᵀ.  So a rotated layer quantises W' = W·H/block
+ * (bitlinear_hadamard with scale 1/block, then bitlinear_quantize_weights)
+ * and rotates x before bitlinear_quantize_act (bitlinear_quantize_act_hadamard,
+ * or BL_LINEAR_HADAMARD on a linear call). */
+#define BITLINEAR_MAX_HADAMARD_BLOCK 8192
+
+/* The block a linear call flagged BL_LINEAR_HADAMARD uses: the largest power
+ * of two dividing K, at most BITLINEAR_MAX_HADAMARD_BLOCK (0 if K < 1). */
+BITLINEAR_API int64_t bitlinear_hadamard_block(int64_t K);
+
+/* out[m][·] = (x[m][·]·H)·scale, each output one binary32 multiply by `scale`
+ * after the last stage (scale 1 for activations, 1/block for weights).
+ *   x    [M][K] row-major, `dtype`, aligned to its element size.
+ *   out  [M][K] float32 (must not overlap x).
+ * Errors: BL_ERR_NULL, BL_ERR_SHAPE (M, K < 1, K > BITLINEAR_MAX_K, M > 2^31,
+ * block not a power of two dividing K or above the maximum), BL_ERR_ALIGN,
+ * BL_ERR_DTYPE, BL_ERR_ARCH, BL_ERR_CUDA. */
+BITLINEAR_API bitlinear_status bitlinear_hadamard(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K,
+                                                  int64_t block, float scale, float* out, bitlinear_stream_t stream);
+
+/* bitlinear_quantize_act of x·H: β_m = max_k |(x·H)[m][k]| + 1e-8 and
+ * x̃ = clip(round((x·H)·127/β), -127, 127), the rotated values never leaving
+ * the chip.  Arguments as bitlinear_quantize_act plus `block`; errors as
+ * bitlinear_hadamard. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_act_hadamard(const void* x, bitlinear_dtype dtype, int64_t M,
+                                                               int64_t K, int64_t block, int8_t* x_q, float* beta,
+                                                               bitlinear_stream_t stream);
+
+/* ---- Finer scale granularity: one α per output row ("1.58 位大模型",
+ * nxmr.cn/news/148658 §3.1, §4.2: alpha = mean(|w|) of each row) or per block
+ * of `group` consecutive input features of a row (2kiu.com/news/4928193 §2.3,
+ * §4.2: one scale per 128 elements, scale[C_out][C_in/128]).  `group` >= K
+ * means one α per row; otherwise it must be a multiple of 64 (the page uses
+ * 128); the last block of a row may be shorter.  alpha is [N][ceil(K/group)]
+ * float32, each the exact mean of |W| over its group rounded once to binary64
+ * and once to binary32 (as for the tensor). */
+
+/* Absmean ternary quantisation with one α per group:
+ * Ŵ[n][k] = clip(round(W[n][k] / α[n][k/group]), -1, 1), packed as for
+ * bitlinear_quantize_weights.  Needs no workspace.
+ * Errors: BL_ERR_NULL, BL_ERR_SHAPE (as bitlinear_quantize_weights, or group
+ * < K and not a positive multiple of 64), BL_ERR_ALIGN, BL_ERR_DTYPE,
+ * BL_ERR_ARCH, BL_ERR_CUDA. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_weights_scaled(const void* W, bitlinear_dtype dtype, int64_t N,
+                                                                 int64_t K, int64_t group, uint8_t* W_packed,
+                                                                 float* alpha, bitlinear_stream_t stream);
+
+/* One problem of bitlinear_linear_scaled.  x (nullable): the input, quantised
+ * into x_q and beta first as by bitlinear_quantize_act; when NULL, x_q and
+ * beta are inputs.  acc_out (nullable) receives the int32 products and is
+ * allowed only with one α per row (group >= K). */
+typedef struct bitlinear_scaled_problem {
+    const void* x;
+    int8_t* x_q;
+    float* beta;
+    const uint8_t* W_packed;
+    const float* alpha;
+    const float* bias;
+    float* y;
+    int32_t* acc_out;
+    int64_t M, N, K, group;
+} bitlinear_scaled_problem;
+
+/* The BitLinear forward with one α per group: for each group b of row n the
+ * exact integer sum acc_b = Σ_{k in b} x̃[m][k]·Ŵ[n][k], S = Σ_b α[n][b]·acc_b,
+ * y[m][n] = RN32( RN32(S)·RN32(RN64(β_m/127)) ) (+ bias[n]).  With one α per
+ * row S = α_n·acc is exact; with several, S is summed in binary64 (each term
+ * exact), in an order that may differ from a sequential sum in the last bits
+ * of binary64.  `problems` is a HOST array; flags: 0 or
+ * BL_LINEAR_WEIGHTS_STATIC.  CUDA cores; for more than four tokens the
+ * weights are streamed once per four tokens (this variant is not the
+ * tensor-core path).
+ * Errors: as bitlinear_linear_grouped, plus BL_ERR_SHAPE for a bad group or
+ * acc_out with several α per row. */
+BITLINEAR_API bitlinear_status bitlinear_linear_scaled(const bitlinear_scaled_problem* problems, int count,
+                                                       bitlinear_dtype dtype, uint32_t flags,
+                                                       bitlinear_stream_t stream);
+
+/* ---- 4-bit activations ("BitNet CPU 实测", cf-1.com/news/5800143 §2.1: later
+ * variants quantise the activations to 4 bits instead of 8).  The absmax rule
+ * of bitlinear_quantize_act with the signed 4-bit range: β_m = max|x| + 1e-8,
+ * x̃ = clip(round((x·7)/β_m), -7, 7), the product and the quotient each
+ * rounded to binary32, half to even.  Storage ("x_q4"): [M][ceil(K/2)] bytes,
+ * element k in byte k/2, the low nibble for even k, two's complement; the
+ * high nibble of the last byte of an odd-K row is 0.  Dequantisation:
+ * y = fp32(acc)·RN32(RN64(α·β/7)) (+ bias), one α for the tensor. */
+BITLINEAR_API bitlinear_status bitlinear_quantize_act_a4(const void* x, bitlinear_dtype dtype, int64_t M, int64_t K,
+                                                         uint8_t* x_q4, float* beta, bitlinear_stream_t stream);
+
+/* acc[m][n] = Σ_k x̃[m][k]·Ŵ[n][k] (exact int32) on 4-bit activations, then
+ * y = RN32(fp32(acc)·RN32(RN64(α·β_m/7))) (+ bias[n], binary32 add).
+ * Arguments as bitlinear_forward with x_q4 in place of x_q.  CUDA cores, four
+ * tokens per pass (this variant is not the tensor-core path). */
+BITLINEAR_API bitlinear_status bitlinear_forward_a4(const uint8_t* x_q4, const float* beta, int64_t M, int64_t K,
+                                                    const uint8_t* W_packed, const float* alpha, int64_t N,
+                                                    const float* bias, float* y, int32_t* acc_out,
+                                                    bitlinear_stream_t stream);
+
+/* bitlinear_quantize_act_a4 then bitlinear_forward_a4 on `count` problems (one
+ * grouped launch each, chained by programmatic dependent launch); the x_q field
+ * of each problem is its x_q4 buffer.  flags: 0 or BL_LINEAR_WEIGHTS_STATIC.
+ * Errors: as bitlinear_linear_grouped. */
+BITLINEAR_API bitlinear_status bitlinear_linear_a4(const bitlinear_linear_problem* problems, int count,
+                                                   bitlinear_dtype dtype, uint32_t flags, bitlinear_stream_t stream);
+
+/* ---- Training with the straight-through estimator ("1.58-bit 大模型极限量化
+ * 实战", chenxutan.com/d/5049.html §3.3, §4.2 training branch, §6.3;
+ * "1.58 位大模型" nxmr.cn/news/148658 §3.4): the layer keeps latent float
+ * weights W, quantises them afresh in every forward, and the backward passes
+ * the gradient straight through both quantisers, except that a weight outside
+ * the clip range (|W/α| > 1) gets no gradient; α and β are constants to it. */
+
+/* Training forward: bitlinear_quantize_weights of the latent W [N][K]
+ * (w_dtype) into W_packed and alpha, then bitlinear_linear of x [M][K]
+ * (x_dtype) into x_q, beta and y, all on `stream` (the outputs the backward
+ * needs are kept).  workspace as for bitlinear_quantize_weights.
+ * Errors: the union of both calls'. */
+BITLINEAR_API bitlinear_status bitlinear_train_forward(const void* W, bitlinear_dtype w_dtype, int64_t N, int64_t K,
+                                                       const void* x, bitlinear_dtype x_dtype, int64_t M,
+                                                       uint8_t* W_packed, float* alpha, int8_t* x_q, float* beta,
+                                                       float* y, void* workspace, size_t workspace_bytes,
+                                                       bitlinear_stream_t stream);
+
+/* Backward for g = ∂L/∂y [M][N] float32:
+ *   grad_x[m][k] = α·Σ_n g[m][n]·Ŵ[n][k]
+ *   grad_W[n][k] = |RN32(W[n][k]/α)| <= 1 ? Σ_m RN32(g[m][n]·s_m)·x̃[m][k] : 0,
+ *                  s_m = RN32(RN64(β_m/127))
+ * from the forward's W_packed, alpha, x_q, beta and the latent W (w_dtype).
+ * Float32 arithmetic: each output summed by one thread in index order with
+ * fused multiply-adds, rounded once (grad_x then times α); a float64 sum
+ * differs by at most the float32 summation bound.  grad_x [M][K] and grad_W
+ * [N][K] float32 are each nullable (not computed).  CUDA cores.
+ * Errors: BL_ERR_NULL, BL_ERR_SHAPE, BL_ERR_ALIGN, BL_ERR_DTYPE, BL_ERR_ARCH,
+ * BL_ERR_CUDA. */
+BITLINEAR_API bitlinear_status bitlinear_ste_backward(const float* g, int64_t M, int64_t N, int64_t K,
+                                                      const uint8_t* W_packed, const float* alpha, const int8_t* x_q,
+                                                      const float* beta, const void* W, bitlinear_dtype w_dtype,
+                                                      float* grad_x, float* grad_W, bitlinear_stream_t stream);
 
 /* Reads and clears the current device's error word, which a kernel sets when
  * one of its bounded waits expires (it then stops early and its outputs are

@@ -34,7 +34,7 @@ def test_header_symbols_exported(L):
     assert {"bitlinear_quantize_weights", "bitlinear_quantize_act", "bitlinear_forward"} <= set(names)
     for n in names:
         assert hasattr(L, n), f"{n} declared in bitlinear.h but not exported"
-    assert L.bitlinear_version() == 100
+    assert L.bitlinear_version() == 101
 
 
 def test_struct_layout_matches_header():
@@ -97,7 +97,7 @@ def test_forward_argument_errors(L):
     arr = (bl.ForwardProblem * 1)()
     assert L.bitlinear_forward_grouped(arr, 0, None) == COUNT
     lin = (bl.LinearProblem * 1)()
-    assert L.bitlinear_linear_grouped(lin, 1, 0, 2, None) == 10  # BL_ERR_FLAGS
+    assert L.bitlinear_linear_grouped(lin, 1, 0, 4, None) == 10  # BL_ERR_FLAGS (2 is BL_LINEAR_HADAMARD)
     assert L.bitlinear_linear_grouped(lin, 1, 0, 0, None) == NULL
     assert L.bitlinear_forward_grouped(None, 1, None) == NULL
 
@@ -143,3 +143,70 @@ def test_linear_block_argument_errors(L):
     acts[0] = bl.ActSumProblem(P, None, None, P, P, 1, 64)
     assert blk(acts, 1, fwd, 1, 0, None) == NULL             # forward problem left empty
     assert blk(None, 0, fwd, 1, 0, None) == NULL
+
+
+def test_hadamard_argument_errors(L):
+    assert L.bitlinear_hadamard_block(4096) == 4096
+    assert L.bitlinear_hadamard_block(11008) == 256
+    assert L.bitlinear_hadamard_block(3 * 16384) == 8192
+    assert L.bitlinear_hadamard_block(7) == 1 and L.bitlinear_hadamard_block(0) == 0
+    h, qh = L.bitlinear_hadamard, L.bitlinear_quantize_act_hadamard
+    assert h(None, 0, 1, 64, 64, 1.0, P, None) == NULL
+    assert h(P, 0, 1, 64, 64, 1.0, None, None) == NULL
+    assert h(P, 5, 1, 64, 64, 1.0, P, None) == DTYPE
+    assert h(P, 0, 1, 64, 48, 1.0, P, None) == SHAPE      # not a power of two
+    assert h(P, 0, 1, 96, 64, 1.0, P, None) == SHAPE      # does not divide K
+    assert h(P, 0, 1, 16384, 16384, 1.0, P, None) == SHAPE  # above the largest block
+    assert h(P, 0, 0, 64, 64, 1.0, P, None) == SHAPE
+    assert h(P + 2, 0, 1, 64, 64, 1.0, P, None) == ALIGN
+    assert qh(P, 0, 1, 64, 64, None, P, None) == NULL
+    assert qh(P, 1, 1, 64, 64, P, P + 2, None) == ALIGN
+    arr = (bl.LinearProblem * 1)()
+    arr[0] = bl.LinearProblem(P, P, P, P, P, None, P, None, 1, 64, 63)
+    assert L.bitlinear_linear_grouped(arr, 1, 0, bl.BL_LINEAR_HADAMARD, None) == SHAPE  # block 1: nothing to rotate
+    assert L.bitlinear_linear_grouped(arr, 1, 0, 4, None) == FLAGS
+
+
+def test_scaled_argument_errors(L):
+    q = L.bitlinear_quantize_weights_scaled
+    assert q(None, 0, 4, 1000, 128, P, P, None) == NULL
+    assert q(P, 0, 4, 1000, 100, P, P, None) == SHAPE   # below K and not a multiple of 64
+    assert q(P, 0, 4, 1000, 0, P, P, None) == SHAPE
+    assert q(P, 0, 4, 1000, 128, P + 8, P, None) == ALIGN
+    assert q(P, 7, 4, 1000, 128, P, P, None) == DTYPE
+    arr = (bl.ScaledProblem * 1)()
+    arr[0] = bl.ScaledProblem(None, P, P, P, P, None, P, P, 1, 64, 1000, 128)  # acc_out with several α per row
+    assert L.bitlinear_linear_scaled(arr, 1, 0, 0, None) == SHAPE
+    arr[0] = bl.ScaledProblem(None, P, P, P, P, None, P, None, 1, 64, 1000, 96)
+    assert L.bitlinear_linear_scaled(arr, 1, 0, 0, None) == SHAPE
+    assert L.bitlinear_linear_scaled(arr, 0, 0, 0, None) == COUNT
+    assert L.bitlinear_linear_scaled(arr, 1, 0, 2, None) == FLAGS
+    assert ctypes.sizeof(bl.ScaledProblem) == 12 * 8
+
+
+def test_a4_argument_errors(L):
+    assert L.bitlinear_quantize_act_a4(None, 0, 1, 64, P, P, None) == NULL
+    assert L.bitlinear_quantize_act_a4(P, 3, 1, 64, P, P, None) == DTYPE
+    assert L.bitlinear_quantize_act_a4(P, 0, 0, 64, P, P, None) == SHAPE
+    assert L.bitlinear_quantize_act_a4(P + 2, 0, 1, 64, P, P, None) == ALIGN
+    assert L.bitlinear_forward_a4(P, P, 1, 64, P + 4, P, 8, None, P, None, None) == ALIGN
+    assert L.bitlinear_forward_a4(P, P, 1, 64, P, P, 0, None, P, None, None) == SHAPE
+    arr = (bl.LinearProblem * 1)()
+    assert L.bitlinear_linear_a4(arr, 1, 0, 0, None) == NULL
+    assert L.bitlinear_linear_a4(arr, 1, 0, 2, None) == FLAGS
+    assert L.bitlinear_linear_a4(arr, 17, 0, 0, None) == COUNT
+
+
+def test_train_argument_errors(L):
+    b = L.bitlinear_ste_backward
+    assert b(None, 1, 8, 64, P, P, P, P, P, 0, P, P, None) == NULL
+    assert b(P, 1, 8, 64, None, P, P, P, P, 0, P, None, None) == NULL   # grad_x needs the codes
+    assert b(P, 1, 8, 64, P, P, None, P, P, 0, None, P, None) == NULL   # grad_W needs x_q
+    assert b(P, 0, 8, 64, P, P, P, P, P, 0, P, P, None) == SHAPE
+    assert b(P, 1, 8, 64, P, P, P, P, P, 9, None, P, None) == DTYPE
+    assert b(P + 2, 1, 8, 64, P, P, P, P, P, 0, P, P, None) == ALIGN
+    ws = L.bitlinear_quantize_weights_workspace_bytes(8, 64)
+    t = L.bitlinear_train_forward
+    assert t(P, 0, 8, 64, None, 0, 1, P, P, P, P, P, P, ws, None) == NULL
+    assert t(P, 0, 8, 64, P, 0, 0, P, P, P, P, P, P, ws, None) == SHAPE
+    assert t(P, 0, 8, 64, P, 0, 1, P, P, P, P, P, P, 0, None) == WORKSPACE
