@@ -905,6 +905,92 @@ def run_a4(args, world, local_rank):
             "bytes_per_step": bps, "steps": K, "replicas": replicas, "clocks": clocks}
 
 
+# ----------------------------------------------------------------------------- training leg
+FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs × FP32 FMA lanes/clk × 2 flops × max SM clock
+
+
+def run_train(args, world, local_rank):
+    """One training step with the straight-through estimator on the three
+    prefill shapes at M = 2048 tokens: bitlinear_train_forward (quantise the
+    float32 latent weights afresh, quantise x, tensor-core product) then
+    bitlinear_ste_backward (grad_x and grad_W, float32 CUDA-core GEMMs)."""
+    import torch
+    import bitlinear_w1_a8_03_b200 as bl
+    from bitlinear_w1_a8_03_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    props = torch.cuda.get_device_properties(dev)
+    specs = prefill_specs()
+    L = bl.lib()
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+    items = []
+    for s in specs:
+        W = torch.from_numpy(synth.weights(s.seed, s.N, s.K, s.w_std)).to(dev)
+        xb = synth.f32_to_bf16_bits(synth.activations(s.x_seed, s.M, s.K, outliers=True))
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        g = torch.randn((s.M, s.N), generator=torch.Generator(device=dev).manual_seed(s.seed), device=dev) * 1e-3
+        ws = torch.empty(L.bitlinear_quantize_weights_workspace_bytes(s.N, s.K), dtype=torch.uint8, device=dev)
+        it = dict(W=W, x=x, g=g, ws=ws, s=s,
+                  Wp=torch.empty((s.N, int(L.bitlinear_packed_row_bytes(s.K))), dtype=torch.uint8, device=dev),
+                  a=torch.empty(1, dtype=torch.float32, device=dev),
+                  xq=torch.empty((s.M, s.K), dtype=torch.int8, device=dev),
+                  b=torch.empty(s.M, dtype=torch.float32, device=dev),
+                  y=torch.empty((s.M, s.N), dtype=torch.float32, device=dev),
+                  gx=torch.empty((s.M, s.K), dtype=torch.float32, device=dev),
+                  gw=torch.empty((s.N, s.K), dtype=torch.float32, device=dev))
+        items.append(it)
+    P = bl._ptr
+
+    def fwd():
+        for it in items:
+            s = it["s"]
+            bl.check(L.bitlinear_train_forward(P(it["W"]), bl.BL_F32, s.N, s.K, P(it["x"]), bl.BL_BF16, s.M, P(it["Wp"]),
+                                               P(it["a"]), P(it["xq"]), P(it["b"]), P(it["y"]), P(it["ws"]),
+                                               it["ws"].numel(), sh), "train_forward")
+
+    def bwd():
+        for it in items:
+            s = it["s"]
+            bl.check(L.bitlinear_ste_backward(P(it["g"]), s.M, s.N, s.K, P(it["Wp"]), P(it["a"]), P(it["xq"]), P(it["b"]),
+                                              P(it["W"]), bl.BL_F32, P(it["gx"]), P(it["gw"]), sh), "ste_backward")
+
+    K = max(3, args.steps // 4)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fwd()
+            bwd()
+    stream.synchronize()
+    sampler = ClockSampler(gpu_id(props, local_rank))
+    fwd_ms = bwd_ms = 0.0
+    with torch.cuda.stream(stream):
+        for _ in range(K):
+            ev[0].record()
+            fwd()
+            ev[1].record()
+            bwd()
+            ev[2].record()
+            ev[2].synchronize()
+            fwd_ms += ev[0].elapsed_time(ev[1]) / K
+            bwd_ms += ev[1].elapsed_time(ev[2]) / K
+    clocks = sampler.stop()
+    fwd_ms, bwd_ms = max_over_ranks([fwd_ms, bwd_ms], dev, world)
+    bwd_flops = sum(4 * s.M * s.N * s.K for s in specs)
+    fwd_ops = sum(2 * s.M * s.N * s.K for s in specs)
+    achieved = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    return {"metric": "training step (straight-through estimator) on the prefill shapes",
+            "workload": "M=2048 tokens; (K,N) = (4096,4096), (4096,11008), (11008,4096); float32 latent W, bf16 x, "
+                        "float32 upstream gradient",
+            "ms_per_step": round(fwd_ms + bwd_ms, 3), "forward_ms": round(fwd_ms, 3), "backward_ms": round(bwd_ms, 3),
+            "forward_TOPS": round(fwd_ops / (fwd_ms * 1e-3) / 1e12, 1),
+            "roofline": {"bound": "alu", "kernel": "ste_grad_x_kernel + ste_grad_w_kernel (float32 FMA on CUDA cores)",
+                         "achieved": round(achieved, 2), "peak": round(FFMA_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                         "frac": round(achieved / FFMA_PEAK_TFLOPS, 4),
+                         "peak_source": "148 SMs x 128 FP32 FMA lanes/clk x 2 flops x 1.965 GHz"},
+            "steps": K, "clocks": clocks}
+
+
 # ----------------------------------------------------------------------------- tiny leg
 def run_tiny(args, world, local_rank):
     """Config 1: M = 1, K = N = 256, float32 x and W (seed 0).  A latency line:
@@ -1135,9 +1221,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--legs", default="decode,tiny,batched_100b,prefill,stack,hadamard,scales,a4",
+    ap.add_argument("--legs", default="decode,tiny,batched_100b,prefill,stack,hadamard,scales,a4,train",
                     help="comma list: decode (the headline line); tiny, batched_100b, prefill, stack, hadamard, "
-                         "scales and a4 are added under their own keys")
+                         "scales, a4 and train are added under their own keys")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     args = ap.parse_args()
     legs = [x for x in args.legs.split(",") if x]
@@ -1180,6 +1266,8 @@ def main():
         result["scales"] = run_scales(args, world, local_rank)
     if "a4" in legs:
         result["a4"] = run_a4(args, world, local_rank)
+    if "train" in legs:
+        result["train"] = run_train(args, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(args)
