@@ -67,7 +67,8 @@ struct GProblem {
     int32_t C;            // 16-byte chunks per row
     int32_t full_chunks;  // chunks entirely inside K (the activation tail needs guards)
     int32_t rgn;          // row groups
-    int64_t unit_begin;   // first unit (row group, chunk) of this problem in the launch
+    int32_t S;            // steps per row group: ceil(C / 32) (a step gives each lane one chunk)
+    int64_t step_begin;   // first step of this problem in the launch
     // fused quantisation (x̃ made in shared memory from x):
     const void* x;          // activations, float32 or bfloat16 [M][K]
     const float* x2;        // nullable float32 second addend
@@ -75,76 +76,29 @@ struct GProblem {
     int32_t write_outputs;  // the owner CTA writes x̃ to xq and β to beta (and x_sum)
 };
 
+constexpr int kMaxCta = 512;  // most CTAs of one launch
+
 struct GParams {
     GProblem p[kMaxGroup];
     int count;
-    int64_t total_units;
+    int64_t total_steps;
+    int32_t cta_begin[kMaxCta + 1];  // first step of each CTA (row-group boundaries), then the end
     int x_bf16;        // fused: activation dtype
     int32_t slot_row;  // fused: bytes per token row of a shared x̃ slot (64·ceil(K/64) of the widest problem)
 };
 
 // ---------------------------------------------------------------- work split
-__host__ __device__ __forceinline__ int problem_of_unit(const GProblem* P, int count, int64_t u) {
+// The work of a launch is a sequence of steps: problem by problem, row group
+// by row group, S steps per row group (step s covers chunks 32s .. 32s+31 of
+// the RG rows).  Each CTA takes a contiguous range of whole row groups (the
+// host balances the ranges, see cta_ranges) and splits it into equal step
+// ranges for its warps.
+__host__ __device__ __forceinline__ int problem_of_step(const GProblem* P, int count, int64_t u) {
     int p = 0;
-    while (p + 1 < count && u >= P[p + 1].unit_begin) ++p;
+    while (p + 1 < count && u >= P[p + 1].step_begin) ++p;
     return p;
 }
 
-// Start of the row group containing unit t, rounded to the nearer boundary.
-__host__ __device__ __forceinline__ int64_t snap_to_row_group(const GProblem* P, int count, int64_t total, int64_t t) {
-    if (t >= total) return total;
-    const int p = problem_of_unit(P, count, t);
-    const int64_t local = t - P[p].unit_begin;
-    int64_t g = local / P[p].C;
-    if (2 * (local - g * P[p].C) >= P[p].C) ++g;
-    return P[p].unit_begin + g * P[p].C;
-}
-
-// Units [a, b) of CTA `c` out of G.
-__host__ __device__ __forceinline__ void cta_units(const GProblem* P, int count, int64_t total, int64_t c, int64_t G,
-                                                   int64_t& a, int64_t& b) {
-    a = snap_to_row_group(P, count, total, (total * c) / G);
-    b = snap_to_row_group(P, count, total, (total * (c + 1)) / G);
-}
-
-// Position in the unit sequence: problem, row group, chunk; and the range end.
-struct Cursor {
-    int p;
-    int32_t rg;
-    int32_t c;
-    int64_t u, end;
-};
-
-__device__ __forceinline__ void cursor_seek(const GProblem* P, int count, Cursor& cur, int64_t u, int64_t end) {
-    cur.p = problem_of_unit(P, count, u);
-    const int64_t local = u - P[cur.p].unit_begin;
-    cur.rg = (int32_t)(local / P[cur.p].C);
-    cur.c = (int32_t)(local - (int64_t)cur.rg * P[cur.p].C);
-    cur.u = u;
-    cur.end = end;
-}
-
-// Chunks of the segment at the cursor: the rest of the row, at most SC, at
-// most the rest of the range.
-template <int SC>
-__device__ __forceinline__ int cursor_len(const GProblem& pr, const Cursor& cur) {
-    int n = pr.C - cur.c;
-    if (n > SC) n = SC;
-    if (n > cur.end - cur.u) n = (int)(cur.end - cur.u);
-    return n;
-}
-
-__device__ __forceinline__ void cursor_advance(const GProblem& pr, Cursor& cur, int n) {
-    cur.u += n;
-    cur.c += n;
-    if (cur.c == pr.C) {
-        cur.c = 0;
-        if (++cur.rg == pr.rgn) {
-            cur.rg = 0;
-            ++cur.p;
-        }
-    }
-}
 // ---------------------------------------------------------------- activations
 // The last activation chunk of a row when K is not a multiple of 64: bytes
 // past K read as zero.  Kept out of line so the full-chunk path stays lean.
@@ -159,43 +113,12 @@ __device__ __noinline__ void load_act_tail(const int8_t* xrow, int K, int chunk,
     }
 }
 
-// 64 activations (chunk `chunk`) of one token from global x̃, zero past K.
-__device__ __forceinline__ void ldg_act_chunk(const int8_t* xrow, int K, int chunk, bool full, uint32_t (&a)[16]) {
-    if (full) {
-        const int8_t* p = xrow + 64 * chunk;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const uint4 u = ld_shared_ro16(p + 16 * v);
-            a[4 * v + 0] = u.x;
-            a[4 * v + 1] = u.y;
-            a[4 * v + 2] = u.z;
-            a[4 * v + 3] = u.w;
-        }
-    } else {
-        uint32_t tmp[16];  // only this rare path goes through local memory
-        load_act_tail(xrow, K, chunk, tmp);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) a[q] = tmp[q];
-    }
-}
-
 // Shared x̃ slot layout: the four 16-byte pieces of 64-byte chunk c are
 // rotated by (c >> 1), so the 16-byte reads of 8 lanes on consecutive chunks
 // fall in distinct banks.
 __device__ __forceinline__ uint32_t xs_offset(int k) {
     const int c = k >> 6, v = (k >> 4) & 3;
     return (uint32_t)(64 * c + 16 * ((v + (c >> 1)) & 3) + (k & 15));
-}
-
-__device__ __forceinline__ void lds_act_chunk(uint32_t row, int chunk, uint32_t (&a)[16]) {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        const uint4 u = lds128(row + 64 * chunk + 16 * ((v + (chunk >> 1)) & 3));
-        a[4 * v + 0] = u.x;
-        a[4 * v + 1] = u.y;
-        a[4 * v + 2] = u.z;
-        a[4 * v + 3] = u.w;
-    }
 }
 
 template <int NT>
@@ -262,6 +185,7 @@ struct QRow {
     int m;            // token
     uint8_t* dst;     // slot row
     float* beta_dst;  // slot β
+    int* sum_dst;     // slot Σx̃ (zeroed before; the CTA's threads add their parts)
     bool out;         // also write x̃, β (and x) to global memory
 };
 
@@ -328,6 +252,7 @@ __device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, 
         const GProblem& pr = *q.pr;
         const int64_t base = (int64_t)q.m * pr.K;
         const int nvec = pr.K / V;
+        int qsum = 0;  // this thread's part of Σx̃
 #pragma unroll
         for (int j = 0; j < kFuseVec; ++j) {
             const int v = threadIdx.x + j * NT;
@@ -341,6 +266,7 @@ __device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, 
 #pragma unroll
                     for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(f[4 * g + e], beta, rbeta) << (8 * e);
                     wq[g] = x;
+                    qsum = dp4a_s8s8(0x01010101u, x, qsum);
                 }
                 const int k = v * V;
 #pragma unroll
@@ -362,6 +288,9 @@ __device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, 
                 }
             }
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
+        if ((threadIdx.x & 31) == 0) atomicAdd(q.sum_dst, qsum);  // integer: exact in any order
         if (threadIdx.x == 0) {
             *q.beta_dst = beta;
             if (q.out) const_cast<float*>(pr.beta)[q.m] = beta;
@@ -400,57 +329,219 @@ __device__ __forceinline__ int reduce_scatter(int (&v)[V], int lane, int& idx) {
 // on a 16-byte boundary (they are read with 16-byte loads).
 template <int W>
 struct alignas(128) GShared {
-    int64_t bound[W + 1];                    // warp unit ranges inside the CTA
+    int64_t bound[W + 1];                     // warp step ranges inside the CTA
     int part[W][2][kRGMax * kGemvMaxTokens];  // a warp's sums of row groups shared with its neighbours
     GProblem prob[kMaxGroup];  // copy of the problem table (indexed reads of it are cheap here)
     float xbeta[kMaxSlots][kGemvMaxTokens];  // fused: β of each slot's tokens
+    int xsum[kMaxSlots][kGemvMaxTokens];     // fused: Σx̃ of each slot's tokens
     float red[kFuseRows][32];                // fused: block reduction scratch
+    uint4 zero[4];                           // 64 zero bytes: what idle lanes read as activations
 };
 
-// The 16-byte words of chunk `chunk` of the row group's RG rows (rows past N
-// read row N-1: valid memory, results discarded), or zeros when !valid.
-template <int RG>
-__device__ __forceinline__ void load_rows(const GProblem& pr, int rg, int chunk, bool valid, uint4 (&w)[RG]) {
-    const int row0 = rg * RG;
-    const uint8_t* base = pr.W + (int64_t)chunk * 16;
-#pragma unroll
-    for (int r = 0; r < RG; ++r) {
-        const int row = min(row0 + r, pr.N - 1);
-        w[r] = valid ? ld_stream16(base + (int64_t)row * pr.row_bytes) : make_uint4(0u, 0u, 0u, 0u);
+// 64 zero bytes in global memory: the activations idle lanes read when x̃
+// comes from global memory.
+__device__ const uint4 g_zero_chunk[4] = {};
+
+// The warp's position in its step range: problem p, row group rg, step s
+// (chunks 32s .. 32s+31), global step index u, and the range end.
+struct Walk {
+    int p, rg, s;
+    int64_t u, end;
+};
+
+__device__ __forceinline__ void walk_seek(const GProblem* T, int count, Walk& w, int64_t u, int64_t end) {
+    w.p = problem_of_step(T, count, u);
+    const int32_t local = (int32_t)(u - T[w.p].step_begin);
+    w.rg = local / T[w.p].S;
+    w.s = local - w.rg * T[w.p].S;
+    w.u = u;
+    w.end = end;
+}
+
+// Chunks of the step at the position (pr = its problem): 32, or the rest of
+// the row in its last step.
+__device__ __forceinline__ int walk_len(const GProblem& pr, const Walk& w) { return min(32, pr.C - 32 * w.s); }
+
+__device__ __forceinline__ void walk_advance(const GProblem& pr, Walk& w) {
+    ++w.u;
+    if (++w.s == pr.S) {
+        w.s = 0;
+        if (++w.rg == pr.rgn) {
+            w.rg = 0;
+            ++w.p;
+        }
     }
 }
 
-// The MT tokens' activations of chunk `chunk` (zero past K, past M, and when !valid).
-template <int MT, bool FUSE>
-__device__ __forceinline__ void load_x(const GProblem& pr, uint32_t xrow0, int32_t slot_row, int chunk, bool valid,
-                                       uint32_t (&a)[MT][16]) {
+// Requests the RG rows' 16 bytes of one step (n chunks) into this lane's
+// column of a stage (row r at dst + 512·r): lane l copies chunk
+// 32s + min(l, n - 1), so every address is valid and needs no predicate; rows
+// past N copy row N-1.  Lanes l >= n pair their words with zero activations,
+// and rows past N are never written, so neither changes a result.
+template <int RG>
+__device__ __forceinline__ void stage_step(const GProblem& pr, const Walk& s, int n, int lane, uint32_t dst) {
+    const int ch = 32 * s.s + min(lane, n - 1);
+    const int row0 = s.rg * RG;
+    const int rlast = min(RG, pr.N - row0) - 1;
+    const int32_t rb = pr.row_bytes;
+    const uint8_t* base = pr.W + (int64_t)row0 * rb + 16 * ch;
+#pragma unroll
+    for (int r = 0; r < RG; ++r) cp_async16(dst + 512u * r, base + (uint32_t)(min(r, rlast) * rb));
+}
+
+// MT tokens' activations of chunk ch from the shared slot rows (token m at
+// xrow + m·slot_row, pieces rotated as xs_offset lays them out); idle lanes
+// read the zero block.  Tokens past M read rows the prologue did not write:
+// their sums are never stored.
+template <int MT>
+__device__ __forceinline__ void lds_x(uint32_t xrow, int32_t slot_row, int ch, bool active, uint32_t zero,
+                                      uint32_t (&a)[MT][16]) {
+    const uint32_t rot = (uint32_t)(ch >> 1);
+    const uint32_t b0 = active ? xrow + 64u * (uint32_t)ch : zero;
+    const uint32_t dm = active ? (uint32_t)slot_row : 0u;
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const uint4 u = lds128(b0 + (uint32_t)m * dm + 16u * ((v + rot) & 3u));
+            a[m][4 * v + 0] = u.x;
+            a[m][4 * v + 1] = u.y;
+            a[m][4 * v + 2] = u.z;
+            a[m][4 * v + 3] = u.w;
+        }
+}
+
+// MT tokens' activations of chunk ch from global x̃ [M][K] (tokens past M
+// read token M-1; their sums are never stored); idle lanes read zeros.  The
+// chunk holding the end of a row when K % 64 != 0 goes through
+// load_act_tail, which reads nothing past K.
+template <int MT>
+__device__ __forceinline__ void ldg_x(const int8_t* xq, int M, int K, int full_chunks, int ch, bool active,
+                                      uint32_t (&a)[MT][16]) {
+    const bool tail = active && ch >= full_chunks;
+    if (__any_sync(0xffffffffu, tail)) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const int8_t* row = xq + (int64_t)min(m, M - 1) * K;
+            if (tail) {
+                uint32_t tmp[16];
+                load_act_tail(row, K, ch, tmp);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) a[m][q] = tmp[q];
+            } else {
+                const uint8_t* p = active ? reinterpret_cast<const uint8_t*>(row) + 64 * ch
+                                          : reinterpret_cast<const uint8_t*>(g_zero_chunk);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 u = ld_shared_ro16(p + 16 * v);
+                    a[m][4 * v + 0] = u.x;
+                    a[m][4 * v + 1] = u.y;
+                    a[m][4 * v + 2] = u.z;
+                    a[m][4 * v + 3] = u.w;
+                }
+            }
+        }
+        return;
+    }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-        if (valid && m < pr.M) {
-            if constexpr (FUSE)
-                lds_act_chunk(xrow0 + m * slot_row, chunk, a[m]);
-            else
-                ldg_act_chunk(pr.xq + (int64_t)m * pr.K, pr.K, chunk, chunk < pr.full_chunks, a[m]);
-        } else {
+        const uint8_t* p = active ? reinterpret_cast<const uint8_t*>(xq + (int64_t)min(m, M - 1) * K) + 64 * ch
+                                  : reinterpret_cast<const uint8_t*>(g_zero_chunk);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) a[m][q] = 0u;
+        for (int v = 0; v < 4; ++v) {
+            const uint4 u = ld_shared_ro16(p + 16 * v);
+            a[m][4 * v + 0] = u.x;
+            a[m][4 * v + 1] = u.y;
+            a[m][4 * v + 2] = u.z;
+            a[m][4 * v + 3] = u.w;
+        }
+    }
+}
+
+// Σx̃ of each of the MT tokens of a global x̃ row (every lane gets the
+// totals; tokens past M give 0): one pass over the row by the warp.
+template <int MT>
+__device__ __forceinline__ void warp_xsum(const int8_t* xq, int M, int K, int C, int full_chunks, int lane,
+                                          int (&sx)[MT]) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        int t = 0;
+        if (m < M) {
+            const int8_t* row = xq + (int64_t)m * K;
+            for (int ch = lane; ch < C; ch += 32) {
+                uint32_t a[16];
+                if (ch < full_chunks) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const uint4 u = ld_shared_ro16(row + 64 * ch + 16 * v);
+                        a[4 * v + 0] = u.x;
+                        a[4 * v + 1] = u.y;
+                        a[4 * v + 2] = u.z;
+                        a[4 * v + 3] = u.w;
+                    }
+                } else {
+                    uint32_t tmp[16];  // the rare tail goes through local memory
+                    load_act_tail(row, K, ch, tmp);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) a[q] = tmp[q];
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q) t = dp4a_s8s8(0x01010101u, a[q], t);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+        sx[m] = t;
+    }
+}
+
+// acc[r][m][q] += codes × x̃ for one step: per (word, field) the RG rows'
+// codes are masked first, then their dp4a go to RG independent accumulators.
+// With NQ = 4 field q keeps its codes in place (×4^q, summed with a shift at
+// the end); with NQ = 1 the codes are shifted down.
+template <int RG, int MT, int NQ>
+__device__ __forceinline__ void step_math(const uint4 (&w)[RG], const uint32_t (&xa)[MT][16],
+                                          int (&acc)[RG][MT][NQ]) {
+#pragma unroll
+    for (int wj = 0; wj < 4; ++wj) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t codes[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                const uint32_t word = word_of(w[r], wj);
+                codes[r] = NQ == 4 ? (word & (0x03030303u << (2 * q))) : ((word >> (2 * q)) & 0x03030303u);
+            }
+#pragma unroll
+            for (int r = 0; r < RG; ++r)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    int& a = acc[r][m][NQ == 4 ? q : 0];
+                    a = dp4a_u8s8(codes[r], xa[m][4 * wj + q], a);
+                }
         }
     }
 }
 
 // MT tokens (M <= MT), W warps per CTA, MINB CTAs per SM, row groups of RG
-// rows.  A warp walks its range one "step" at a time: up to 32 chunks of one
-// row group, one chunk per lane, the RG rows' words loaded straight into
-// registers; with PF the next step's words are requested before this step's
-// arithmetic.
-template <int MT, int W, int MINB, int RG, bool PF, bool FUSE>
+// rows, D stages.  A warp walks its range one step at a time (up to 32
+// chunks of one row group, one chunk per lane).  Each warp has a ring of D
+// shared-memory stages (RG rows × 512 bytes): lane l copies its own 16 bytes
+// of every row with cp.async and later reads back only those, so the wait is
+// per thread and needs no warp barrier.  D-1 steps are in flight while one is
+// computed; the first D-1 are requested before the dependency wait.  Σx̃ is
+// not accumulated per step: the warp that holds a row group's first chunk
+// subtracts the token's whole-row Σx̃ once, so every row's total is
+// Σ c·x̃ - Σ x̃ over the full row.
+template <int MT, int W, int MINB, int RG, int D, bool FUSE>
 __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_constant__ GParams P) {
-    constexpr bool kFields = MT <= 2;  // one accumulator per code field (no shifts)
-    constexpr int NQ = kFields ? 4 : 1;
-    constexpr int V = RG * MT;         // sums per lane when a row group is done
+    constexpr int NQ = MT <= 2 ? 4 : 1;  // one accumulator per code field (no shifts) for few tokens
+    constexpr int V = RG * MT;           // sums per lane when a row group is done
+    constexpr uint32_t kStage = RG * 512;
     static_assert(RG <= kRGMax && V <= 32, "row group too large");
+    static_assert(D >= 2, "at least one step in flight");
     using Shared = GShared<W>;
-    static_assert(sizeof(Shared) % 16 == 0, "the x̃ slots after the shared block need 16-byte alignment");
+    static_assert(sizeof(Shared) % 16 == 0, "the stages after the shared block need 16-byte alignment");
     extern __shared__ __align__(128) uint8_t smem_raw[];
     Shared& S = *reinterpret_cast<Shared*>(smem_raw);
     const int warp = threadIdx.x >> 5;
@@ -462,28 +553,32 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
 
     // ---- CTA and warp ranges (equal chunk counts, CTA edges on row groups)
     for (int i = threadIdx.x; i < P.count; i += W * 32) S.prob[i] = P.p[i];
+    if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(S.zero)[threadIdx.x] = 0u;
+    if (threadIdx.x < kMaxSlots * kGemvMaxTokens) (&S.xsum[0][0])[threadIdx.x] = 0;
     __syncthreads();
     const GProblem* T = S.prob;
     const int count = P.count;
-    int64_t ca, cb;
-    cta_units(T, count, P.total_units, blockIdx.x, gridDim.x, ca, cb);
+    const int64_t ca = P.cta_begin[blockIdx.x], cb = P.cta_begin[blockIdx.x + 1];
     if (threadIdx.x <= W) S.bound[threadIdx.x] = ca + ((cb - ca) * threadIdx.x) / W;
     __syncthreads();
     const int64_t wu0 = S.bound[warp], wu1 = S.bound[warp + 1];
 
-    // ---- the first step's weights do not depend on the previous kernel
-    Cursor cur, nxt;
-    cursor_seek(T, count, cur, wu0, wu1);
+    // ---- the first D-1 steps' weights do not depend on the previous kernel
+    const uint32_t ring = smem_addr(smem_raw + sizeof(Shared)) + (uint32_t)warp * (D * kStage) + 16u * lane;
+    Walk cur, nxt;
+    walk_seek(T, count, cur, wu0, wu1);
     nxt = cur;
-    uint4 w[RG];
-    int n = 0;
-    bool have_w = false;  // w holds the current step's words
-    if (cur.u < cur.end) {
-        const GProblem& pr = T[cur.p];
-        n = cursor_len<32>(pr, cur);
-        load_rows<RG>(pr, cur.rg, cur.c + lane, lane < n, w);
-        have_w = true;
-        cursor_advance(pr, nxt, n);
+    int nq[D - 1];  // chunk counts of the steps in flight; nq[0] is the current step's
+#pragma unroll
+    for (int d = 0; d < D - 1; ++d) {
+        nq[d] = 0;
+        if (nxt.u < nxt.end) {
+            const GProblem& pq = T[nxt.p];
+            nq[d] = walk_len(pq, nxt);
+            stage_step<RG>(pq, nxt, nq[d], lane, ring + d * kStage);
+            walk_advance(pq, nxt);
+        }
+        cp_async_commit();
     }
     griddep_wait();  // x̃, β (and α) may come from the preceding kernels
 
@@ -492,17 +587,17 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
     int second_slot = 1;  // slot of the CTA's second problem (0 when it shares the first one's input)
     uint32_t xs_base = 0;
     if constexpr (FUSE) {
-        uint8_t* xs = smem_raw + sizeof(Shared);
+        uint8_t* xs = smem_raw + sizeof(Shared) + W * D * kStage;
         xs_base = smem_addr(xs);
-        p_first = problem_of_unit(T, count, ca);
-        const int p_last = cb > ca ? problem_of_unit(T, count, cb - 1) : p_first;
+        p_first = problem_of_step(T, count, ca);
+        const int p_last = cb > ca ? problem_of_step(T, count, cb - 1) : p_first;
         QRow rows[kMaxSlots * MT];
         int nr = 0;
         for (int slot = 0; slot < kMaxSlots && ca < cb; ++slot) {
             const int p = p_first + slot;
             if (p > p_last) break;
             const GProblem& pr = T[p];
-            const bool owner = ca <= pr.unit_begin && pr.unit_begin < cb;
+            const bool owner = ca <= pr.step_begin && pr.step_begin < cb;
             if (slot == 1) {
                 const GProblem& p0 = T[p_first];
                 if (pr.x == p0.x && pr.x2 == p0.x2 && pr.K == p0.K && pr.M == p0.M) {
@@ -514,7 +609,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                 }
             }
             for (int m = 0; m < pr.M && m < MT; ++m)
-                rows[nr++] = QRow{&pr, m, xs + (slot * MT + m) * P.slot_row, &S.xbeta[slot][m],
+                rows[nr++] = QRow{&pr, m, xs + (slot * MT + m) * P.slot_row, &S.xbeta[slot][m], &S.xsum[slot][m],
                                   owner && pr.write_outputs != 0};
         }
         for (int i = 0; i < nr; i += kFuseRows) {
@@ -525,113 +620,107 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
         }
         __syncthreads();
     }
+    const uint32_t zero_addr = smem_addr(S.zero);
 
-    // ---- main loop over this warp's steps
-    int sp = -1;                          // problem of the α, β this lane holds
-    float alpha_v = 0.0f, beta_v = 0.0f;  // lane m < MT: α and β of token m, loaded ahead of use
-    int scale_p = -1;                     // problem of the scale below
-    float my_scale = 0.0f;                // lane m < MT: dequant scale of token m
-    uint32_t xrow0 = 0;                   // fused: shared address of the problem's slot
+    // ---- state of the problem of the current step
+    int sp = -1;                          // that problem
+    float alpha_v = 0.0f, beta_v = 0.0f;  // lane m < MT: α and token m's β
+    int sx[MT];                           // Σx̃ of each token over the whole row
+    uint32_t xrow = 0;                    // fused: shared address of the problem's slot
+    const int8_t* xq = nullptr;           // unfused: the problem's x̃ and its shape
+    int xM = 1, xK = 0, xfull = 0;
+    int scale_p = -1;       // problem of my_scale
+    float my_scale = 0.0f;  // lane m < MT: dequant scale of token m
+#pragma unroll
+    for (int m = 0; m < MT; ++m) sx[m] = 0;
+
     int acc[RG][MT][NQ];
-    int sx[MT];                           // this lane's Σx̃ over the chunks it added (per token)
-    int rg_chunks = 0;                    // chunks of the current row group done by this warp
-    int own_p = -1, own_rg = 0;           // a shared row group this warp finishes after the loop
+    bool fresh = true;           // the next step begins a row group for this warp
+    bool rg_own = false;         // this warp holds the current row group's first chunk
+    int own_p = -1, own_rg = 0;  // a shared row group this warp finishes after the loop
+    uint32_t stage = ring;       // the current step's stage
+    uint32_t fill = ring + (D - 1) * kStage;  // the stage the next request goes to
 
-    while (cur.u < cur.end) {
-        const GProblem& pr = T[cur.p];
-        if (cur.p != sp) {
+    while (nq[0] > 0) {
+        if (cur.p != sp) {  // entering a problem: its α, β, Σx̃ and activations
             sp = cur.p;
-            if constexpr (FUSE) xrow0 = xs_base + (uint32_t)((cur.p == p_first ? 0 : second_slot) * MT) * P.slot_row;
+            const GProblem& pr = T[sp];
             alpha_v = *pr.alpha;
-            if (lane < MT && lane < pr.M) {
-                if constexpr (FUSE)
-                    beta_v = S.xbeta[cur.p == p_first ? 0 : second_slot][lane];
-                else
-                    beta_v = pr.beta[lane];
+            if constexpr (FUSE) {
+                const int slot = sp == p_first ? 0 : second_slot;
+                xrow = xs_base + (uint32_t)(slot * MT) * (uint32_t)P.slot_row;
+                if (lane < MT) beta_v = S.xbeta[slot][lane];
+#pragma unroll
+                for (int m = 0; m < MT; ++m) sx[m] = S.xsum[slot][m];
+            } else {
+                xq = pr.xq;
+                xM = pr.M;
+                xK = pr.K;
+                xfull = pr.full_chunks;
+                if (lane < MT && lane < pr.M) beta_v = pr.beta[lane];
+                warp_xsum<MT>(pr.xq, pr.M, pr.K, pr.C, pr.full_chunks, lane, sx);
             }
         }
-        if (rg_chunks == 0) {  // first step of a row group for this warp
+        if (fresh) {
 #pragma unroll
             for (int r = 0; r < RG; ++r)
 #pragma unroll
                 for (int m = 0; m < MT; ++m)
 #pragma unroll
                     for (int q = 0; q < NQ; ++q) acc[r][m][q] = 0;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) sx[m] = 0;
+            rg_own = cur.s == 0;
+            fresh = false;
         }
-        if constexpr (!PF) {  // this step's weights (the first step's were requested in the prologue)
-            if (!have_w) load_rows<RG>(pr, cur.rg, cur.c + lane, lane < n, w);
-            have_w = false;
-        }
-        const bool valid = lane < n;
-        uint32_t xa[MT][16];
-        load_x<MT, FUSE>(pr, xrow0, P.slot_row, cur.c + lane, valid, xa);
-
-        // request the next step's weights before this step's arithmetic
-        uint4 wn[PF ? RG : 1];
+        const int nc = nq[0];
+        // request the step D-1 ahead into the stage freed by the previous step
         int nn = 0;
         if (nxt.u < nxt.end) {
             const GProblem& pq = T[nxt.p];
-            nn = cursor_len<32>(pq, nxt);
-            if constexpr (PF) load_rows<RG>(pq, nxt.rg, nxt.c + lane, lane < nn, wn);
+            nn = walk_len(pq, nxt);
+            stage_step<RG>(pq, nxt, nn, lane, fill);
+            walk_advance(pq, nxt);
         }
+        cp_async_commit();
+        cp_async_wait<D - 1>();  // this lane's copies of the current step have landed
+        uint4 w[RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) w[r] = lds128_after(stage + 512u * r);
 
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int q = 0; q < 16; ++q) sx[m] = dp4a_s8s8(0x01010101u, xa[m][q], sx[m]);
-#pragma unroll
-        for (int wj = 0; wj < 4; ++wj) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t codes[RG];  // the RG rows' codes of this (word, field), then their products
-#pragma unroll
-                for (int r = 0; r < RG; ++r) {
-                    const uint32_t word = word_of(w[r], wj);
-                    codes[r] = kFields ? (word & (0x03030303u << (2 * q))) : ((word >> (2 * q)) & 0x03030303u);
-                }
-#pragma unroll
-                for (int r = 0; r < RG; ++r)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        int& a = acc[r][m][kFields ? q : 0];
-                        a = dp4a_u8s8(codes[r], xa[m][4 * wj + q], a);
-                    }
-            }
-        }
+        const bool active = lane < nc;
+        const int ch = 32 * cur.s + lane;
+        uint32_t xa[MT][16];
+        if constexpr (FUSE)
+            lds_x<MT>(xrow, P.slot_row, ch, active, zero_addr, xa);
+        else
+            ldg_x<MT>(xq, xM, xK, xfull, ch, active, xa);
+        step_math<RG, MT, NQ>(w, xa, acc);
 
-        rg_chunks += n;
-        const bool rg_whole = (cur.c + n == pr.C) && (rg_chunks == pr.C);
-        const bool rg_done = (cur.c + n == pr.C) || (cur.u + n == cur.end);
-        const int seg_p = cur.p;
-        const int rg = cur.rg;
-        const int64_t rg_u0 = pr.unit_begin + (int64_t)rg * pr.C;
-
-        if (rg_done) {
+        const GProblem& pr = T[sp];
+        const bool rg_end = cur.s + 1 == pr.S;
+        if (rg_end || cur.u + 1 == cur.end) {
+            // this warp's sums of the row group; the holder of its first
+            // chunk takes Σx̃ off (in one lane, so once)
+            const bool sub = lane == 0 && rg_own;
             int v[V];
 #pragma unroll
             for (int r = 0; r < RG; ++r)
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    if constexpr (kFields)
-                        v[m * RG + r] =
-                            acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6) - sx[m];
-                    else
-                        v[m * RG + r] = acc[r][m][0] - sx[m];
+                    int t = acc[r][m][0];
+                    if constexpr (NQ == 4) t += (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) + (acc[r][m][3] >> 6);
+                    v[m * RG + r] = t - (sub ? sx[m] : 0);
                 }
             int idx;
-            int val = reduce_scatter<V>(v, lane, idx);
+            const int val = reduce_scatter<V>(v, lane, idx);
             const bool writer = (lane & (32 / V - 1)) == 0;
             const int r = idx % RG, m = idx / RG;
-
-            if (rg_whole) {
-                if (scale_p != seg_p) {  // once per problem: α·β/127 of each token
-                    scale_p = seg_p;
+            if (rg_own && rg_end) {  // the whole row group: write y
+                if (scale_p != sp) {
+                    scale_p = sp;
                     my_scale = dequant_scale(alpha_v, beta_v);
                 }
                 const float sc = __shfl_sync(0xffffffffu, my_scale, m);
-                const int row = rg * RG + r;
+                const int row = cur.rg * RG + r;
                 if (writer && row < pr.N && m < pr.M) {
                     float out = __fmul_rn((float)val, sc);
                     if (pr.bias) out = __fadd_rn(out, pr.bias[row]);
@@ -640,34 +729,31 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                 }
             } else {
                 // a row group shared with the neighbouring warps: keep this
-                // warp's part; the warp holding its first chunk adds the parts
-                // up after the main loop
-                const bool starts_here = rg_u0 >= wu0;
-                if (writer) S.part[warp][starts_here ? 1 : 0][idx] = val;
-                if (starts_here) {
-                    own_p = seg_p;
-                    own_rg = rg;
+                // warp's part; the holder of its first chunk adds the parts up
+                // after the main loop
+                if (writer) S.part[warp][rg_own ? 1 : 0][idx] = val;
+                if (rg_own) {
+                    own_p = sp;
+                    own_rg = cur.rg;
                 }
             }
-            rg_chunks = 0;
+            fresh = true;
         }
-
-        // move to the next step
-        cursor_advance(pr, cur, n);
-        if constexpr (PF) {
+        walk_advance(pr, cur);
 #pragma unroll
-            for (int r = 0; r < RG; ++r) w[r] = wn[r];
-        }
-        n = nn;
-        if (nxt.u < nxt.end) cursor_advance(T[nxt.p], nxt, nn);
+        for (int d = 0; d + 1 < D - 1; ++d) nq[d] = nq[d + 1];
+        nq[D - 2] = nn;
+        fill = stage;
+        stage = stage + kStage == ring + D * kStage ? ring : stage + kStage;
     }
+    cp_async_wait<0>();
 
     // ---- row groups shared between warps: the warp holding the first chunk
     // adds the parts of the warps after it that worked on the same row group
     __syncthreads();
     if (own_p >= 0) {
         const GProblem& pr = T[own_p];
-        const int64_t rg_end = pr.unit_begin + (int64_t)(own_rg + 1) * pr.C;
+        const int64_t rg_end = pr.step_begin + (int64_t)(own_rg + 1) * pr.S;
         int idx = 0;
 #pragma unroll
         for (int half = V / 2, off = 16; half >= 1; half >>= 1, off >>= 1)
@@ -762,18 +848,15 @@ template <int MT>
 struct StreamCfg;
 template <>
 struct StreamCfg<1> {
-    static constexpr int W = 12, MINB = 1, RG = 8;
-    static constexpr bool PF = true;
+    static constexpr int W = 12, MINB = 1, RG = 8, D = 2;
 };
 template <>
 struct StreamCfg<2> {
-    static constexpr int W = 12, MINB = 1, RG = 4;
-    static constexpr bool PF = true;
+    static constexpr int W = 12, MINB = 1, RG = 4, D = 4;
 };
 template <>
 struct StreamCfg<4> {
-    static constexpr int W = 8, MINB = 1, RG = 4;
-    static constexpr bool PF = true;
+    static constexpr int W = 8, MINB = 1, RG = 4, D = 4;
 };
 
 constexpr size_t kSmemOptIn = 232448;  // opt-in dynamic shared memory per block on sm_100
@@ -799,17 +882,80 @@ void fill_params(GParams& P, const bitlinear_forward_problem* problems, int coun
         q.C = q.row_bytes / 16;
         q.full_chunks = q.K / 64;
         q.rgn = (q.N + RG - 1) / RG;
-        q.unit_begin = total;
-        total += (int64_t)q.rgn * q.C;
+        q.S = (q.C + 31) / 32;
+        q.step_begin = total;
+        total += (int64_t)q.rgn * q.S;
     }
-    P.total_units = total;
+    P.total_steps = total;
 }
 
-// Launches gemv_stream_kernel<MT, W, MINB, RG, PF, fused>; with `fused` (one entry per
+// Prologue cost of quantising one input row of K elements in a CTA of W
+// warps, in warp-steps (the time one warp takes for one step): measured on
+// B200 with 12 warps as about 1.27 + K / 4930 step times.
+inline double prologue_cost(int W, int64_t K) { return W * (1.27 + (double)K / 4930.0); }
+
+// Splits the steps of P into at most G contiguous CTA ranges of whole row
+// groups whose costs (their steps, plus, with `pro`, the prologue cost of
+// each distinct input they quantise) are as even as a greedy fill allows:
+// the smallest cost bound T for which the fill needs at most G CTAs is found
+// by bisection.  Writes P.cta_begin[0..n] and returns n (the CTAs to launch).
+int cta_ranges(GParams& P, int G, const double* pro) {
+    const int count = P.count;
+    auto same_input = [&](int a, int b) {
+        return P.p[a].x == P.p[b].x && P.p[a].x2 == P.p[b].x2 && P.p[a].K == P.p[b].K && P.p[a].M == P.p[b].M;
+    };
+    auto fill = [&](double T, bool write) {
+        int c = 0;
+        double cost = 0.0;
+        int64_t pos = 0;
+        int last = -1;  // the last problem the current CTA took
+        if (write) P.cta_begin[0] = 0;
+        for (int p = 0; p < count; ++p) {
+            const GProblem& q = P.p[p];
+            int64_t left = q.rgn;
+            while (left > 0) {
+                const double pc = (!pro || last == p || (last >= 0 && same_input(p, last))) ? 0.0 : pro[p];
+                const double room = T - cost - pc;
+                int64_t k = room >= q.S ? (int64_t)(room / q.S) : 0;
+                if (k == 0) {
+                    if (cost == 0.0) {
+                        k = 1;  // an empty CTA takes one row group even above T
+                    } else {
+                        ++c;
+                        if (write && c <= kMaxCta) P.cta_begin[c] = (int32_t)pos;
+                        cost = 0.0;
+                        last = -1;
+                        continue;
+                    }
+                }
+                if (k > left) k = left;
+                cost += pc + (double)k * q.S;
+                last = p;
+                pos += k * q.S;
+                left -= k;
+            }
+        }
+        if (write && c + 1 <= kMaxCta) P.cta_begin[c + 1] = (int32_t)pos;
+        return c + 1;
+    };
+    double lo = 0.0, hi = 0.0;
+    for (int p = 0; p < count; ++p) hi += (double)P.p[p].rgn * P.p[p].S + (pro ? pro[p] : 0.0);
+    hi += 1.0;
+    for (int it = 0; it < 40 && hi - lo > 0.5; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (fill(mid, false) <= G)
+            hi = mid;
+        else
+            lo = mid;
+    }
+    return fill(hi, true);
+}
+
+// Launches gemv_stream_kernel<MT, W, MINB, RG, D, fused>; with `fused` (one entry per
 // problem) the kernel quantises x itself, if every CTA's range meets at most
 // two problems, the slots fit shared memory and the CTAs' input reads stay
 // small next to the weights (else *launched = false and nothing runs).
-template <int MT, int W, int MINB, int RG, bool PF>
+template <int MT, int W, int MINB, int RG, int D>
 cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
                               cudaStream_t stream, bool pdl, const FusedInput* fused, bool x_bf16, bool* launched,
                               bool fuse_always) {
@@ -817,14 +963,12 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
     if (launched) *launched = true;
     GParams P;
     fill_params(P, problems, count, RG);
-    int64_t row_groups = 0, weight_bytes = 0;
-    for (int i = 0; i < count; ++i) {
-        row_groups += P.p[i].rgn;
-        weight_bytes += (int64_t)P.p[i].N * P.p[i].row_bytes;
-    }
-    int64_t grid = (int64_t)dev.sm_count * MINB;
-    if (grid > row_groups) grid = row_groups;
-    size_t smem = sizeof(Shared);
+    int64_t weight_bytes = 0;
+    for (int i = 0; i < count; ++i) weight_bytes += (int64_t)P.p[i].N * P.p[i].row_bytes;
+    if (P.total_steps >= INT32_MAX) return cudaErrorInvalidValue;  // over 8 TB of weights in one call
+    const int G = (int)std::min<int64_t>((int64_t)dev.sm_count * MINB, kMaxCta);
+    int grid = 0;
+    size_t smem = sizeof(Shared) + (size_t)W * D * RG * 512;  // the table, then the warps' stage rings
     const size_t smem_cap = kSmemOptIn / MINB - (MINB > 1 ? 1024 : 0);
     if (fused) {
         int32_t slot_row = 0;
@@ -842,17 +986,19 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
         // the prologue holds a row in registers: at most W·32·kFuseVec 16-byte vectors
         for (int i = 0; i < count; ++i)
             fits = fits && (int64_t)P.p[i].K * (x_bf16 ? 2 : 4) <= (int64_t)W * 32 * kFuseVec * 16;
+        double pro[kMaxGroup];
+        for (int i = 0; i < count; ++i) pro[i] = prologue_cost(W, P.p[i].K) * std::min<int>(P.p[i].M, MT);
+        grid = cta_ranges(P, G, pro);
         // Every CTA reads its problems' whole input rows before its main loop;
         // that pays off only while those reads are small next to the weights.
         auto input_bytes = [&](const GProblem& q) {
             return (int64_t)q.M * q.K * (x_bf16 ? 2 : 4) * (q.x2 ? 2 : 1);
         };
         int64_t prologue_bytes = 0;
-        for (int64_t c = 0; c < grid && fits; ++c) {
-            int64_t a, b;
-            cta_units(P.p, count, P.total_units, c, grid, a, b);
+        for (int c = 0; c < grid && fits; ++c) {
+            const int64_t a = P.cta_begin[c], b = P.cta_begin[c + 1];
             if (a >= b) continue;
-            const int pa = problem_of_unit(P.p, count, a), pb = problem_of_unit(P.p, count, b - 1);
+            const int pa = problem_of_step(P.p, count, a), pb = problem_of_step(P.p, count, b - 1);
             fits = pb - pa <= 1;
             prologue_bytes += input_bytes(P.p[pa]);
             if (pb != pa && !(P.p[pb].x == P.p[pa].x && P.p[pb].x2 == P.p[pa].x2)) prologue_bytes += input_bytes(P.p[pb]);
@@ -863,9 +1009,12 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
             return cudaSuccess;
         }
         smem += (size_t)kMaxSlots * MT * slot_row;
+    } else {
+        grid = cta_ranges(P, G, nullptr);
     }
-    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, PF, true>)
-                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, PF, false>);
+    if (smem > smem_cap) return cudaErrorInvalidConfiguration;  // a shape that does not fit (not built)
+    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, D, true>)
+                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, D, false>);
     // the opt-in is per device: set once on each device that launches the kernel
     cudaError_t err = set_max_dynamic_smem(kernel, (int)smem_cap);
     if (err != cudaSuccess) return err;
@@ -888,7 +1037,7 @@ cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, 
                           cudaStream_t stream, bool pdl, const FusedInput* fused = nullptr, bool x_bf16 = false,
                           bool* launched = nullptr, bool fuse_always = false) {
     using C = StreamCfg<MT>;
-    return launch_stream_cfg<MT, C::W, C::MINB, C::RG, C::PF>(problems, count, dev, stream, pdl, fused, x_bf16,
+    return launch_stream_cfg<MT, C::W, C::MINB, C::RG, C::D>(problems, count, dev, stream, pdl, fused, x_bf16,
                                                               launched, fuse_always);
 }
 
