@@ -66,32 +66,41 @@ __device__ __forceinline__ float dequant_scale(float alpha, float beta) {
     return __double2float_rn(s);
 }
 
+// Per-row factor of the fast path of quantize_one: c = RN(127·RN(1/β)), or
+// NaN (every element takes the exact path) when β >= 2^120 or is not finite,
+// where RN(1/β) could lose relative precision.
+__device__ __forceinline__ float quant_factor(float beta, float scale) {
+    return beta < 0x1p120f ? __fmul_rn(scale, __frcp_rn(beta)) : __int_as_float(0x7fffffff);
+}
+
 // clip(rint(RN(RN(127·v) / β)), -127, 127), exactly (the per-token int8
-// quantisation of "1.58-bit 大模型极限量化实战" §2.4).  With a = RN(127·v) and
-// |v| <= β, |a/β| <= 127·(1 + 2^-24), so q = RN(a·RN(1/β)) is within
-// 127·2^-23 < 1.6e-5 of a/β, and RN(a/β) within 127·2^-24 of it.  When q is
-// farther than 1e-4 from every half-integer, both lie on the same side of it
-// and round to the same integer; otherwise (rare, and for non-finite q) the
-// correctly rounded quotient is taken.  rbeta = RN(1/β).
-__device__ __forceinline__ int8_t quantize_one(float v, float beta, float rbeta) {
-    const float a = __fmul_rn(v, 127.0f);
-    const float q = __fmul_rn(a, rbeta);
+// quantisation of "1.58-bit 大模型极限量化实战" §2.4), with c = quant_factor(β, 127).
+// Fast path: q = RN(v·c) is within 4·2^-24 relative of t = RN(127·v)/β
+// (three binary32 roundings against one), so for |v| <= β it is within
+// 127·4·2^-24 + 127·2^-24 < 4e-5 of RN(t).  When q is farther than 1e-4 from
+// every half-integer, q and RN(t) lie on the same side of it and round to the
+// same integer, which is at most 127 in magnitude (|q| < 127.5), so no clip
+// is needed.  Otherwise (rare; always for non-finite q) the exact quotient
+// is taken and clipped.
+__device__ __forceinline__ int8_t quantize_one(float v, float beta, float c) {
+    const float q = __fmul_rn(v, c);
     float r = rintf(q);  // round half to even
-    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) r = rintf(__fdiv_rn(a, beta));
-    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) {
+        r = rintf(__fdiv_rn(__fmul_rn(v, 127.0f), beta));
+        r = fminf(fmaxf(r, -127.0f), 127.0f);
+    }
     return (int8_t)__float2int_rn(r);
 }
 
 // clip(rint(RN(RN(7·v) / β)), -7, 7): the 4-bit variant of quantize_one, with
-// the same argument (|a/β| <= 7·(1 + 2^-24), so q = RN(a·RN(1/β)) is within
-// 7·2^-23 of a/β; away from half-integers by more than 1e-4 both round alike,
-// otherwise the correctly rounded quotient is taken).
-__device__ __forceinline__ int quantize_one_a4(float v, float beta, float rbeta) {
-    const float a = __fmul_rn(v, 7.0f);
-    const float q = __fmul_rn(a, rbeta);
+// c = quant_factor(β, 7) and the same argument (q within 7·5·2^-24 of RN(t)).
+__device__ __forceinline__ int quantize_one_a4(float v, float beta, float c) {
+    const float q = __fmul_rn(v, c);
     float r = rintf(q);
-    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) r = rintf(__fdiv_rn(a, beta));
-    r = fminf(fmaxf(r, -7.0f), 7.0f);
+    if (!(fabsf(__fsub_rn(q, r)) < 0.4999f)) {
+        r = rintf(__fdiv_rn(__fmul_rn(v, 7.0f), beta));
+        r = fminf(fmaxf(r, -7.0f), 7.0f);
+    }
     return __float2int_rn(r);
 }
 

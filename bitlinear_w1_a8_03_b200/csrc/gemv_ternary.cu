@@ -137,13 +137,27 @@ __device__ __forceinline__ float block_max_n(float mx, float* red) {
 // 16 bytes of x (+ x2): 8 bfloat16 or 4 float32 elements, kept raw in
 // registers between the absmax and the quantisation (a float32 sum x + x2 is
 // formed on load, one binary32 rounding).
+// One input row the fused prologue quantises into a shared slot row; the
+// fields are copied by value so the prologue reads them from registers.
+struct QRow {
+    const void* x;    // the problem's activations, float32 or bfloat16 [M][K]
+    const float* x2;  // nullable float32 second addend
+    int8_t* xq;       // x̃ out (with `out`)
+    float* beta;      // β out (with `out`)
+    float* x_sum;     // nullable x (+ x2) out (with `out`)
+    uint32_t dst;     // shared address of the slot row
+    int slot, m, K;
+    bool valid;  // a row to quantise
+    bool out;    // also write x̃, β (and x) to global memory
+};
+
 template <typename T>
 struct FusedVec;
 template <>
 struct FusedVec<uint16_t> {
     static constexpr int n = 8;
-    __device__ static uint4 load(const GProblem& pr, int64_t e) {
-        return ld_shared_ro16(static_cast<const uint16_t*>(pr.x) + e);
+    __device__ static uint4 load(const QRow& q, int64_t e) {
+        return ld_shared_ro16(static_cast<const uint16_t*>(q.x) + e);
     }
     __device__ static void unpack(const uint4& u, float (&f)[8]) {
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -157,10 +171,10 @@ struct FusedVec<uint16_t> {
 template <>
 struct FusedVec<float> {
     static constexpr int n = 4;
-    __device__ static uint4 load(const GProblem& pr, int64_t e) {
-        uint4 u = ld_shared_ro16(static_cast<const float*>(pr.x) + e);
-        if (pr.x2) {
-            const uint4 v = ld_shared_ro16(pr.x2 + e);
+    __device__ static uint4 load(const QRow& q, int64_t e) {
+        uint4 u = ld_shared_ro16(static_cast<const float*>(q.x) + e);
+        if (q.x2) {
+            const uint4 v = ld_shared_ro16(q.x2 + e);
             u.x = __float_as_uint(__fadd_rn(__uint_as_float(u.x), __uint_as_float(v.x)));
             u.y = __float_as_uint(__fadd_rn(__uint_as_float(u.y), __uint_as_float(v.y)));
             u.z = __float_as_uint(__fadd_rn(__uint_as_float(u.z), __uint_as_float(v.z)));
@@ -179,45 +193,36 @@ struct FusedVec<float> {
 constexpr int kFuseVec = 8;  // 16-byte vectors per thread and row held in registers
 constexpr int kFuseRows = 2;  // input rows quantised together (one block reduction)
 
-// One input row the fused prologue quantises into a shared slot row.
-struct QRow {
-    const GProblem* pr;
-    int m;            // token
-    uint8_t* dst;     // slot row
-    float* beta_dst;  // slot β
-    int* sum_dst;     // slot Σx̃ (zeroed before; the CTA's threads add their parts)
-    bool out;         // also write x̃, β (and x) to global memory
-};
-
-// Quantises two input rows at once (the second may be absent) with the
-// arithmetic of act_quant_kernel (β = max|x| + 1e-8, x̃ = quantize_one), zero
-// past K: every load of both rows is issued before the first use, and one
-// block reduction yields both β.  Each row must fit NT·kFuseVec 16-byte
-// vectors (the host checks); K is a multiple of 16 and x, x2 are 16-byte
-// aligned.
+// Quantises the kFuseRows input rows q[] at once (invalid ones are skipped)
+// with the arithmetic of act_quant_kernel (β = max|x| + 1e-8, x̃ =
+// quantize_one), zero past K: every load of the rows is issued before the
+// first use, and one block reduction yields every β.  β and Σx̃ of a row go
+// to xbeta / xsum[slot][m] (xsum zeroed before; the CTA's warps add their
+// parts).  Each row must fit NT·kFuseVec 16-byte vectors (the host checks);
+// K is a multiple of 16 and x, x2 are 16-byte aligned.
 template <typename T, int NT>
-__device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, float (*red)[32]) {
+__device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row, float (*red)[32],
+                                    float (*xbeta)[kGemvMaxTokens], int (*xsum)[kGemvMaxTokens]) {
     constexpr int V = FusedVec<T>::n;
     uint4 raw[kFuseRows][kFuseVec];
     float mx[kFuseRows];
 #pragma unroll
     for (int i = 0; i < kFuseRows; ++i) {
         mx[i] = 0.0f;
-        if (i < nr) {
-            const GProblem& pr = *rows[i].pr;
-            const int64_t base = (int64_t)rows[i].m * pr.K;
-            const int nvec = pr.K / V;
+        if (q[i].valid) {
+            const int64_t base = (int64_t)q[i].m * q[i].K;
+            const int nvec = q[i].K / V;
 #pragma unroll
             for (int j = 0; j < kFuseVec; ++j) {
                 const int v = threadIdx.x + j * NT;
-                if (v < nvec) raw[i][j] = FusedVec<T>::load(pr, base + (int64_t)v * V);
+                if (v < nvec) raw[i][j] = FusedVec<T>::load(q[i], base + (int64_t)v * V);
             }
         }
     }
 #pragma unroll
     for (int i = 0; i < kFuseRows; ++i) {
-        if (i < nr) {
-            const int nvec = rows[i].pr->K / V;
+        if (q[i].valid) {
+            const int nvec = q[i].K / V;
 #pragma unroll
             for (int j = 0; j < kFuseVec; ++j) {
                 if ((int)threadIdx.x + j * NT < nvec) {
@@ -242,16 +247,14 @@ __device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, 
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kFuseRows; ++i) {
-        if (i >= nr) continue;
+        if (!q[i].valid) continue;
         float b = red[i][0];
 #pragma unroll
         for (int w = 1; w < NT / 32; ++w) b = fmaxf(b, red[i][w]);
         const float beta = __fadd_rn(b, 1e-8f);
-        const float rbeta = __frcp_rn(beta);
-        const QRow& q = rows[i];
-        const GProblem& pr = *q.pr;
-        const int64_t base = (int64_t)q.m * pr.K;
-        const int nvec = pr.K / V;
+        const float qf = quant_factor(beta, 127.0f);
+        const int64_t base = (int64_t)q[i].m * q[i].K;
+        const int nvec = q[i].K / V;
         int qsum = 0;  // this thread's part of Σx̃
 #pragma unroll
         for (int j = 0; j < kFuseVec; ++j) {
@@ -264,25 +267,25 @@ __device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, 
                 for (int g = 0; g < V / 4; ++g) {
                     uint32_t x = 0;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(f[4 * g + e], beta, rbeta) << (8 * e);
+                    for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(f[4 * g + e], beta, qf) << (8 * e);
                     wq[g] = x;
                     qsum = dp4a_s8s8(0x01010101u, x, qsum);
                 }
                 const int k = v * V;
 #pragma unroll
-                for (int g = 0; g < V / 4; ++g) *reinterpret_cast<uint32_t*>(q.dst + xs_offset(k + 4 * g)) = wq[g];
-                if (q.out) {
-                    int8_t* o = const_cast<int8_t*>(pr.xq) + base + k;
+                for (int g = 0; g < V / 4; ++g) sts32(q[i].dst + xs_offset(k + 4 * g), wq[g]);
+                if (q[i].out) {
+                    int8_t* o = q[i].xq + base + k;
                     if constexpr (V == 8)
                         *reinterpret_cast<uint2*>(o) = make_uint2(wq[0], wq[1]);
                     else
                         *reinterpret_cast<uint32_t*>(o) = wq[0];
-                    if (pr.x_sum) {
+                    if (q[i].x_sum) {
                         if constexpr (V == 4) {
-                            *reinterpret_cast<uint4*>(pr.x_sum + base + k) = raw[i][j];
+                            *reinterpret_cast<uint4*>(q[i].x_sum + base + k) = raw[i][j];
                         } else {
 #pragma unroll
-                            for (int e = 0; e < V; ++e) pr.x_sum[base + k + e] = f[e];
+                            for (int e = 0; e < V; ++e) q[i].x_sum[base + k + e] = f[e];
                         }
                     }
                 }
@@ -290,13 +293,12 @@ __device__ void fused_quantize_rows(const QRow* rows, int nr, int32_t slot_row, 
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
-        if ((threadIdx.x & 31) == 0) atomicAdd(q.sum_dst, qsum);  // integer: exact in any order
+        if ((threadIdx.x & 31) == 0) atomicAdd(&xsum[q[i].slot][q[i].m], qsum);  // integer: exact in any order
         if (threadIdx.x == 0) {
-            *q.beta_dst = beta;
-            if (q.out) const_cast<float*>(pr.beta)[q.m] = beta;
+            xbeta[q[i].slot][q[i].m] = beta;
+            if (q[i].out) q[i].beta[q[i].m] = beta;
         }
-        for (int k = pr.K + 4 * threadIdx.x; k < slot_row; k += 4 * NT)
-            *reinterpret_cast<uint32_t*>(q.dst + xs_offset(k)) = 0u;
+        for (int k = q[i].K + 4 * threadIdx.x; k < slot_row; k += 4 * NT) sts32(q[i].dst + xs_offset(k), 0u);
     }
 }
 
@@ -587,36 +589,59 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
     int second_slot = 1;  // slot of the CTA's second problem (0 when it shares the first one's input)
     uint32_t xs_base = 0;
     if constexpr (FUSE) {
-        uint8_t* xs = smem_raw + sizeof(Shared) + W * D * kStage;
-        xs_base = smem_addr(xs);
+        xs_base = smem_addr(smem_raw + sizeof(Shared) + W * D * kStage);
         p_first = problem_of_step(T, count, ca);
         const int p_last = cb > ca ? problem_of_step(T, count, cb - 1) : p_first;
+        // rows[slot·MT + m]: token m of the slot's problem (static indices keep them in registers)
         QRow rows[kMaxSlots * MT];
-        int nr = 0;
-        for (int slot = 0; slot < kMaxSlots && ca < cb; ++slot) {
+#pragma unroll
+        for (int slot = 0; slot < kMaxSlots; ++slot) {
             const int p = p_first + slot;
-            if (p > p_last) break;
-            const GProblem& pr = T[p];
-            const bool owner = ca <= pr.step_begin && pr.step_begin < cb;
-            if (slot == 1) {
-                const GProblem& p0 = T[p_first];
-                if (pr.x == p0.x && pr.x2 == p0.x2 && pr.K == p0.K && pr.M == p0.M) {
-                    // same input as slot 0: reuse it (the owner still publishes x̃, β)
-                    second_slot = 0;
-                    if (owner && pr.write_outputs && (pr.xq != p0.xq || pr.beta != p0.beta || pr.x_sum != p0.x_sum))
-                        second_slot = 1;  // distinct output buffers: quantise again to write them
-                    if (second_slot == 0) break;
+            bool use = ca < cb && p <= p_last;
+            bool owner = false;
+            if (use) {
+                const GProblem& pr = T[p];
+                owner = ca <= pr.step_begin && pr.step_begin < cb;
+                if (slot == 1) {
+                    const GProblem& p0 = T[p_first];
+                    if (pr.x == p0.x && pr.x2 == p0.x2 && pr.K == p0.K && pr.M == p0.M) {
+                        // same input as slot 0: reuse it (the owner still publishes x̃, β)
+                        second_slot = 0;
+                        if (owner && pr.write_outputs && (pr.xq != p0.xq || pr.beta != p0.beta || pr.x_sum != p0.x_sum))
+                            second_slot = 1;  // distinct output buffers: quantise again to write them
+                        use = second_slot == 1;
+                    }
                 }
             }
-            for (int m = 0; m < pr.M && m < MT; ++m)
-                rows[nr++] = QRow{&pr, m, xs + (slot * MT + m) * P.slot_row, &S.xbeta[slot][m], &S.xsum[slot][m],
-                                  owner && pr.write_outputs != 0};
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                QRow& r = rows[slot * MT + m];
+                r.valid = false;
+                if (use) {
+                    const GProblem& pr = T[p];
+                    r.valid = m < pr.M;
+                    r.x = pr.x;
+                    r.x2 = pr.x2;
+                    r.xq = const_cast<int8_t*>(pr.xq);
+                    r.beta = const_cast<float*>(pr.beta);
+                    r.x_sum = pr.x_sum;
+                    r.dst = xs_base + (uint32_t)((slot * MT + m) * P.slot_row);
+                    r.slot = slot;
+                    r.m = m;
+                    r.K = pr.K;
+                    r.out = owner && pr.write_outputs != 0;
+                }
+            }
         }
-        for (int i = 0; i < nr; i += kFuseRows) {
-            if (P.x_bf16)
-                fused_quantize_rows<uint16_t, W * 32>(rows + i, min(kFuseRows, nr - i), P.slot_row, S.red);
-            else
-                fused_quantize_rows<float, W * 32>(rows + i, min(kFuseRows, nr - i), P.slot_row, S.red);
+#pragma unroll
+        for (int i = 0; i < kMaxSlots * MT; i += kFuseRows) {
+            const QRow(&pair)[kFuseRows] = *reinterpret_cast<const QRow(*)[kFuseRows]>(&rows[i]);
+            if (pair[0].valid || pair[1].valid) {  // the same in every thread of the CTA
+                if (P.x_bf16)
+                    fused_quantize_rows<uint16_t, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum);
+                else
+                    fused_quantize_rows<float, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum);
+            }
         }
         __syncthreads();
     }
@@ -848,7 +873,7 @@ template <int MT>
 struct StreamCfg;
 template <>
 struct StreamCfg<1> {
-    static constexpr int W = 12, MINB = 1, RG = 8, D = 2;
+    static constexpr int W = 16, MINB = 1, RG = 8, D = 2;
 };
 template <>
 struct StreamCfg<2> {

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kMaxThreads) hadamard_kernel(const __grid_cons
             for (int e = 0; e < kE; ++e) mx = fmaxf(mx, fabsf(v[e]));  // zeros past K do not change it
         }
         const float beta = __fadd_rn(block_max_h(mx, red), 1e-8f);
-        const float rbeta = __frcp_rn(beta);
+        const float qf = quant_factor(beta, 127.0f);
         if (threadIdx.x == 0) P.beta[m] = beta;
         int8_t* q = P.x_q + m * P.K;
         for (int ti = 0; ti < ntiles; ++ti) {
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kMaxThreads) hadamard_kernel(const __grid_cons
             for (int g = 0; g < kE / 4; ++g) {
                 uint32_t x = 0;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(v[4 * g + e], beta, rbeta) << (8 * e);
+                for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(v[4 * g + e], beta, qf) << (8 * e);
                 w[g] = x;
             }
             if (vec && k0 + kE <= P.K && (reinterpret_cast<uintptr_t>(P.x_q) & 15) == 0) {

@@ -82,13 +82,13 @@ __device__ __forceinline__ float load_sum1(const T* x, const float* b, int64_t i
 }
 
 template <int V>
-__device__ __forceinline__ void store_codes(int8_t* q, const float* f, float beta, float rbeta) {
+__device__ __forceinline__ void store_codes(int8_t* q, const float* f, float beta, float qf) {
     uint32_t packed[V / 4];
 #pragma unroll
     for (int j = 0; j < V / 4; ++j) {
         uint32_t w = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)quantize_one(f[4 * j + b], beta, rbeta) << (8 * b);
+        for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)quantize_one(f[4 * j + b], beta, qf) << (8 * b);
         packed[j] = w;
     }
     if constexpr (V == 4) {
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
             }
         }
         const float beta = __fadd_rn(block_max(mx), 1e-8f);
-        const float rbeta = __frcp_rn(beta);
+        const float qf = quant_factor(beta, 127.0f);
         if (threadIdx.x == 0) pr.beta[m] = beta;
 #pragma unroll
         for (int j = 0; j < kVecPerThread; ++j) {
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
             if (i < nvec) {
                 float f[V];
                 Vec<T>::unpack(buf[j], f);
-                store_codes<V>(q + i * V, f, beta, rbeta);
+                store_codes<V>(q + i * V, f, beta, qf);
             }
         }
         return;
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
         for (int64_t i = threadIdx.x; i < K; i += nt) mx = fmaxf(mx, fabsf(load_sum1(x, b, i)));
     }
     const float beta = __fadd_rn(block_max(mx), 1e-8f);
-    const float rbeta = __frcp_rn(beta);
+    const float qf = quant_factor(beta, 127.0f);
     if (threadIdx.x == 0) pr.beta[m] = beta;
 
     if (vec) {
@@ -196,13 +196,13 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_kernel(const __grid_con
             }
             float f[V];
             Vec<T>::unpack(v, f);
-            store_codes<V>(q + i, f, beta, rbeta);
+            store_codes<V>(q + i, f, beta, qf);
         }
     } else {
         for (int64_t i = threadIdx.x; i < K; i += nt) {
             const float v = load_sum1(x, b, i);
             if (xs) xs[i] = v;
-            q[i] = quantize_one(v, beta, rbeta);
+            q[i] = quantize_one(v, beta, qf);
         }
     }
 }
@@ -228,11 +228,11 @@ __global__ void __launch_bounds__(kMaxThreads) act_quant_a4_kernel(const __grid_
     float mx = 0.0f;
     for (int64_t i = threadIdx.x; i < K; i += blockDim.x) mx = fmaxf(mx, fabsf(load_as_f32(x, i)));
     const float beta = __fadd_rn(block_max(mx), 1e-8f);
-    const float rbeta = __frcp_rn(beta);
+    const float qf = quant_factor(beta, 7.0f);
     if (threadIdx.x == 0) pr.beta[m] = beta;
     for (int64_t j = threadIdx.x; j < rb; j += blockDim.x) {
-        const int lo = quantize_one_a4(load_as_f32(x, 2 * j), beta, rbeta);
-        const int hi = 2 * j + 1 < K ? quantize_one_a4(load_as_f32(x, 2 * j + 1), beta, rbeta) : 0;
+        const int lo = quantize_one_a4(load_as_f32(x, 2 * j), beta, qf);
+        const int hi = 2 * j + 1 < K ? quantize_one_a4(load_as_f32(x, 2 * j + 1), beta, qf) : 0;
         q[j] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
     }
 }

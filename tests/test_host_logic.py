@@ -3,6 +3,9 @@ problem arrays, and the benchmark's byte accounting.  Tensors live on the
 CPU; nothing here calls into the CUDA library."""
 import ctypes
 
+import numpy as np
+import pytest
+
 import torch
 
 import bitlinear_w1_a8_03_b200 as bl
@@ -101,3 +104,58 @@ def test_kernel_attribute_set_once_per_device(tmp_path):
                            os.path.join(root, "tests", "native", "attr_once_check.cpp"), "-o", exe, "-pthread"])
     out = subprocess.run([exe], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout
+
+
+def _exact_code(v, beta, scale):
+    """clip(rint(RN(RN(scale·v) / β)), ±scale) in binary32 (the definition)."""
+    a = np.float32(v) * np.float32(scale)
+    return np.clip(np.rint(a / np.float32(beta)), -scale, scale)
+
+
+def _fast_code(v, beta, scale):
+    """The kernels' path: q = RN(v·RN(scale·RN(1/β))), kept when it is farther
+    than 1e-4 from every half-integer, else the definition."""
+    with np.errstate(invalid="ignore", over="ignore"):
+        c = np.float32(scale) * (np.float32(1.0) / np.float32(beta)) if beta < np.float32(2.0 ** 120) else np.float32(np.nan)
+        q = np.float32(v) * np.float32(c)
+        r = np.rint(q)
+        ok = np.abs(q - r) < np.float32(0.4999)
+    return np.where(ok, r, _exact_code(v, beta, scale)), ok
+
+
+@pytest.mark.parametrize("scale", [127, 7])
+def test_fast_quantisation_matches_the_definition(scale):
+    """The per-element fast path of the activation quantisers (one multiply by
+    a per-row factor, checked against the half-integers) gives the defined
+    code for every element: random rows over many binades, rows with
+    outliers, and values built to land within a few ulps of a half-integer."""
+    rng = np.random.default_rng(scale)
+    total = fast = 0
+    for trial in range(400):
+        K = 4096
+        x = (rng.standard_normal(K) * np.exp2(rng.integers(-60, 60))).astype(np.float32)
+        if trial % 3 == 0:
+            x[rng.integers(0, K, 4)] *= np.float32(50.0)
+        beta = np.float32(np.max(np.abs(x)) + np.float32(1e-8))
+        if trial % 2 == 1:  # near ties: v with v·scale/β = j + 1/2 + a few ulps
+            j = rng.integers(-scale, scale, K).astype(np.float64)
+            t = j + 0.5 + rng.integers(-6, 7, K) * 2.0 ** -19
+            x = np.clip((t * np.float64(beta) / scale), -np.float64(beta) * 0.9999999, np.float64(beta) * 0.9999999)
+            x = x.astype(np.float32)
+        got, ok = _fast_code(x, beta, scale)
+        want = _exact_code(x, beta, scale)
+        assert np.array_equal(got, want), trial
+        if trial % 2 == 0:
+            total += K
+            fast += int(ok.sum())
+    assert fast > 0.99 * total  # on ordinary rows the fast path does nearly all the work
+
+
+def test_fast_quantisation_non_finite_and_huge_rows():
+    for beta in (np.float32(np.inf), np.float32(np.nan), np.float32(3e38), np.float32(2.0 ** 121)):
+        x = np.array([0.0, 1.0, -2.5, 3e38, -np.inf, np.nan], dtype=np.float32)
+        for scale in (127, 7):
+            got, _ = _fast_code(x, beta, scale)
+            with np.errstate(invalid="ignore", over="ignore"):
+                want = _exact_code(x, beta, scale)
+            assert np.array_equal(got, want, equal_nan=True)
