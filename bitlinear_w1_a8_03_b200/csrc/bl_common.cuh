@@ -92,6 +92,38 @@ __device__ __forceinline__ int8_t quantize_one(float v, float beta, float c) {
     return (int8_t)__float2int_rn(r);
 }
 
+// quantize_one of N consecutive elements (N a multiple of 4), packed four
+// codes to a word (element e in byte e % 4 of word e / 4).  The fast values
+// of all N are formed first; the exact path runs only for the elements that
+// need it, behind one branch for the N.
+template <int N>
+__device__ __forceinline__ void quantize_codes(const float (&f)[N], float beta, float c, uint32_t (&w)[N / 4]) {
+    float r[N];
+    uint32_t bad = 0;
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+        const float q = __fmul_rn(f[e], c);
+        r[e] = rintf(q);
+        bad |= (fabsf(__fsub_rn(q, r[e])) < 0.4999f ? 0u : 1u) << e;
+    }
+    if (bad) {
+#pragma unroll
+        for (int e = 0; e < N; ++e)
+            if ((bad >> e) & 1u) {
+                const float t = rintf(__fdiv_rn(__fmul_rn(f[e], 127.0f), beta));
+                r[e] = fminf(fmaxf(t, -127.0f), 127.0f);
+            }
+    }
+#pragma unroll
+    for (int g = 0; g < N / 4; ++g) {
+        const uint32_t b0 = (uint32_t)__float2int_rn(r[4 * g + 0]) & 0xFFu;
+        const uint32_t b1 = (uint32_t)__float2int_rn(r[4 * g + 1]) & 0xFFu;
+        const uint32_t b2 = (uint32_t)__float2int_rn(r[4 * g + 2]) & 0xFFu;
+        const uint32_t b3 = (uint32_t)__float2int_rn(r[4 * g + 3]) & 0xFFu;
+        w[g] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+}
+
 // clip(rint(RN(RN(7·v) / β)), -7, 7): the 4-bit variant of quantize_one, with
 // c = quant_factor(β, 7) and the same argument (q within 7·5·2^-24 of RN(t)).
 __device__ __forceinline__ int quantize_one_a4(float v, float beta, float c) {

@@ -263,14 +263,9 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
                 float f[V];
                 FusedVec<T>::unpack(raw[i][j], f);
                 uint32_t wq[V / 4];
+                quantize_codes<V>(f, beta, qf, wq);
 #pragma unroll
-                for (int g = 0; g < V / 4; ++g) {
-                    uint32_t x = 0;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(f[4 * g + e], beta, qf) << (8 * e);
-                    wq[g] = x;
-                    qsum = dp4a_s8s8(0x01010101u, x, qsum);
-                }
+                for (int g = 0; g < V / 4; ++g) qsum = dp4a_s8s8(0x01010101u, wq[g], qsum);
                 const int k = v * V;
 #pragma unroll
                 for (int g = 0; g < V / 4; ++g) sts32(q[i].dst + xs_offset(k + 4 * g), wq[g]);
@@ -344,51 +339,72 @@ struct alignas(128) GShared {
 // comes from global memory.
 __device__ const uint4 g_zero_chunk[4] = {};
 
-// The warp's position in its step range: problem p, row group rg, step s
-// (chunks 32s .. 32s+31), global step index u, and the range end.
-struct Walk {
-    int p, rg, s;
-    int64_t u, end;
-};
+// Where a warp's next weight request comes from: problem p, row group rg,
+// step s, the steps left in the warp's range, the problem's fields, and this
+// lane's source address in row 0 of the row group for step s (chunk
+// 32s + lane) with the other rows' offsets (rows past N repeat row N-1, whose
+// results are never written).  The fields and offsets are re-derived only
+// when the position enters a new row group; a step moves the address by 512.
+template <int RG, int CPL>
+struct Feed {
+    int p, rg, s, rem;
+    int32_t C, S, rgn, N, rb;
+    const uint8_t* W;
+    const uint8_t* src;    // row 0 of the row group, this lane's chunk of step s
+    uint32_t off[RG];      // row r at src + off[r]
 
-__device__ __forceinline__ void walk_seek(const GProblem* T, int count, Walk& w, int64_t u, int64_t end) {
-    w.p = problem_of_step(T, count, u);
-    const int32_t local = (int32_t)(u - T[w.p].step_begin);
-    w.rg = local / T[w.p].S;
-    w.s = local - w.rg * T[w.p].S;
-    w.u = u;
-    w.end = end;
-}
-
-// Chunks of the step at the position (pr = its problem): 32, or the rest of
-// the row in its last step.
-__device__ __forceinline__ int walk_len(const GProblem& pr, const Walk& w) { return min(32, pr.C - 32 * w.s); }
-
-__device__ __forceinline__ void walk_advance(const GProblem& pr, Walk& w) {
-    ++w.u;
-    if (++w.s == pr.S) {
-        w.s = 0;
-        if (++w.rg == pr.rgn) {
-            w.rg = 0;
-            ++w.p;
+    __device__ __forceinline__ void fields(const GProblem* T) {
+        const GProblem& q = T[p];
+        C = q.C;
+        S = q.S;
+        rgn = q.rgn;
+        N = q.N;
+        rb = q.row_bytes;
+        W = q.W;
+    }
+    __device__ __forceinline__ void rows(int lane) {
+        const int row0 = rg * RG;
+        const int rlast = min(RG, N - row0) - 1;
+        src = W + (int64_t)row0 * rb + 16 * (32 * CPL * s + lane);
+#pragma unroll
+        for (int r = 0; r < RG; ++r) off[r] = (uint32_t)(min(r, rlast) * rb);
+    }
+    // Requests step s into this lane's column of a stage: chunk 32·CPL·s +
+    // 32j + lane of row r at dst + 512·(j·RG + r).  In a row's last step
+    // chunks past the end are replaced by the last chunk: their words meet
+    // zero activations.
+    __device__ __forceinline__ void request(uint32_t dst, int lane) const {
+        const int n = C - 32 * CPL * s;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            const uint8_t* b =
+                src + 512 * j - (n >= 32 * CPL ? 0u : 16u * (uint32_t)max(0, 32 * j + lane - (n - 1)));
+#pragma unroll
+            for (int r = 0; r < RG; ++r) cp_async16(dst + 512u * (j * RG + r), b + off[r]);
         }
     }
-}
+    __device__ __forceinline__ void advance(const GProblem* T, int lane) {
+        --rem;
+        if (++s < S) {
+            src += 512 * CPL;
+            return;
+        }
+        s = 0;
+        if (++rg == rgn) {
+            rg = 0;
+            ++p;
+            if (rem > 0) fields(T);
+        }
+        if (rem > 0) rows(lane);
+    }
+};
 
-// Requests the RG rows' 16 bytes of one step (n chunks) into this lane's
-// column of a stage (row r at dst + 512·r): lane l copies chunk
-// 32s + min(l, n - 1), so every address is valid and needs no predicate; rows
-// past N copy row N-1.  Lanes l >= n pair their words with zero activations,
-// and rows past N are never written, so neither changes a result.
-template <int RG>
-__device__ __forceinline__ void stage_step(const GProblem& pr, const Walk& s, int n, int lane, uint32_t dst) {
-    const int ch = 32 * s.s + min(lane, n - 1);
-    const int row0 = s.rg * RG;
-    const int rlast = min(RG, pr.N - row0) - 1;
-    const int32_t rb = pr.row_bytes;
-    const uint8_t* base = pr.W + (int64_t)row0 * rb + 16 * ch;
-#pragma unroll
-    for (int r = 0; r < RG; ++r) cp_async16(dst + 512u * r, base + (uint32_t)(min(r, rlast) * rb));
+// Problem, row group and step of global step u.
+__device__ __forceinline__ void locate_step(const GProblem* T, int count, int64_t u, int& p, int& rg, int& s) {
+    p = problem_of_step(T, count, u);
+    const int32_t local = (int32_t)(u - T[p].step_begin);
+    rg = local / T[p].S;
+    s = local - rg * T[p].S;
 }
 
 // MT tokens' activations of chunk ch from the shared slot rows (token m at
@@ -535,11 +551,11 @@ __device__ __forceinline__ void step_math(const uint4 (&w)[RG], const uint32_t (
 // not accumulated per step: the warp that holds a row group's first chunk
 // subtracts the token's whole-row Σx̃ once, so every row's total is
 // Σ c·x̃ - Σ x̃ over the full row.
-template <int MT, int W, int MINB, int RG, int D, bool FUSE>
+template <int MT, int W, int MINB, int RG, int CPL, int D, bool FUSE>
 __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_constant__ GParams P) {
     constexpr int NQ = MT <= 2 ? 4 : 1;  // one accumulator per code field (no shifts) for few tokens
     constexpr int V = RG * MT;           // sums per lane when a row group is done
-    constexpr uint32_t kStage = RG * 512;
+    constexpr uint32_t kStage = CPL * RG * 512;
     static_assert(RG <= kRGMax && V <= 32, "row group too large");
     static_assert(D >= 2, "at least one step in flight");
     using Shared = GShared<W>;
@@ -567,33 +583,36 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
 
     // ---- the first D-1 steps' weights do not depend on the previous kernel
     const uint32_t ring = smem_addr(smem_raw + sizeof(Shared)) + (uint32_t)warp * (D * kStage) + 16u * lane;
-    Walk cur, nxt;
-    walk_seek(T, count, cur, wu0, wu1);
-    nxt = cur;
-    int nq[D - 1];  // chunk counts of the steps in flight; nq[0] is the current step's
+    int p0 = 0, rg0 = 0, s0 = 0;
+    if (wu1 > wu0) locate_step(T, count, wu0, p0, rg0, s0);
+    Feed<RG, CPL> fd;
+    fd.p = p0;
+    fd.rg = rg0;
+    fd.s = s0;
+    fd.rem = (int)(wu1 - wu0);
+    if (fd.rem > 0) {
+        fd.fields(T);
+        fd.rows(lane);
+    }
 #pragma unroll
     for (int d = 0; d < D - 1; ++d) {
-        nq[d] = 0;
-        if (nxt.u < nxt.end) {
-            const GProblem& pq = T[nxt.p];
-            nq[d] = walk_len(pq, nxt);
-            stage_step<RG>(pq, nxt, nq[d], lane, ring + d * kStage);
-            walk_advance(pq, nxt);
+        if (fd.rem > 0) {
+            fd.request(ring + d * kStage, lane);
+            fd.advance(T, lane);
         }
         cp_async_commit();
     }
-    griddep_wait();  // x̃, β (and α) may come from the preceding kernels
-
-    // ---- fused quantisation: x̃ of the (at most two) problems of this CTA
+    // ---- fused quantisation: x̃ of the (at most two) problems of this CTA;
+    // the rows are set up before the dependency wait (they need only the table)
     int p_first = 0;
     int second_slot = 1;  // slot of the CTA's second problem (0 when it shares the first one's input)
     uint32_t xs_base = 0;
+    // rows[slot·MT + m]: token m of the slot's problem (static indices keep them in registers)
+    QRow rows[FUSE ? kMaxSlots * MT : 1];
     if constexpr (FUSE) {
         xs_base = smem_addr(smem_raw + sizeof(Shared) + W * D * kStage);
         p_first = problem_of_step(T, count, ca);
         const int p_last = cb > ca ? problem_of_step(T, count, cb - 1) : p_first;
-        // rows[slot·MT + m]: token m of the slot's problem (static indices keep them in registers)
-        QRow rows[kMaxSlots * MT];
 #pragma unroll
         for (int slot = 0; slot < kMaxSlots; ++slot) {
             const int p = p_first + slot;
@@ -633,6 +652,9 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                 }
             }
         }
+    }
+    griddep_wait();  // x̃, β (and α) may come from the preceding kernels
+    if constexpr (FUSE) {
 #pragma unroll
         for (int i = 0; i < kMaxSlots * MT; i += kFuseRows) {
             const QRow(&pair)[kFuseRows] = *reinterpret_cast<const QRow(*)[kFuseRows]>(&rows[i]);
@@ -654,6 +676,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
     uint32_t xrow = 0;                    // fused: shared address of the problem's slot
     const int8_t* xq = nullptr;           // unfused: the problem's x̃ and its shape
     int xM = 1, xK = 0, xfull = 0;
+    int cC = 0, cS = 1, crgn = 1;  // the problem's chunks per row, steps per row group, row groups
     int scale_p = -1;       // problem of my_scale
     float my_scale = 0.0f;  // lane m < MT: dequant scale of token m
 #pragma unroll
@@ -665,12 +688,17 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
     int own_p = -1, own_rg = 0;  // a shared row group this warp finishes after the loop
     uint32_t stage = ring;       // the current step's stage
     uint32_t fill = ring + (D - 1) * kStage;  // the stage the next request goes to
+    int cp = p0, crg = rg0, cs = s0;          // the current step
+    int crem = (int)(wu1 - wu0);              // steps left, the current one included
 
-    while (nq[0] > 0) {
-        if (cur.p != sp) {  // entering a problem: its α, β, Σx̃ and activations
-            sp = cur.p;
+    while (crem > 0) {
+        if (cp != sp) {  // entering a problem: its α, β, Σx̃, activations and shape
+            sp = cp;
             const GProblem& pr = T[sp];
             alpha_v = *pr.alpha;
+            cC = pr.C;
+            cS = pr.S;
+            crgn = pr.rgn;
             if constexpr (FUSE) {
                 const int slot = sp == p_first ? 0 : second_slot;
                 xrow = xs_base + (uint32_t)(slot * MT) * (uint32_t)P.slot_row;
@@ -693,36 +721,34 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                 for (int m = 0; m < MT; ++m)
 #pragma unroll
                     for (int q = 0; q < NQ; ++q) acc[r][m][q] = 0;
-            rg_own = cur.s == 0;
+            rg_own = cs == 0;
             fresh = false;
         }
-        const int nc = nq[0];
         // request the step D-1 ahead into the stage freed by the previous step
-        int nn = 0;
-        if (nxt.u < nxt.end) {
-            const GProblem& pq = T[nxt.p];
-            nn = walk_len(pq, nxt);
-            stage_step<RG>(pq, nxt, nn, lane, fill);
-            walk_advance(pq, nxt);
+        if (fd.rem > 0) {
+            fd.request(fill, lane);
+            fd.advance(T, lane);
         }
         cp_async_commit();
         cp_async_wait<D - 1>();  // this lane's copies of the current step have landed
-        uint4 w[RG];
+        const int nc = min(32 * CPL, cC - 32 * CPL * cs);  // chunks of this step
 #pragma unroll
-        for (int r = 0; r < RG; ++r) w[r] = lds128_after(stage + 512u * r);
+        for (int j = 0; j < CPL; ++j) {
+            uint4 w[RG];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) w[r] = lds128_after(stage + 512u * (j * RG + r));
+            const bool active = 32 * j + lane < nc;
+            const int ch = 32 * CPL * cs + 32 * j + lane;
+            uint32_t xa[MT][16];
+            if constexpr (FUSE)
+                lds_x<MT>(xrow, P.slot_row, ch, active, zero_addr, xa);
+            else
+                ldg_x<MT>(xq, xM, xK, xfull, ch, active, xa);
+            step_math<RG, MT, NQ>(w, xa, acc);
+        }
 
-        const bool active = lane < nc;
-        const int ch = 32 * cur.s + lane;
-        uint32_t xa[MT][16];
-        if constexpr (FUSE)
-            lds_x<MT>(xrow, P.slot_row, ch, active, zero_addr, xa);
-        else
-            ldg_x<MT>(xq, xM, xK, xfull, ch, active, xa);
-        step_math<RG, MT, NQ>(w, xa, acc);
-
-        const GProblem& pr = T[sp];
-        const bool rg_end = cur.s + 1 == pr.S;
-        if (rg_end || cur.u + 1 == cur.end) {
+        const bool rg_end = cs + 1 == cS;
+        if (rg_end || crem == 1) {
             // this warp's sums of the row group; the holder of its first
             // chunk takes Σx̃ off (in one lane, so once)
             const bool sub = lane == 0 && rg_own;
@@ -745,7 +771,8 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                     my_scale = dequant_scale(alpha_v, beta_v);
                 }
                 const float sc = __shfl_sync(0xffffffffu, my_scale, m);
-                const int row = cur.rg * RG + r;
+                const GProblem& pr = T[sp];
+                const int row = crg * RG + r;
                 if (writer && row < pr.N && m < pr.M) {
                     float out = __fmul_rn((float)val, sc);
                     if (pr.bias) out = __fadd_rn(out, pr.bias[row]);
@@ -759,15 +786,20 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                 if (writer) S.part[warp][rg_own ? 1 : 0][idx] = val;
                 if (rg_own) {
                     own_p = sp;
-                    own_rg = cur.rg;
+                    own_rg = crg;
                 }
             }
             fresh = true;
         }
-        walk_advance(pr, cur);
-#pragma unroll
-        for (int d = 0; d + 1 < D - 1; ++d) nq[d] = nq[d + 1];
-        nq[D - 2] = nn;
+        // the next step
+        --crem;
+        if (++cs == cS) {
+            cs = 0;
+            if (++crg == crgn) {
+                crg = 0;
+                ++cp;
+            }
+        }
         fill = stage;
         stage = stage + kStage == ring + D * kStage ? ring : stage + kStage;
     }
@@ -873,20 +905,20 @@ template <int MT>
 struct StreamCfg;
 template <>
 struct StreamCfg<1> {
-    static constexpr int W = 16, MINB = 1, RG = 8, D = 2;
+    static constexpr int W = 12, MINB = 1, RG = 8, CPL = 2, D = 2;
 };
 template <>
 struct StreamCfg<2> {
-    static constexpr int W = 12, MINB = 1, RG = 4, D = 4;
+    static constexpr int W = 12, MINB = 1, RG = 4, CPL = 1, D = 4;
 };
 template <>
 struct StreamCfg<4> {
-    static constexpr int W = 8, MINB = 1, RG = 4, D = 4;
+    static constexpr int W = 8, MINB = 1, RG = 4, CPL = 1, D = 4;
 };
 
 constexpr size_t kSmemOptIn = 232448;  // opt-in dynamic shared memory per block on sm_100
 
-void fill_params(GParams& P, const bitlinear_forward_problem* problems, int count, int RG) {
+void fill_params(GParams& P, const bitlinear_forward_problem* problems, int count, int RG, int CPL) {
     P = GParams{};
     P.count = count;
     int64_t total = 0;
@@ -907,7 +939,7 @@ void fill_params(GParams& P, const bitlinear_forward_problem* problems, int coun
         q.C = q.row_bytes / 16;
         q.full_chunks = q.K / 64;
         q.rgn = (q.N + RG - 1) / RG;
-        q.S = (q.C + 31) / 32;
+        q.S = (q.C + 32 * CPL - 1) / (32 * CPL);
         q.step_begin = total;
         total += (int64_t)q.rgn * q.S;
     }
@@ -915,9 +947,10 @@ void fill_params(GParams& P, const bitlinear_forward_problem* problems, int coun
 }
 
 // Prologue cost of quantising one input row of K elements in a CTA of W
-// warps, in warp-steps (the time one warp takes for one step): measured on
-// B200 with 12 warps as about 1.27 + K / 4930 step times.
-inline double prologue_cost(int W, int64_t K) { return W * (1.27 + (double)K / 4930.0); }
+// warps, in warp-steps (the time one warp takes for one step of CPL chunks
+// per lane): measured on B200 with 12 warps and one chunk per lane as about
+// 1.27 + K / 4930 step times.
+inline double prologue_cost(int W, int CPL, int64_t K) { return W * (1.27 + (double)K / 4930.0) / CPL; }
 
 // Splits the steps of P into at most G contiguous CTA ranges of whole row
 // groups whose costs (their steps, plus, with `pro`, the prologue cost of
@@ -976,24 +1009,24 @@ int cta_ranges(GParams& P, int G, const double* pro) {
     return fill(hi, true);
 }
 
-// Launches gemv_stream_kernel<MT, W, MINB, RG, D, fused>; with `fused` (one entry per
+// Launches gemv_stream_kernel<MT, W, MINB, RG, CPL, D, fused>; with `fused` (one entry per
 // problem) the kernel quantises x itself, if every CTA's range meets at most
 // two problems, the slots fit shared memory and the CTAs' input reads stay
 // small next to the weights (else *launched = false and nothing runs).
-template <int MT, int W, int MINB, int RG, int D>
+template <int MT, int W, int MINB, int RG, int CPL, int D>
 cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
                               cudaStream_t stream, bool pdl, const FusedInput* fused, bool x_bf16, bool* launched,
                               bool fuse_always) {
     using Shared = GShared<W>;
     if (launched) *launched = true;
     GParams P;
-    fill_params(P, problems, count, RG);
+    fill_params(P, problems, count, RG, CPL);
     int64_t weight_bytes = 0;
     for (int i = 0; i < count; ++i) weight_bytes += (int64_t)P.p[i].N * P.p[i].row_bytes;
     if (P.total_steps >= INT32_MAX) return cudaErrorInvalidValue;  // over 8 TB of weights in one call
     const int G = (int)std::min<int64_t>((int64_t)dev.sm_count * MINB, kMaxCta);
     int grid = 0;
-    size_t smem = sizeof(Shared) + (size_t)W * D * RG * 512;  // the table, then the warps' stage rings
+    size_t smem = sizeof(Shared) + (size_t)W * D * CPL * RG * 512;  // the table, then the warps' stage rings
     const size_t smem_cap = kSmemOptIn / MINB - (MINB > 1 ? 1024 : 0);
     if (fused) {
         int32_t slot_row = 0;
@@ -1012,7 +1045,7 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
         for (int i = 0; i < count; ++i)
             fits = fits && (int64_t)P.p[i].K * (x_bf16 ? 2 : 4) <= (int64_t)W * 32 * kFuseVec * 16;
         double pro[kMaxGroup];
-        for (int i = 0; i < count; ++i) pro[i] = prologue_cost(W, P.p[i].K) * std::min<int>(P.p[i].M, MT);
+        for (int i = 0; i < count; ++i) pro[i] = prologue_cost(W, CPL, P.p[i].K) * std::min<int>(P.p[i].M, MT);
         grid = cta_ranges(P, G, pro);
         // Every CTA reads its problems' whole input rows before its main loop;
         // that pays off only while those reads are small next to the weights.
@@ -1038,8 +1071,8 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
         grid = cta_ranges(P, G, nullptr);
     }
     if (smem > smem_cap) return cudaErrorInvalidConfiguration;  // a shape that does not fit (not built)
-    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, D, true>)
-                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, D, false>);
+    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, true>)
+                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, false>);
     // the opt-in is per device: set once on each device that launches the kernel
     cudaError_t err = set_max_dynamic_smem(kernel, (int)smem_cap);
     if (err != cudaSuccess) return err;
@@ -1062,7 +1095,7 @@ cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, 
                           cudaStream_t stream, bool pdl, const FusedInput* fused = nullptr, bool x_bf16 = false,
                           bool* launched = nullptr, bool fuse_always = false) {
     using C = StreamCfg<MT>;
-    return launch_stream_cfg<MT, C::W, C::MINB, C::RG, C::D>(problems, count, dev, stream, pdl, fused, x_bf16,
+    return launch_stream_cfg<MT, C::W, C::MINB, C::RG, C::CPL, C::D>(problems, count, dev, stream, pdl, fused, x_bf16,
                                                               launched, fuse_always);
 }
 

@@ -82,15 +82,9 @@ __device__ __forceinline__ float load_sum1(const T* x, const float* b, int64_t i
 }
 
 template <int V>
-__device__ __forceinline__ void store_codes(int8_t* q, const float* f, float beta, float qf) {
+__device__ __forceinline__ void store_codes(int8_t* q, const float (&f)[V], float beta, float qf) {
     uint32_t packed[V / 4];
-#pragma unroll
-    for (int j = 0; j < V / 4; ++j) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)quantize_one(f[4 * j + b], beta, qf) << (8 * b);
-        packed[j] = w;
-    }
+    quantize_codes<V>(f, beta, qf, packed);
     if constexpr (V == 4) {
         *reinterpret_cast<uint32_t*>(q) = packed[0];
     } else {
