@@ -93,34 +93,38 @@ __device__ __forceinline__ int8_t quantize_one(float v, float beta, float c) {
 }
 
 // quantize_one of N consecutive elements (N a multiple of 4), packed four
-// codes to a word (element e in byte e % 4 of word e / 4).  The fast values
-// of all N are formed first; the exact path runs only for the elements that
-// need it, behind one branch for the N.
+// codes to a word (element e in byte e % 4 of word e / 4).  The rounding uses
+// t = RN(q + 1.5·2^23): for |q| < 2^22 the sum lies where binary32 steps are
+// 1, so t - 1.5·2^23 is rint(q) (ties to even, as RN breaks them) and the low
+// byte of t's bits is that integer in two's complement; this avoids the
+// float-to-integer conversions.  The fast values of all N are formed first;
+// the exact path runs only for the elements that need it, behind one branch.
 template <int N>
 __device__ __forceinline__ void quantize_codes(const float (&f)[N], float beta, float c, uint32_t (&w)[N / 4]) {
-    float r[N];
+    constexpr float kRound = 12582912.0f;  // 1.5·2^23
+    float t[N];
     uint32_t bad = 0;
 #pragma unroll
     for (int e = 0; e < N; ++e) {
         const float q = __fmul_rn(f[e], c);
-        r[e] = rintf(q);
-        bad |= (fabsf(__fsub_rn(q, r[e])) < 0.4999f ? 0u : 1u) << e;
+        t[e] = __fadd_rn(q, kRound);
+        const float r = __fsub_rn(t[e], kRound);
+        bad |= (fabsf(__fsub_rn(q, r)) < 0.4999f ? 0u : 1u) << e;
     }
     if (bad) {
 #pragma unroll
         for (int e = 0; e < N; ++e)
             if ((bad >> e) & 1u) {
-                const float t = rintf(__fdiv_rn(__fmul_rn(f[e], 127.0f), beta));
-                r[e] = fminf(fmaxf(t, -127.0f), 127.0f);
+                float r = rintf(__fdiv_rn(__fmul_rn(f[e], 127.0f), beta));
+                r = fminf(fmaxf(r, -127.0f), 127.0f);  // also maps NaN to -127
+                t[e] = __fadd_rn(r, kRound);
             }
     }
 #pragma unroll
     for (int g = 0; g < N / 4; ++g) {
-        const uint32_t b0 = (uint32_t)__float2int_rn(r[4 * g + 0]) & 0xFFu;
-        const uint32_t b1 = (uint32_t)__float2int_rn(r[4 * g + 1]) & 0xFFu;
-        const uint32_t b2 = (uint32_t)__float2int_rn(r[4 * g + 2]) & 0xFFu;
-        const uint32_t b3 = (uint32_t)__float2int_rn(r[4 * g + 3]) & 0xFFu;
-        w[g] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        const uint32_t lo = __byte_perm(__float_as_uint(t[4 * g]), __float_as_uint(t[4 * g + 1]), 0x0040);
+        const uint32_t hi = __byte_perm(__float_as_uint(t[4 * g + 2]), __float_as_uint(t[4 * g + 3]), 0x0040);
+        w[g] = __byte_perm(lo, hi, 0x5410);
     }
 }
 

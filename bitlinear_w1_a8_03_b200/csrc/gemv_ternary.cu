@@ -206,31 +206,30 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
     constexpr int V = FusedVec<T>::n;
     uint4 raw[kFuseRows][kFuseVec];
     float mx[kFuseRows];
+    int nv[kFuseRows];  // 16-byte vectors per thread (the same in every thread; the last may be empty)
 #pragma unroll
     for (int i = 0; i < kFuseRows; ++i) {
         mx[i] = 0.0f;
-        if (q[i].valid) {
-            const int64_t base = (int64_t)q[i].m * q[i].K;
-            const int nvec = q[i].K / V;
+        const int nvec = q[i].valid ? q[i].K / V : 0;
+        nv[i] = (nvec + NT - 1) / NT;
+        const int64_t base = (int64_t)q[i].m * q[i].K;
 #pragma unroll
-            for (int j = 0; j < kFuseVec; ++j) {
+        for (int j = 0; j < kFuseVec; ++j) {
+            if (j < nv[i]) {
                 const int v = threadIdx.x + j * NT;
-                if (v < nvec) raw[i][j] = FusedVec<T>::load(q[i], base + (int64_t)v * V);
+                raw[i][j] = v < nvec ? FusedVec<T>::load(q[i], base + (int64_t)v * V) : make_uint4(0u, 0u, 0u, 0u);
             }
         }
     }
 #pragma unroll
     for (int i = 0; i < kFuseRows; ++i) {
-        if (q[i].valid) {
-            const int nvec = q[i].K / V;
 #pragma unroll
-            for (int j = 0; j < kFuseVec; ++j) {
-                if ((int)threadIdx.x + j * NT < nvec) {
-                    float f[V];
-                    FusedVec<T>::unpack(raw[i][j], f);
+        for (int j = 0; j < kFuseVec; ++j) {
+            if (j < nv[i]) {  // zero vectors past K leave the max unchanged
+                float f[V];
+                FusedVec<T>::unpack(raw[i][j], f);
 #pragma unroll
-                    for (int e = 0; e < V; ++e) mx[i] = fmaxf(mx[i], fabsf(f[e]));  // exact, order-free
-                }
+                for (int e = 0; e < V; ++e) mx[i] = fmaxf(mx[i], fabsf(f[e]));  // exact, order-free
             }
         }
     }
@@ -258,18 +257,25 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
         int qsum = 0;  // this thread's part of Σx̃
 #pragma unroll
         for (int j = 0; j < kFuseVec; ++j) {
-            const int v = threadIdx.x + j * NT;
-            if (v < nvec) {
+            if (j < nv[i]) {
+                // vectors past K give zero codes, which is what the slot holds
+                // there, so they are stored too while inside it
+                const int v = threadIdx.x + j * NT;
                 float f[V];
                 FusedVec<T>::unpack(raw[i][j], f);
                 uint32_t wq[V / 4];
                 quantize_codes<V>(f, beta, qf, wq);
 #pragma unroll
-                for (int g = 0; g < V / 4; ++g) qsum = dp4a_s8s8(0x01010101u, wq[g], qsum);
+                for (int g = 0; g < V / 4; ++g) {
+                    if (v >= nvec) wq[g] = 0u;  // past K the codes are 0 whatever β is
+                    qsum = dp4a_s8s8(0x01010101u, wq[g], qsum);
+                }
                 const int k = v * V;
+                if (k < slot_row) {
 #pragma unroll
-                for (int g = 0; g < V / 4; ++g) sts32(q[i].dst + xs_offset(k + 4 * g), wq[g]);
-                if (q[i].out) {
+                    for (int g = 0; g < V / 4; ++g) sts32(q[i].dst + xs_offset(k + 4 * g), wq[g]);
+                }
+                if (q[i].out && v < nvec) {
                     int8_t* o = q[i].xq + base + k;
                     if constexpr (V == 8)
                         *reinterpret_cast<uint2*>(o) = make_uint2(wq[0], wq[1]);
@@ -293,7 +299,7 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
             xbeta[q[i].slot][q[i].m] = beta;
             if (q[i].out) q[i].beta[q[i].m] = beta;
         }
-        for (int k = q[i].K + 4 * threadIdx.x; k < slot_row; k += 4 * NT) sts32(q[i].dst + xs_offset(k), 0u);
+        for (int k = nv[i] * NT * V + 4 * threadIdx.x; k < slot_row; k += 4 * NT) sts32(q[i].dst + xs_offset(k), 0u);
     }
 }
 
@@ -542,11 +548,11 @@ __device__ __forceinline__ void step_math(const uint4 (&w)[RG], const uint32_t (
 }
 
 // MT tokens (M <= MT), W warps per CTA, MINB CTAs per SM, row groups of RG
-// rows, D stages.  A warp walks its range one step at a time (up to 32
-// chunks of one row group, one chunk per lane).  Each warp has a ring of D
-// shared-memory stages (RG rows × 512 bytes): lane l copies its own 16 bytes
-// of every row with cp.async and later reads back only those, so the wait is
-// per thread and needs no warp barrier.  D-1 steps are in flight while one is
+// rows, CPL chunks per lane, D stages.  A warp walks its range one step at a
+// time (up to 32·CPL chunks of one row group).  Each warp has a ring of D
+// shared-memory stages (CPL·RG·512 bytes): lane l copies its own 16-byte
+// pieces with cp.async and later reads back only those, so the wait is per
+// thread and needs no warp barrier.  D-1 steps are in flight while one is
 // computed; the first D-1 are requested before the dependency wait.  Σx̃ is
 // not accumulated per step: the warp that holds a row group's first chunk
 // subtracts the token's whole-row Σx̃ once, so every row's total is

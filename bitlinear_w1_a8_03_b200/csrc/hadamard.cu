@@ -183,13 +183,7 @@ __global__ void __launch_bounds__(kMaxThreads) hadamard_kernel(const __grid_cons
                 rotate_tile(v, P.block, s_tile);
             }
             uint32_t w[kE / 4];
-#pragma unroll
-            for (int g = 0; g < kE / 4; ++g) {
-                uint32_t x = 0;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) x |= (uint32_t)(uint8_t)quantize_one(v[4 * g + e], beta, qf) << (8 * e);
-                w[g] = x;
-            }
+            quantize_codes<kE>(v, beta, qf, w);
             if (vec && k0 + kE <= P.K && (reinterpret_cast<uintptr_t>(P.x_q) & 15) == 0) {
                 *reinterpret_cast<uint4*>(q + k0) = make_uint4(w[0], w[1], w[2], w[3]);
             } else {
