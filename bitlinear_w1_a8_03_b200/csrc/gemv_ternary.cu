@@ -482,43 +482,6 @@ __device__ __forceinline__ void ldg_x(const int8_t* xq, int M, int K, int full_c
     }
 }
 
-// Σx̃ of each of the MT tokens of a global x̃ row (every lane gets the
-// totals; tokens past M give 0): one pass over the row by the warp.
-template <int MT>
-__device__ __forceinline__ void warp_xsum(const int8_t* xq, int M, int K, int C, int full_chunks, int lane,
-                                          int (&sx)[MT]) {
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        int t = 0;
-        if (m < M) {
-            const int8_t* row = xq + (int64_t)m * K;
-            for (int ch = lane; ch < C; ch += 32) {
-                uint32_t a[16];
-                if (ch < full_chunks) {
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const uint4 u = ld_shared_ro16(row + 64 * ch + 16 * v);
-                        a[4 * v + 0] = u.x;
-                        a[4 * v + 1] = u.y;
-                        a[4 * v + 2] = u.z;
-                        a[4 * v + 3] = u.w;
-                    }
-                } else {
-                    uint32_t tmp[16];  // the rare tail goes through local memory
-                    load_act_tail(row, K, ch, tmp);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) a[q] = tmp[q];
-                }
-#pragma unroll
-                for (int q = 0; q < 16; ++q) t = dp4a_s8s8(0x01010101u, a[q], t);
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-        sx[m] = t;
-    }
-}
-
 // acc[r][m][q] += codes × x̃ for one step: per (word, field) the RG rows'
 // codes are masked first, then their dp4a go to RG independent accumulators.
 // With NQ = 4 field q keeps its codes in place (×4^q, summed with a shift at
@@ -553,10 +516,12 @@ __device__ __forceinline__ void step_math(const uint4 (&w)[RG], const uint32_t (
 // shared-memory stages (CPL·RG·512 bytes): lane l copies its own 16-byte
 // pieces with cp.async and later reads back only those, so the wait is per
 // thread and needs no warp barrier.  D-1 steps are in flight while one is
-// computed; the first D-1 are requested before the dependency wait.  Σx̃ is
-// not accumulated per step: the warp that holds a row group's first chunk
-// subtracts the token's whole-row Σx̃ once, so every row's total is
-// Σ c·x̃ - Σ x̃ over the full row.
+// computed; the first D-1 are requested before the dependency wait.  With
+// the fused prologue Σx̃ is not accumulated per step: the warp that holds a
+// row group's first chunk subtracts the token's whole-row Σx̃ (summed while
+// quantising) once, so every row's total is Σ c·x̃ - Σ x̃ over the full row.
+// With x̃ from global memory each lane adds up the Σx̃ of the chunks it
+// multiplies and subtracts it from its own partial sums.
 template <int MT, int W, int MINB, int RG, int CPL, int D, bool FUSE>
 __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_constant__ GParams P) {
     constexpr int NQ = MT <= 2 ? 4 : 1;  // one accumulator per code field (no shifts) for few tokens
@@ -575,7 +540,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
     // grid before touching memory this grid writes
     griddep_launch_dependents();
 
-    // ---- CTA and warp ranges (equal chunk counts, CTA edges on row groups)
+    // ---- CTA range (from the host, on row-group edges) and equal warp step ranges
     for (int i = threadIdx.x; i < P.count; i += W * 32) S.prob[i] = P.p[i];
     if (threadIdx.x < 16) reinterpret_cast<uint32_t*>(S.zero)[threadIdx.x] = 0u;
     if (threadIdx.x < kMaxSlots * kGemvMaxTokens) (&S.xsum[0][0])[threadIdx.x] = 0;
@@ -678,7 +643,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
     // ---- state of the problem of the current step
     int sp = -1;                          // that problem
     float alpha_v = 0.0f, beta_v = 0.0f;  // lane m < MT: α and token m's β
-    int sx[MT];                           // Σx̃ of each token over the whole row
+    int sx[MT];  // fused: Σx̃ of each token over the whole row; else this lane's part of the row group's
     uint32_t xrow = 0;                    // fused: shared address of the problem's slot
     const int8_t* xq = nullptr;           // unfused: the problem's x̃ and its shape
     int xM = 1, xK = 0, xfull = 0;
@@ -717,7 +682,6 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                 xK = pr.K;
                 xfull = pr.full_chunks;
                 if (lane < MT && lane < pr.M) beta_v = pr.beta[lane];
-                warp_xsum<MT>(pr.xq, pr.M, pr.K, pr.C, pr.full_chunks, lane, sx);
             }
         }
         if (fresh) {
@@ -729,6 +693,10 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                     for (int q = 0; q < NQ; ++q) acc[r][m][q] = 0;
             rg_own = cs == 0;
             fresh = false;
+            if constexpr (!FUSE) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) sx[m] = 0;
+            }
         }
         // request the step D-1 ahead into the stage freed by the previous step
         if (fd.rem > 0) {
@@ -751,13 +719,20 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
             else
                 ldg_x<MT>(xq, xM, xK, xfull, ch, active, xa);
             step_math<RG, MT, NQ>(w, xa, acc);
+            if constexpr (!FUSE) {  // this lane's Σx̃ over the chunks it added
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) sx[m] = dp4a_s8s8(0x01010101u, xa[m][q], sx[m]);
+            }
         }
 
         const bool rg_end = cs + 1 == cS;
         if (rg_end || crem == 1) {
-            // this warp's sums of the row group; the holder of its first
-            // chunk takes Σx̃ off (in one lane, so once)
-            const bool sub = lane == 0 && rg_own;
+            // this warp's sums of the row group.  Fused: the holder of its
+            // first chunk takes the row's Σx̃ off (in one lane, so once);
+            // otherwise every lane takes off the Σx̃ of the chunks it added.
+            const bool sub = FUSE ? (lane == 0 && rg_own) : true;
             int v[V];
 #pragma unroll
             for (int r = 0; r < RG; ++r)
@@ -1067,7 +1042,7 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
             prologue_bytes += input_bytes(P.p[pa]);
             if (pb != pa && !(P.p[pb].x == P.p[pa].x && P.p[pb].x2 == P.p[pa].x2)) prologue_bytes += input_bytes(P.p[pb]);
         }
-        if (!fuse_always && 8 * prologue_bytes > weight_bytes) fits = false;
+        if (!fuse_always && 2 * prologue_bytes > weight_bytes) fits = false;
         if (!fits) {
             *launched = false;
             return cudaSuccess;
