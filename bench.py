@@ -199,13 +199,16 @@ def gpu_id(props, local_rank) -> str:
     return "GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local_rank)
 
 
-def settle(stream, replay, props, local_rank, seconds: float = 1.0) -> ClockSampler:
+SETTLE_SECONDS = 1.0  # --settle-seconds; 0 only for profiler runs, whose numbers are not bench values
+
+
+def settle(stream, replay, props, local_rank, seconds: float | None = None) -> ClockSampler:
     """Starts the clock sampler, then runs about `seconds` of identical replays
     so the timed region that follows runs at settled clocks; the caller stops
     the sampler after its timed region (and a few more replays)."""
     import torch
     sampler = ClockSampler(gpu_id(props, local_rank))
-    t_end = time.time() + seconds
+    t_end = time.time() + (SETTLE_SECONDS if seconds is None else seconds)
     with torch.cuda.stream(stream):
         while time.time() < t_end:
             replay()
@@ -1228,7 +1231,11 @@ def main():
                     help="comma list: decode (the headline line); tiny, batched_100b, prefill, stack, hadamard, "
                          "scales, a4 and train are added under their own keys")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
+    ap.add_argument("--settle-seconds", type=float, default=1.0,
+                    help="seconds of identical replays before each timed region (0: profiler runs only)")
     args = ap.parse_args()
+    global SETTLE_SECONDS
+    SETTLE_SECONDS = max(0.0, args.settle_seconds)
     legs = [x for x in args.legs.split(",") if x]
     if args.warmup < 3:
         args.warmup = 3

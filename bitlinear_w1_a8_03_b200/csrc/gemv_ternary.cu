@@ -706,8 +706,8 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
         cp_async_commit();
         cp_async_wait<D - 1>();  // this lane's copies of the current step have landed
         const int nc = min(32 * CPL, cC - 32 * CPL * cs);  // chunks of this step
-#pragma unroll
-        for (int j = 0; j < CPL; ++j) {
+#pragma unroll 1
+        for (int j = 0; j < CPL; ++j) {  // not unrolled: one copy of the arithmetic keeps the loop in the instruction cache
             uint4 w[RG];
 #pragma unroll
             for (int r = 0; r < RG; ++r) w[r] = lds128_after(stage + 512u * (j * RG + r));
