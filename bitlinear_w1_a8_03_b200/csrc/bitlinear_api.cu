@@ -409,6 +409,32 @@ bitlinear_status bitlinear_linear_scaled(const bitlinear_scaled_problem* problem
     if (st != BL_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    // One α per row and at most four tokens: the streaming GEMV with the row's
+    // α in its epilogue, quantising x in its prologue when it can.
+    bool rows_path = true;
+    for (int i = 0; i < count && rows_path; ++i) {
+        const bitlinear_scaled_problem& q = problems[i];
+        rows_path = q.group >= q.K && q.M <= 4 && q.K % 16 == 0 && !misaligned(q.x_q, 16);
+    }
+    if (rows_path) {
+        bitlinear_forward_problem f[BITLINEAR_MAX_GROUP];
+        for (int i = 0; i < count; ++i) {
+            const bitlinear_scaled_problem& q = problems[i];
+            f[i] = bitlinear_forward_problem{q.x_q, q.beta, q.W_packed, q.alpha, q.bias, q.y, q.acc_out, q.M, q.N, q.K};
+        }
+        if (nact == count) {
+            bl::FusedInput fin[BITLINEAR_MAX_GROUP];
+            for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
+            bool launched = false;
+            st = from_cuda(bl::launch_linear_fused(f, fin, count, dtype, s, weights_static, &launched, true));
+            if (st != BL_OK || launched) return st;
+        }
+        if (nact > 0) {
+            st = from_cuda(bl::launch_quantize_act(act, nact, dtype, s, true, weights_static));
+            if (st != BL_OK) return st;
+        }
+        return from_cuda(bl::launch_forward(f, count, s, nact > 0 || weights_static, true));
+    }
     if (nact > 0) {
         st = from_cuda(bl::launch_quantize_act(act, nact, dtype, s, true, weights_static));
         if (st != BL_OK) return st;

@@ -60,7 +60,11 @@ cudaError_t launch_quantize_weights_static(const void* W, bitlinear_dtype dtype,
 // pdl: launch with programmatic dependent launch; only valid right after the
 // library's own activation-quantisation kernel on the same stream (the weight
 // stream starts before the dependency wait).
-cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl);
+// alpha_rows: each problem's alpha is a per-row table [N] ("1.58 位大模型" §3.1:
+// one α per output row), applied as y = RN32(RN32(fp32(acc)·α_n)·RN32(RN64(β/127)));
+// only for at most four tokens (the streaming GEMV).
+cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl,
+                           bool alpha_rows = false);
 
 // Fused linear for at most four tokens: the streaming GEMV quantises its own
 // activations (x, or x + x2 in float32) into shared memory, so the pair of
@@ -75,7 +79,8 @@ struct FusedInput {
 // *launched = false (and nothing enqueued) when the problems do not fit the
 // fused kernel; the caller then runs the quantisation and product separately.
 cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
-                                bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched);
+                                bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched,
+                                bool alpha_rows = false);
 
 // Hadamard rotation (out = x·H·scale) or rotation + per-token int8
 // quantisation (x_q, beta), one job per problem of a grouped launch; all jobs

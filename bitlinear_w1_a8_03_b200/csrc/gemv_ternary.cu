@@ -67,6 +67,7 @@ struct GProblem {
     int32_t C;            // 16-byte chunks per row
     int32_t full_chunks;  // chunks entirely inside K (the activation tail needs guards)
     int32_t rgn;          // row groups
+    int32_t alpha_rows;   // alpha is a per-row table [N] (else one α for the matrix)
     int32_t S;            // steps per row group: ceil(C / 32) (a step gives each lane one chunk)
     int64_t step_begin;   // first step of this problem in the launch
     // fused quantisation (x̃ made in shared memory from x):
@@ -301,6 +302,13 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
         }
         for (int k = nv[i] * NT * V + 4 * threadIdx.x; k < slot_row; k += 4 * NT) sts32(q[i].dst + xs_offset(k), 0u);
     }
+}
+
+// A token's dequantisation factor: RN32(RN64(α·β/127)) for one α per matrix;
+// with one α per row the row's α is applied first, y = RN32(RN32(acc·α_n)·s)
+// with s = RN32(RN64(β/127)) ("1.58 位大模型", nxmr.cn/news/148658 §3.1, §4.2).
+__device__ __forceinline__ float token_scale(int alpha_rows, float alpha, float beta) {
+    return alpha_rows ? __double2float_rn(__ddiv_rn((double)beta, 127.0)) : dequant_scale(alpha, beta);
 }
 
 // ---------------------------------------------------------------- reductions
@@ -666,7 +674,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
         if (cp != sp) {  // entering a problem: its α, β, Σx̃, activations and shape
             sp = cp;
             const GProblem& pr = T[sp];
-            alpha_v = *pr.alpha;
+            alpha_v = pr.alpha_rows ? 0.0f : *pr.alpha;
             cC = pr.C;
             cS = pr.S;
             crgn = pr.rgn;
@@ -749,13 +757,14 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
             if (rg_own && rg_end) {  // the whole row group: write y
                 if (scale_p != sp) {
                     scale_p = sp;
-                    my_scale = dequant_scale(alpha_v, beta_v);
+                    my_scale = token_scale(T[sp].alpha_rows, alpha_v, beta_v);
                 }
                 const float sc = __shfl_sync(0xffffffffu, my_scale, m);
                 const GProblem& pr = T[sp];
                 const int row = crg * RG + r;
                 if (writer && row < pr.N && m < pr.M) {
-                    float out = __fmul_rn((float)val, sc);
+                    float out = pr.alpha_rows ? __fmul_rn(__fmul_rn((float)val, pr.alpha[row]), sc)
+                                              : __fmul_rn((float)val, sc);
                     if (pr.bias) out = __fadd_rn(out, pr.bias[row]);
                     pr.y[(int64_t)m * pr.N + row] = out;
                     if (pr.acc_out) pr.acc_out[(int64_t)m * pr.N + row] = val;
@@ -800,12 +809,13 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
         int val = writer ? S.part[warp][1][idx] : 0;
         for (int w2 = warp + 1; w2 < W && S.bound[w2] < rg_end; ++w2)
             if (writer && S.bound[w2 + 1] > S.bound[w2]) val += S.part[w2][0][idx];  // skip empty ranges
-        if (scale_p != own_p) my_scale = dequant_scale(alpha_v, beta_v);
+        if (scale_p != own_p) my_scale = token_scale(pr.alpha_rows, alpha_v, beta_v);
         const int r = idx % RG, m = idx / RG;
         const float sc = __shfl_sync(0xffffffffu, my_scale, m);
         const int row = own_rg * RG + r;
         if (writer && row < pr.N && m < pr.M) {
-            float out = __fmul_rn((float)val, sc);
+            float out = pr.alpha_rows ? __fmul_rn(__fmul_rn((float)val, pr.alpha[row]), sc)
+                                      : __fmul_rn((float)val, sc);
             if (pr.bias) out = __fadd_rn(out, pr.bias[row]);
             pr.y[(int64_t)m * pr.N + row] = out;
             if (pr.acc_out) pr.acc_out[(int64_t)m * pr.N + row] = val;
@@ -899,7 +909,8 @@ struct StreamCfg<4> {
 
 constexpr size_t kSmemOptIn = 232448;  // opt-in dynamic shared memory per block on sm_100
 
-void fill_params(GParams& P, const bitlinear_forward_problem* problems, int count, int RG, int CPL) {
+void fill_params(GParams& P, const bitlinear_forward_problem* problems, int count, int RG, int CPL,
+                 bool alpha_rows = false) {
     P = GParams{};
     P.count = count;
     int64_t total = 0;
@@ -920,6 +931,7 @@ void fill_params(GParams& P, const bitlinear_forward_problem* problems, int coun
         q.C = q.row_bytes / 16;
         q.full_chunks = q.K / 64;
         q.rgn = (q.N + RG - 1) / RG;
+        q.alpha_rows = alpha_rows ? 1 : 0;
         q.S = (q.C + 32 * CPL - 1) / (32 * CPL);
         q.step_begin = total;
         total += (int64_t)q.rgn * q.S;
@@ -997,11 +1009,11 @@ int cta_ranges(GParams& P, int G, const double* pro) {
 template <int MT, int W, int MINB, int RG, int CPL, int D>
 cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
                               cudaStream_t stream, bool pdl, const FusedInput* fused, bool x_bf16, bool* launched,
-                              bool fuse_always) {
+                              bool fuse_always, bool alpha_rows = false) {
     using Shared = GShared<W>;
     if (launched) *launched = true;
     GParams P;
-    fill_params(P, problems, count, RG, CPL);
+    fill_params(P, problems, count, RG, CPL, alpha_rows);
     int64_t weight_bytes = 0;
     for (int i = 0; i < count; ++i) weight_bytes += (int64_t)P.p[i].N * P.p[i].row_bytes;
     if (P.total_steps >= INT32_MAX) return cudaErrorInvalidValue;  // over 8 TB of weights in one call
@@ -1074,10 +1086,10 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
 template <int MT>
 cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
                           cudaStream_t stream, bool pdl, const FusedInput* fused = nullptr, bool x_bf16 = false,
-                          bool* launched = nullptr, bool fuse_always = false) {
+                          bool* launched = nullptr, bool fuse_always = false, bool alpha_rows = false) {
     using C = StreamCfg<MT>;
     return launch_stream_cfg<MT, C::W, C::MINB, C::RG, C::CPL, C::D>(problems, count, dev, stream, pdl, fused, x_bf16,
-                                                              launched, fuse_always);
+                                                                     launched, fuse_always, alpha_rows);
 }
 
 cudaError_t launch_generic(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
@@ -1112,7 +1124,8 @@ cudaError_t launch_generic(const bitlinear_forward_problem* problems, int count,
 
 }  // namespace
 
-cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl) {
+cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl,
+                           bool alpha_rows) {
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
@@ -1122,6 +1135,11 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
         const bitlinear_forward_problem& s = problems[i];
         fast = fast && (s.K % 16 == 0) && ((reinterpret_cast<uintptr_t>(s.x_q) & 15) == 0);
         if (s.M > max_m) max_m = s.M;
+    }
+    if (alpha_rows) {  // per-row α: the streaming GEMV only (the caller checked shape and alignment)
+        if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl, nullptr, false, nullptr, false, true);
+        if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl, nullptr, false, nullptr, false, true);
+        return launch_stream<4>(problems, count, dev, stream, pdl, nullptr, false, nullptr, false, true);
     }
     if (max_m > kGemvMaxTokens) {
         // many tokens: the int8 tensor cores, all problems in one launch
@@ -1137,7 +1155,8 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
 }
 
 cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
-                                bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched) {
+                                bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched,
+                                bool alpha_rows) {
     *launched = false;
     // BITLINEAR_LINEAR_FUSION=off never fuses, =on fuses whenever the
     // problems fit the kernel (skipping the byte-ratio rule); default: auto
@@ -1158,9 +1177,9 @@ cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const
         if (s.M > max_m) max_m = s.M;
     }
     const bool bf16 = dtype == BL_BF16;
-    if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl, in, bf16, launched, always);
-    if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl, in, bf16, launched, always);
-    if (max_m <= 4) return launch_stream<4>(problems, count, dev, stream, pdl, in, bf16, launched, always);
+    if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows);
+    if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows);
+    if (max_m <= 4) return launch_stream<4>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows);
     return cudaSuccess;
 }
 

@@ -368,9 +368,11 @@ typedef struct bitlinear_scaled_problem {
  * row S = α_n·acc is exact; with several, S is summed in binary64 (each term
  * exact), in an order that may differ from a sequential sum in the last bits
  * of binary64.  `problems` is a HOST array; flags: 0 or
- * BL_LINEAR_WEIGHTS_STATIC.  CUDA cores; for more than four tokens the
- * weights are streamed once per four tokens (this variant is not the
- * tensor-core path).
+ * BL_LINEAR_WEIGHTS_STATIC.  CUDA cores: with one α per row and at most four
+ * tokens (K a multiple of 16, x_q 16-byte aligned) the streaming GEMV of
+ * bitlinear_linear_grouped with the row's α in its epilogue (one launch when
+ * it can quantise x itself); otherwise a GEMV that streams the weights once
+ * per four tokens (this variant is not the tensor-core path).
  * Errors: as bitlinear_linear_grouped, plus BL_ERR_SHAPE for a bad group or
  * acc_out with several α per row. */
 BITLINEAR_API bitlinear_status bitlinear_linear_scaled(const bitlinear_scaled_problem* problems, int count,
