@@ -488,6 +488,19 @@ bitlinear_status bitlinear_linear_a4(const bitlinear_linear_problem* problems, i
     bitlinear_status st = check_device();
     if (st != BL_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
+    // at most four tokens: one launch of the streaming GEMV that quantises x
+    // to 4 bits in its prologue, when the problems fit it
+    bool fusable = true;
+    for (int i = 0; i < count && fusable; ++i)
+        fusable = problems[i].M <= 4 && problems[i].K % 16 == 0 && !misaligned(problems[i].x_q, 4);
+    if (fusable) {
+        bl::FusedInput fin[BITLINEAR_MAX_GROUP];
+        for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
+        bool launched = false;
+        st = from_cuda(bl::launch_linear_fused(fwd, fin, count, dtype, s, weights_static, &launched, false, true));
+        if (st != BL_OK || launched) return st;
+    }
     st = from_cuda(bl::launch_quantize_act_a4(act, count, dtype, s, true));
     if (st != BL_OK) return st;
     return from_cuda(bl::launch_forward_a4(fwd, count, s, true));

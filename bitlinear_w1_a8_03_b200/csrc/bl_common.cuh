@@ -93,14 +93,16 @@ __device__ __forceinline__ int8_t quantize_one(float v, float beta, float c) {
 }
 
 // quantize_one of N consecutive elements (N a multiple of 4), packed four
-// codes to a word (element e in byte e % 4 of word e / 4).  The rounding uses
+// codes to a word (element e in byte e % 4 of word e / 4); with qmax = 7 (and
+// c = quant_factor(β, 7)) the codes of quantize_one_a4, as int8 bytes.  The rounding uses
 // t = RN(q + 1.5·2^23): for |q| < 2^22 the sum lies where binary32 steps are
 // 1, so t - 1.5·2^23 is rint(q) (ties to even, as RN breaks them) and the low
 // byte of t's bits is that integer in two's complement; this avoids the
 // float-to-integer conversions.  The fast values of all N are formed first;
 // the exact path runs only for the elements that need it, behind one branch.
 template <int N>
-__device__ __forceinline__ void quantize_codes(const float (&f)[N], float beta, float c, uint32_t (&w)[N / 4]) {
+__device__ __forceinline__ void quantize_codes(const float (&f)[N], float beta, float c, uint32_t (&w)[N / 4],
+                                               float qmax = 127.0f) {
     constexpr float kRound = 12582912.0f;  // 1.5·2^23
     float t[N];
     uint32_t bad = 0;
@@ -115,8 +117,8 @@ __device__ __forceinline__ void quantize_codes(const float (&f)[N], float beta, 
 #pragma unroll
         for (int e = 0; e < N; ++e)
             if ((bad >> e) & 1u) {
-                float r = rintf(__fdiv_rn(__fmul_rn(f[e], 127.0f), beta));
-                r = fminf(fmaxf(r, -127.0f), 127.0f);  // also maps NaN to -127
+                float r = rintf(__fdiv_rn(__fmul_rn(f[e], qmax), beta));
+                r = fminf(fmaxf(r, -qmax), qmax);  // also maps NaN to -qmax
                 t[e] = __fadd_rn(r, kRound);
             }
     }

@@ -78,9 +78,11 @@ struct FusedInput {
 };
 // *launched = false (and nothing enqueued) when the problems do not fit the
 // fused kernel; the caller then runs the quantisation and product separately.
+// a4: 4-bit activations ("BitNet CPU 实测" §2.1 variant): codes clip(rint(7x/β), ±7),
+// x_q written as nibbles [M][K/2], y = fp32(acc)·RN32(RN64(α·β/7)).
 cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
                                 bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched,
-                                bool alpha_rows = false);
+                                bool alpha_rows = false, bool a4 = false);
 
 // Hadamard rotation (out = x·H·scale) or rotation + per-token int8
 // quantisation (x_q, beta), one job per problem of a grouped launch; all jobs

@@ -85,6 +85,7 @@ struct GParams {
     int64_t total_steps;
     int32_t cta_begin[kMaxCta + 1];  // first step of each CTA (row-group boundaries), then the end
     int x_bf16;        // fused: activation dtype
+    int a4;            // fused: 4-bit activations (codes in [-7, 7], x̃ written as nibbles, scale α·β/7)
     int32_t slot_row;  // fused: bytes per token row of a shared x̃ slot (64·ceil(K/64) of the widest problem)
 };
 
@@ -203,7 +204,8 @@ constexpr int kFuseRows = 2;  // input rows quantised together (one block reduct
 // K is a multiple of 16 and x, x2 are 16-byte aligned.
 template <typename T, int NT>
 __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row, float (*red)[32],
-                                    float (*xbeta)[kGemvMaxTokens], int (*xsum)[kGemvMaxTokens]) {
+                                    float (*xbeta)[kGemvMaxTokens], int (*xsum)[kGemvMaxTokens], bool a4) {
+    const float qmax = a4 ? 7.0f : 127.0f;
     constexpr int V = FusedVec<T>::n;
     uint4 raw[kFuseRows][kFuseVec];
     float mx[kFuseRows];
@@ -252,7 +254,7 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
 #pragma unroll
         for (int w = 1; w < NT / 32; ++w) b = fmaxf(b, red[i][w]);
         const float beta = __fadd_rn(b, 1e-8f);
-        const float qf = quant_factor(beta, 127.0f);
+        const float qf = quant_factor(beta, qmax);
         const int64_t base = (int64_t)q[i].m * q[i].K;
         const int nvec = q[i].K / V;
         int qsum = 0;  // this thread's part of Σx̃
@@ -265,7 +267,7 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
                 float f[V];
                 FusedVec<T>::unpack(raw[i][j], f);
                 uint32_t wq[V / 4];
-                quantize_codes<V>(f, beta, qf, wq);
+                quantize_codes<V>(f, beta, qf, wq, qmax);
 #pragma unroll
                 for (int g = 0; g < V / 4; ++g) {
                     if (v >= nvec) wq[g] = 0u;  // past K the codes are 0 whatever β is
@@ -276,7 +278,18 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
 #pragma unroll
                     for (int g = 0; g < V / 4; ++g) sts32(q[i].dst + xs_offset(k + 4 * g), wq[g]);
                 }
-                if (q[i].out && v < nvec) {
+                if (q[i].out && v < nvec && a4) {
+                    // two codes per byte, element 2j in the low nibble ("BitNet CPU 实测" §2.1 variant)
+                    uint8_t* o = reinterpret_cast<uint8_t*>(q[i].xq) + (int64_t)q[i].m * (q[i].K / 2) + k / 2;
+                    const uint32_t lo = wq[0] & 0x0F0F0F0Fu;
+                    const uint32_t t0 = lo | (lo >> 4);  // bytes 0 and 2: codes (0,1) and (2,3)
+                    if constexpr (V == 8) {
+                        const uint32_t hi = wq[1] & 0x0F0F0F0Fu;
+                        *reinterpret_cast<uint32_t*>(o) = __byte_perm(t0, hi | (hi >> 4), 0x6420);
+                    } else {
+                        *reinterpret_cast<uint16_t*>(o) = (uint16_t)__byte_perm(t0, 0u, 0x0020);
+                    }
+                } else if (q[i].out && v < nvec) {
                     int8_t* o = q[i].xq + base + k;
                     if constexpr (V == 8)
                         *reinterpret_cast<uint2*>(o) = make_uint2(wq[0], wq[1]);
@@ -307,7 +320,9 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
 // A token's dequantisation factor: RN32(RN64(α·β/127)) for one α per matrix;
 // with one α per row the row's α is applied first, y = RN32(RN32(acc·α_n)·s)
 // with s = RN32(RN64(β/127)) ("1.58 位大模型", nxmr.cn/news/148658 §3.1, §4.2).
-__device__ __forceinline__ float token_scale(int alpha_rows, float alpha, float beta) {
+// With 4-bit activations the factor is RN32(RN64(α·β/7)).
+__device__ __forceinline__ float token_scale(int alpha_rows, int a4, float alpha, float beta) {
+    if (a4) return dequant_scale_a4(alpha, beta);
     return alpha_rows ? __double2float_rn(__ddiv_rn((double)beta, 127.0)) : dequant_scale(alpha, beta);
 }
 
@@ -639,9 +654,9 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
             const QRow(&pair)[kFuseRows] = *reinterpret_cast<const QRow(*)[kFuseRows]>(&rows[i]);
             if (pair[0].valid || pair[1].valid) {  // the same in every thread of the CTA
                 if (P.x_bf16)
-                    fused_quantize_rows<uint16_t, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum);
+                    fused_quantize_rows<uint16_t, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum, P.a4 != 0);
                 else
-                    fused_quantize_rows<float, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum);
+                    fused_quantize_rows<float, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum, P.a4 != 0);
             }
         }
         __syncthreads();
@@ -757,7 +772,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
             if (rg_own && rg_end) {  // the whole row group: write y
                 if (scale_p != sp) {
                     scale_p = sp;
-                    my_scale = token_scale(T[sp].alpha_rows, alpha_v, beta_v);
+                    my_scale = token_scale(T[sp].alpha_rows, P.a4, alpha_v, beta_v);
                 }
                 const float sc = __shfl_sync(0xffffffffu, my_scale, m);
                 const GProblem& pr = T[sp];
@@ -809,7 +824,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
         int val = writer ? S.part[warp][1][idx] : 0;
         for (int w2 = warp + 1; w2 < W && S.bound[w2] < rg_end; ++w2)
             if (writer && S.bound[w2 + 1] > S.bound[w2]) val += S.part[w2][0][idx];  // skip empty ranges
-        if (scale_p != own_p) my_scale = token_scale(pr.alpha_rows, alpha_v, beta_v);
+        if (scale_p != own_p) my_scale = token_scale(pr.alpha_rows, P.a4, alpha_v, beta_v);
         const int r = idx % RG, m = idx / RG;
         const float sc = __shfl_sync(0xffffffffu, my_scale, m);
         const int row = own_rg * RG + r;
@@ -1009,9 +1024,10 @@ int cta_ranges(GParams& P, int G, const double* pro) {
 template <int MT, int W, int MINB, int RG, int CPL, int D>
 cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
                               cudaStream_t stream, bool pdl, const FusedInput* fused, bool x_bf16, bool* launched,
-                              bool fuse_always, bool alpha_rows = false) {
+                              bool fuse_always, bool alpha_rows = false, bool a4 = false) {
     using Shared = GShared<W>;
     if (launched) *launched = true;
+    if (a4 && !fused) return cudaErrorInvalidValue;  // 4-bit activations only with the fused prologue
     GParams P;
     fill_params(P, problems, count, RG, CPL, alpha_rows);
     int64_t weight_bytes = 0;
@@ -1032,6 +1048,7 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
             slot_row = std::max(slot_row, 64 * q.C);
         }
         P.x_bf16 = x_bf16 ? 1 : 0;
+        P.a4 = a4 ? 1 : 0;
         P.slot_row = slot_row;
         bool fits = smem + (size_t)kMaxSlots * MT * slot_row <= smem_cap;
         // the prologue holds a row in registers: at most W·32·kFuseVec 16-byte vectors
@@ -1086,10 +1103,11 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
 template <int MT>
 cudaError_t launch_stream(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
                           cudaStream_t stream, bool pdl, const FusedInput* fused = nullptr, bool x_bf16 = false,
-                          bool* launched = nullptr, bool fuse_always = false, bool alpha_rows = false) {
+                          bool* launched = nullptr, bool fuse_always = false, bool alpha_rows = false,
+                          bool a4 = false) {
     using C = StreamCfg<MT>;
     return launch_stream_cfg<MT, C::W, C::MINB, C::RG, C::CPL, C::D>(problems, count, dev, stream, pdl, fused, x_bf16,
-                                                                     launched, fuse_always, alpha_rows);
+                                                                     launched, fuse_always, alpha_rows, a4);
 }
 
 cudaError_t launch_generic(const bitlinear_forward_problem* problems, int count, const DeviceInfo& dev,
@@ -1156,7 +1174,7 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
 
 cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const FusedInput* in, int count,
                                 bitlinear_dtype dtype, cudaStream_t stream, bool pdl, bool* launched,
-                                bool alpha_rows) {
+                                bool alpha_rows, bool a4) {
     *launched = false;
     // BITLINEAR_LINEAR_FUSION=off never fuses, =on fuses whenever the
     // problems fit the kernel (skipping the byte-ratio rule); default: auto
@@ -1177,9 +1195,12 @@ cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const
         if (s.M > max_m) max_m = s.M;
     }
     const bool bf16 = dtype == BL_BF16;
-    if (max_m == 1) return launch_stream<1>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows);
-    if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows);
-    if (max_m <= 4) return launch_stream<4>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows);
+    if (max_m == 1)
+        return launch_stream<1>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows, a4);
+    if (max_m == 2)
+        return launch_stream<2>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows, a4);
+    if (max_m <= 4)
+        return launch_stream<4>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows, a4);
     return cudaSuccess;
 }
 
