@@ -770,8 +770,8 @@ def run_hadamard(args, world, local_rank):
     """The 7B decode set with the Hadamard rotation before the absmax
     quantisation ("1.58-bit 大模型极限量化实战" §6.2): weights quantised once from
     W·H/b (not timed); one step = one bitlinear_linear_grouped call flagged
-    BL_LINEAR_HADAMARD | BL_LINEAR_WEIGHTS_STATIC (the grouped rotate+quantise
-    kernel, then the GEMV, chained by PDL)."""
+    BL_LINEAR_HADAMARD | BL_LINEAR_WEIGHTS_STATIC: one GEMV launch whose CTAs
+    rotate and quantise their input rows in the prologue; steps chained by PDL)."""
     import torch
     import bitlinear_w1_a8_03_b200 as bl
     from bitlinear_w1_a8_03_b200 import synth
@@ -811,7 +811,7 @@ def run_hadamard(args, world, local_rank):
                         "power of two dividing K (4096 for K=4096, 256 for K=11008)",
             "us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
             "bytes_per_step": bps, "steps": K, "replicas": replicas,
-            "launches_per_step": 2, "clocks": clocks}
+            "launches_per_step": 1, "clocks": clocks}
 
 
 # ----------------------------------------------------------------------------- scale-granularity leg

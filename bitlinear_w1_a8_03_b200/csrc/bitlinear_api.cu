@@ -232,7 +232,15 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool weights_static = (flags & BL_LINEAR_WEIGHTS_STATIC) != 0;
     if (rotate) {
-        // rotation + quantisation in one grouped launch, then the product
+        // one token: rotation and quantisation in the product kernel's prologue
+        bl::FusedInput rin[BITLINEAR_MAX_GROUP];
+        for (int i = 0; i < count; ++i)
+            rin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true,
+                                    (int32_t)bitlinear_hadamard_block(problems[i].K)};
+        bool fused = false;
+        st = from_cuda(bl::launch_linear_fused(fwd, rin, count, dtype, s, weights_static, &fused));
+        if (st != BL_OK || fused) return st;
+        // else rotation + quantisation in one grouped launch, then the product
         // (the product kernel streams weights early only under the flag)
         bl::HadJob jobs[BITLINEAR_MAX_GROUP];
         for (int i = 0; i < count; ++i)
@@ -244,7 +252,7 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     }
     // few tokens: one launch that quantises in the product kernel's prologue
     bl::FusedInput fin[BITLINEAR_MAX_GROUP];
-    for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
+    for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true, 0};
     bool launched = false;
     st = from_cuda(bl::launch_linear_fused(fwd, fin, count, dtype, s, weights_static, &launched));
     if (st != BL_OK || launched) return st;
@@ -298,7 +306,7 @@ bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, i
                 ok = false;
                 break;
             }
-            fin[i] = bl::FusedInput{acts[j].a, acts[j].b, used[j] ? nullptr : acts[j].x_sum, !used[j]};
+            fin[i] = bl::FusedInput{acts[j].a, acts[j].b, used[j] ? nullptr : acts[j].x_sum, !used[j], 0};
             used[j] = true;
         }
         for (int j = 0; j < n_acts && ok; ++j) ok = used[j];
@@ -424,7 +432,7 @@ bitlinear_status bitlinear_linear_scaled(const bitlinear_scaled_problem* problem
         }
         if (nact == count) {
             bl::FusedInput fin[BITLINEAR_MAX_GROUP];
-            for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
+            for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true, 0};
             bool launched = false;
             st = from_cuda(bl::launch_linear_fused(f, fin, count, dtype, s, weights_static, &launched, true));
             if (st != BL_OK || launched) return st;
@@ -496,7 +504,7 @@ bitlinear_status bitlinear_linear_a4(const bitlinear_linear_problem* problems, i
         fusable = problems[i].M <= 4 && problems[i].K % 16 == 0 && !misaligned(problems[i].x_q, 4);
     if (fusable) {
         bl::FusedInput fin[BITLINEAR_MAX_GROUP];
-        for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true};
+        for (int i = 0; i < count; ++i) fin[i] = bl::FusedInput{problems[i].x, nullptr, nullptr, true, 0};
         bool launched = false;
         st = from_cuda(bl::launch_linear_fused(fwd, fin, count, dtype, s, weights_static, &launched, false, true));
         if (st != BL_OK || launched) return st;

@@ -75,6 +75,7 @@ struct FusedInput {
     const float* x2;
     float* x_sum;
     bool write_outputs;
+    int32_t had_block;  // > 0: rotate x by the block-diagonal Hadamard of this block first (x2, x_sum NULL)
 };
 // *launched = false (and nothing enqueued) when the problems do not fit the
 // fused kernel; the caller then runs the quantisation and product separately.

@@ -75,6 +75,7 @@ struct GProblem {
     const float* x2;        // nullable float32 second addend
     float* x_sum;           // nullable: stores x (+ x2)
     int32_t write_outputs;  // the owner CTA writes x̃ to xq and β to beta (and x_sum)
+    int32_t had_block;      // > 0: x is rotated by the block-diagonal Hadamard first
 };
 
 constexpr int kMaxCta = 512;  // most CTAs of one launch
@@ -86,6 +87,7 @@ struct GParams {
     int32_t cta_begin[kMaxCta + 1];  // first step of each CTA (row-group boundaries), then the end
     int x_bf16;        // fused: activation dtype
     int a4;            // fused: 4-bit activations (codes in [-7, 7], x̃ written as nibbles, scale α·β/7)
+    int had;           // fused: the inputs are rotated (every problem has a Hadamard block)
     int32_t slot_row;  // fused: bytes per token row of a shared x̃ slot (64·ceil(K/64) of the widest problem)
 };
 
@@ -149,6 +151,7 @@ struct QRow {
     float* x_sum;     // nullable x (+ x2) out (with `out`)
     uint32_t dst;     // shared address of the slot row
     int slot, m, K;
+    int had;     // > 0: rotate by the block-diagonal Hadamard of this block size first
     bool valid;  // a row to quantise
     bool out;    // also write x̃, β (and x) to global memory
 };
@@ -324,6 +327,135 @@ __device__ void fused_quantize_rows(const QRow (&q)[kFuseRows], int32_t slot_row
 __device__ __forceinline__ float token_scale(int alpha_rows, int a4, float alpha, float beta) {
     if (a4) return dequant_scale_a4(alpha, beta);
     return alpha_rows ? __double2float_rn(__ddiv_rn((double)beta, 127.0)) : dequant_scale(alpha, beta);
+}
+
+__host__ __device__ constexpr int ilog2_const(int v) { return v <= 1 ? 0 : 1 + ilog2_const(v / 2); }
+
+// Scratch for a rotated row, in the stages that no copy targets before the
+// main loop: segment s (SEG floats) is the last stage of warp s's ring.
+struct RotScratch {
+    uint32_t base;    // shared address of segment 0
+    uint32_t stride;  // bytes from one segment to the next (one warp's ring)
+    int seg_log2;     // log2 of the floats per segment
+    __device__ __forceinline__ uint32_t addr(int e) const {
+        return base + (uint32_t)(e >> seg_log2) * stride + 4u * (uint32_t)(e & ((1 << seg_log2) - 1));
+    }
+};
+
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+// One input row rotated, then quantised like fused_quantize_rows: x·H with H
+// block-diagonal Sylvester Hadamard of block q.had ("1.58-bit 大模型极限量化实战",
+// chenxutan.com/d/5049.html §6.2), butterfly stages h = 1, 2, 4, … each
+// rounded to binary32 (the first log2(V) inside a thread's vector, the rest
+// in the shared scratch with a barrier per stage), then β = max|x·H| + 1e-8
+// and the codes.  K ≤ the scratch's floats, q.had ≥ 8 (the host checks).
+template <typename T, int NT>
+__device__ void fused_rotate_quantize_row(const QRow& q, const RotScratch& sc, int32_t slot_row, float (*red)[32],
+                                          float (*xbeta)[kGemvMaxTokens], int (*xsum)[kGemvMaxTokens], bool a4) {
+    constexpr int V = FusedVec<T>::n;
+    const float qmax = a4 ? 7.0f : 127.0f;
+    const int K = q.K, nvec = K / V;
+    const int64_t base = (int64_t)q.m * K;
+    // load, the in-vector stages, store as binary32
+    for (int v = threadIdx.x; v < nvec; v += NT) {
+        float f[V];
+        FusedVec<T>::unpack(FusedVec<T>::load(q, base + (int64_t)v * V), f);
+#pragma unroll
+        for (int h = 1; h < V; h <<= 1)
+#pragma unroll
+            for (int e = 0; e < V; ++e)
+                if (!(e & h)) {
+                    const float a = f[e], b = f[e + h];
+                    f[e] = __fadd_rn(a, b);
+                    f[e + h] = __fsub_rn(a, b);
+                }
+#pragma unroll
+        for (int g = 0; g < V / 4; ++g)
+            sts128(sc.addr(v * V + 4 * g), make_uint4(__float_as_uint(f[4 * g]), __float_as_uint(f[4 * g + 1]),
+                                                      __float_as_uint(f[4 * g + 2]), __float_as_uint(f[4 * g + 3])));
+    }
+    __syncthreads();
+    // the remaining stages, pairs (i, i + h) inside each block
+    for (int lh = ilog2_const(V); (1 << lh) < q.had; ++lh) {
+        const int h = 1 << lh;
+        for (int pidx = threadIdx.x; pidx < K / 2; pidx += NT) {
+            const int i = ((pidx >> lh) << (lh + 1)) | (pidx & (h - 1));
+            const uint32_t ai = sc.addr(i), bi = sc.addr(i + h);
+            const float a = lds_f32(ai), b = lds_f32(bi);
+            sts_f32(ai, __fadd_rn(a, b));
+            sts_f32(bi, __fsub_rn(a, b));
+        }
+        __syncthreads();
+    }
+    // β of the rotated row (eight elements per item: two 16-byte reads)
+    auto item = [&](int v, float (&f)[8]) {
+        const uint4 u0 = lds128_after(sc.addr(8 * v)), u1 = lds128_after(sc.addr(8 * v + 4));
+        f[0] = __uint_as_float(u0.x);
+        f[1] = __uint_as_float(u0.y);
+        f[2] = __uint_as_float(u0.z);
+        f[3] = __uint_as_float(u0.w);
+        f[4] = __uint_as_float(u1.x);
+        f[5] = __uint_as_float(u1.y);
+        f[6] = __uint_as_float(u1.z);
+        f[7] = __uint_as_float(u1.w);
+    };
+    float mx = 0.0f;
+    for (int v = threadIdx.x; v < K / 8; v += NT) {
+        float f[8];
+        item(v, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));  // exact, order-free
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    __syncthreads();  // red[] free from any previous use
+    if ((threadIdx.x & 31) == 0) red[0][threadIdx.x >> 5] = mx;
+    __syncthreads();
+    float bmax = red[0][0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) bmax = fmaxf(bmax, red[0][w]);
+    const float beta = __fadd_rn(bmax, 1e-8f);
+    const float qf = quant_factor(beta, qmax);
+    // codes
+    int qsum = 0;
+    for (int v = threadIdx.x; v < K / 8; v += NT) {
+        float f[8];
+        item(v, f);
+        uint32_t wq[2];
+        quantize_codes<8>(f, beta, qf, wq, qmax);
+        qsum = dp4a_s8s8(0x01010101u, wq[0], qsum);
+        qsum = dp4a_s8s8(0x01010101u, wq[1], qsum);
+        const int k = 8 * v;
+        sts32(q.dst + xs_offset(k), wq[0]);
+        sts32(q.dst + xs_offset(k + 4), wq[1]);
+        if (q.out) {
+            if (a4) {
+                // two codes per byte, element 2j in the low nibble ("BitNet CPU 实测" §2.1 variant)
+                const uint32_t lo = wq[0] & 0x0F0F0F0Fu, hi = wq[1] & 0x0F0F0F0Fu;
+                *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(q.xq) + (int64_t)q.m * (K / 2) + k / 2) =
+                    __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6420);
+            } else {
+                *reinterpret_cast<uint2*>(q.xq + base + k) = make_uint2(wq[0], wq[1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&xsum[q.slot][q.m], qsum);  // integer: exact in any order
+    if (threadIdx.x == 0) {
+        xbeta[q.slot][q.m] = beta;
+        if (q.out) q.beta[q.m] = beta;
+    }
+    for (int k = K + 4 * threadIdx.x; k < slot_row; k += 4 * NT) sts32(q.dst + xs_offset(k), 0u);
+    __syncthreads();  // the scratch is free again (for a next row)
 }
 
 // ---------------------------------------------------------------- reductions
@@ -544,8 +676,10 @@ __device__ __forceinline__ void step_math(const uint4 (&w)[RG], const uint32_t (
 // row group's first chunk subtracts the token's whole-row Σx̃ (summed while
 // quantising) once, so every row's total is Σ c·x̃ - Σ x̃ over the full row.
 // With x̃ from global memory each lane adds up the Σx̃ of the chunks it
-// multiplies and subtracts it from its own partial sums.
-template <int MT, int W, int MINB, int RG, int CPL, int D, bool FUSE>
+// multiplies and subtracts it from its own partial sums.  FUSE: 0 x̃ from
+// global memory, 1 the prologue quantises x, 2 it rotates x, then quantises
+// (a separate instance, so the rotation's code does not weigh on the others).
+template <int MT, int W, int MINB, int RG, int CPL, int D, int FUSE>
 __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_constant__ GParams P) {
     constexpr int NQ = MT <= 2 ? 4 : 1;  // one accumulator per code field (no shifts) for few tokens
     constexpr int V = RG * MT;           // sums per lane when a row group is done
@@ -642,6 +776,7 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
                     r.slot = slot;
                     r.m = m;
                     r.K = pr.K;
+                    r.had = pr.had_block;
                     r.out = owner && pr.write_outputs != 0;
                 }
             }
@@ -652,7 +787,20 @@ __global__ void __launch_bounds__(W * 32, MINB) gemv_stream_kernel(const __grid_
 #pragma unroll
         for (int i = 0; i < kMaxSlots * MT; i += kFuseRows) {
             const QRow(&pair)[kFuseRows] = *reinterpret_cast<const QRow(*)[kFuseRows]>(&rows[i]);
-            if (pair[0].valid || pair[1].valid) {  // the same in every thread of the CTA
+            if constexpr (FUSE == 2) {  // rotated rows one at a time through the scratch
+                const RotScratch sc{smem_addr(smem_raw + sizeof(Shared)) + (uint32_t)((D - 1) * kStage),
+                                    (uint32_t)(D * kStage), ilog2_const(kStage / 4)};
+#pragma unroll
+                for (int e = 0; e < kFuseRows; ++e) {
+                    if (!pair[e].valid) continue;  // the same in every thread of the CTA
+                    if (P.x_bf16)
+                        fused_rotate_quantize_row<uint16_t, W * 32>(pair[e], sc, P.slot_row, S.red, S.xbeta, S.xsum,
+                                                                    P.a4 != 0);
+                    else
+                        fused_rotate_quantize_row<float, W * 32>(pair[e], sc, P.slot_row, S.red, S.xbeta, S.xsum,
+                                                                 P.a4 != 0);
+                }
+            } else if (pair[0].valid || pair[1].valid) {  // the same in every thread of the CTA
                 if (P.x_bf16)
                     fused_quantize_rows<uint16_t, W * 32>(pair, P.slot_row, S.red, S.xbeta, S.xsum, P.a4 != 0);
                 else
@@ -1045,17 +1193,29 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
             q.x2 = fused[i].x2;
             q.x_sum = fused[i].x_sum;
             q.write_outputs = fused[i].write_outputs ? 1 : 0;
+            q.had_block = fused[i].had_block;
             slot_row = std::max(slot_row, 64 * q.C);
         }
         P.x_bf16 = x_bf16 ? 1 : 0;
         P.a4 = a4 ? 1 : 0;
+        P.had = fused[0].had_block > 0 ? 1 : 0;
         P.slot_row = slot_row;
         bool fits = smem + (size_t)kMaxSlots * MT * slot_row <= smem_cap;
+        for (int i = 0; i < count; ++i) {
+            // all problems rotated or none; a rotated row fits the scratch in the
+            // last stage of every warp's ring, which nothing fills before the loop
+            fits = fits && (fused[i].had_block > 0) == (P.had != 0);
+            if (P.had)  // (built for one token; blocks of at least 8 dividing K)
+                fits = fits && MT == 1 && D >= 2 && fused[i].had_block >= 8 &&
+                       (fused[i].had_block & (fused[i].had_block - 1)) == 0 && P.p[i].K % fused[i].had_block == 0 && (int64_t)P.p[i].K <= (int64_t)W * (CPL * RG * 512 / 4) && !fused[i].x2 &&
+                       !fused[i].x_sum;
+        }
         // the prologue holds a row in registers: at most W·32·kFuseVec 16-byte vectors
         for (int i = 0; i < count; ++i)
             fits = fits && (int64_t)P.p[i].K * (x_bf16 ? 2 : 4) <= (int64_t)W * 32 * kFuseVec * 16;
         double pro[kMaxGroup];
-        for (int i = 0; i < count; ++i) pro[i] = prologue_cost(W, CPL, P.p[i].K) * std::min<int>(P.p[i].M, MT);
+        for (int i = 0; i < count; ++i)  // a rotation about doubles the prologue
+            pro[i] = prologue_cost(W, CPL, P.p[i].K) * std::min<int>(P.p[i].M, MT) * (P.had ? 2 : 1);
         grid = cta_ranges(P, G, pro);
         // Every CTA reads its problems' whole input rows before its main loop;
         // that pays off only while those reads are small next to the weights.
@@ -1081,8 +1241,10 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
         grid = cta_ranges(P, G, nullptr);
     }
     if (smem > smem_cap) return cudaErrorInvalidConfiguration;  // a shape that does not fit (not built)
-    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, true>)
-                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, false>);
+    const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, 1>)
+                               : reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, 0>);
+    if constexpr (MT == 1)
+        if (fused && P.had) kernel = reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, 2>);
     // the opt-in is per device: set once on each device that launches the kernel
     cudaError_t err = set_max_dynamic_smem(kernel, (int)smem_cap);
     if (err != cudaSuccess) return err;

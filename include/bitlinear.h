@@ -239,8 +239,9 @@ BITLINEAR_API bitlinear_status bitlinear_linear(const void* x, bitlinear_dtype d
 /* bitlinear_linear on `count` independent problems of one input dtype: one
  * grouped quantisation launch and one grouped product launch.  `problems` is a
  * HOST array.  flags: BL_LINEAR_WEIGHTS_STATIC and/or BL_LINEAR_HADAMARD.
- * With at most four tokens per problem (and no rotation) the quantisation may instead run in
- * the product kernel's prologue (one launch; x_q and beta are still written),
+ * With at most four tokens per problem (one token when rotated, K ≤ 24576) the
+ * quantisation (and rotation) may instead run in the product kernel's prologue
+ * (one launch; x_q and beta are still written),
  * when the problems fit it and the input rows are small next to the weights;
  * the environment variable BITLINEAR_LINEAR_FUSION=on|off forces the choice.
  * Results are identical either way.

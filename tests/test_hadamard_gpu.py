@@ -118,3 +118,45 @@ def test_rotated_prefill_grouped():
         assert np.array_equal(np_(p["acc_out"])[:, rows], acc_r)
         y = np_(p["y"])[:, rows].astype(np.float64)
         assert np.all(np.abs(y - y_r) <= 1e-5 * np.abs(y_r) + 1e-37)
+
+
+# (N, K): rotation blocks of 64 (K = 64, and a row ending in a partial
+# 64-element chunk), 16, 256, the largest row the one-token kernel rotates
+# in its prologue, and one longer (28672: the separate rotation launch)
+ONE_TOKEN = [(40, 64), (136, 2112), (72, 1040), (1000, 11008), (264, 16384), (24, 24576), (16, 28672)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_rotated_linear_one_token(dtype, fusion):
+    """One token with BL_LINEAR_HADAMARD, with the rotation inside the product
+    kernel's prologue (forced on), in its own launch (off) or as the library
+    picks: x̃, β and the int32 accumulators bit-exact, y within 1e-5."""
+    probs, refs = [], []
+    for j, (N, K) in enumerate(ONE_TOKEN):
+        b = bl.hadamard_block(K)
+        W = synth.weights(100 + j, N, K, 0.02)
+        packed, alpha = bl.bitlinear_quantize_weights_rotated(torch.from_numpy(W).cuda(), b)
+        _, a_ref, codes, _ = oracle.quantize_weights_rotated(W, b)
+        x = synth.activations(200 + j, 1, K, outliers=True)
+        if j == 2:
+            x[:] = 0.0  # a zero token: β = 1e-8 and every code 0
+        xd, xo = as_input(x, dtype)
+        probs.append(dict(x=xd, x_q=torch.empty((1, K), dtype=torch.int8, device="cuda"),
+                          beta=torch.empty(1, dtype=torch.float32, device="cuda"), W_packed=packed, alpha=alpha,
+                          N=N, y=torch.empty((1, N), dtype=torch.float32, device="cuda"),
+                          acc_out=torch.empty((1, N), dtype=torch.int32, device="cuda")))
+        refs.append((xo, codes, a_ref, b))
+    # one call per problem: forced on, every row that fits the prologue is fused
+    for p in probs:
+        bl.bitlinear_linear_grouped([p], flags=bl.BL_LINEAR_HADAMARD)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    for p, (xo, codes, a_ref, b) in zip(probs, refs):
+        xq_r, beta_r, _ = oracle.quantize_act_rotated(xo, b)
+        acc_r = oracle.ternary_matmul(xq_r, codes, threads=8)
+        y_r = oracle.dequant(acc_r, beta_r, a_ref).astype(np.float64)
+        assert np.array_equal(np_(p["beta"]), beta_r)
+        assert np.array_equal(np_(p["x_q"]), xq_r)
+        assert np.array_equal(np_(p["acc_out"]), acc_r)
+        y = np_(p["y"]).astype(np.float64)
+        assert np.all(np.abs(y - y_r) <= 1e-5 * np.abs(y_r) + 1e-37)
