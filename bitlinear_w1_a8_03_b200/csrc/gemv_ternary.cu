@@ -351,84 +351,139 @@ __device__ __forceinline__ void sts_f32(uint32_t a, float v) {
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
 
+// Butterfly stages h, 2h, …, h·R/2 of the rotation over the scratch in one
+// pass: each item holds the R elements i + j·h (closed under those stages)
+// in registers and runs the stages in order, so every butterfly is the same
+// binary32 add or subtract as in a pass per stage.  Returns this thread's
+// max |value| written.
+template <int R>
+__device__ __forceinline__ float rotate_pass(const RotScratch& sc, int K, int lh, int nt) {
+    constexpr int r = R == 2 ? 1 : R == 4 ? 2 : 3;
+    const int h = 1 << lh;
+    float mx = 0.0f;
+    for (int it = threadIdx.x; it < K / R; it += nt) {
+        const int i = ((it >> lh) << (lh + r)) | (it & (h - 1));
+        float f[R];
+#pragma unroll
+        for (int j = 0; j < R; ++j) f[j] = lds_f32(sc.addr(i + j * h));
+#pragma unroll
+        for (int st = 1; st < R; st <<= 1)
+#pragma unroll
+            for (int j = 0; j < R; ++j)
+                if (!(j & st)) {
+                    const float a = f[j], b = f[j + st];
+                    f[j] = __fadd_rn(a, b);
+                    f[j + st] = __fsub_rn(a, b);
+                }
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            sts_f32(sc.addr(i + j * h), f[j]);
+            mx = fmaxf(mx, fabsf(f[j]));
+        }
+    }
+    return mx;
+}
+
 // One input row rotated, then quantised like fused_quantize_rows: x·H with H
 // block-diagonal Sylvester Hadamard of block q.had ("1.58-bit 大模型极限量化实战",
 // chenxutan.com/d/5049.html §6.2), butterfly stages h = 1, 2, 4, … each
-// rounded to binary32 (the first log2(V) inside a thread's vector, the rest
-// in the shared scratch with a barrier per stage), then β = max|x·H| + 1e-8
-// and the codes.  K ≤ the scratch's floats, q.had ≥ 8 (the host checks).
+// rounded to binary32, then β = max|x·H| + 1e-8 and the codes.  A lane holds
+// 8 consecutive elements of a 256-element tile (a warp per tile): stages
+// h < 8 run in its registers, 8 ≤ h < 256 between lanes by shuffles, and the
+// tile goes to the scratch; larger stages run there, up to three per pass.
+// K ≤ the scratch's floats, K·(element bytes) ≤ NT·kFuseVec·16, q.had ≥ 8
+// (the host checks).
 template <typename T, int NT>
 __device__ void fused_rotate_quantize_row(const QRow& q, const RotScratch& sc, int32_t slot_row, float (*red)[32],
                                           float (*xbeta)[kGemvMaxTokens], int (*xsum)[kGemvMaxTokens], bool a4) {
     constexpr int V = FusedVec<T>::n;
+    constexpr int kLd = 8 / V;                 // 16-byte loads per 8-element unit
+    constexpr int kUnits = kFuseVec / kLd;     // units per thread at most
+    constexpr int kW = NT / 32;
     const float qmax = a4 ? 7.0f : 127.0f;
-    const int K = q.K, nvec = K / V;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int K = q.K, tiles = (K + 255) / 256;
     const int64_t base = (int64_t)q.m * K;
-    // load, the in-vector stages, store as binary32
-    for (int v = threadIdx.x; v < nvec; v += NT) {
-        float f[V];
-        FusedVec<T>::unpack(FusedVec<T>::load(q, base + (int64_t)v * V), f);
+    // every load first: unit j of this lane is elements 256·(warp + j·kW) + 8·lane + [0, 8)
+    uint4 raw[kUnits][kLd];
 #pragma unroll
-        for (int h = 1; h < V; h <<= 1)
+    for (int j = 0; j < kUnits; ++j) {
+        const int e = 256 * (warp + j * kW) + 8 * lane;
+        if (warp + j * kW < tiles) {
 #pragma unroll
-            for (int e = 0; e < V; ++e)
+            for (int l = 0; l < kLd; ++l)
+                raw[j][l] = e < K ? FusedVec<T>::load(q, base + e + l * V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    const int lhad = 31 - __clz(q.had);
+    const int lsh = lhad < 8 ? lhad : 8;  // stages below 2^lsh stay in the warp
+    float mx = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kUnits; ++j) {
+        if (warp + j * kW >= tiles) continue;  // the same in every lane of the warp
+        float f[8];
+#pragma unroll
+        for (int l = 0; l < kLd; ++l) {
+            float g[V];
+            FusedVec<T>::unpack(raw[j][l], g);
+#pragma unroll
+            for (int e = 0; e < V; ++e) f[l * V + e] = g[e];
+        }
+#pragma unroll
+        for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
                 if (!(e & h)) {
                     const float a = f[e], b = f[e + h];
                     f[e] = __fadd_rn(a, b);
                     f[e + h] = __fsub_rn(a, b);
                 }
+        for (int lh = 3; lh < lsh; ++lh) {
+            // pair (i, i + h) across lanes lane and lane ^ h/8: the lower lane keeps
+            // a + b, the upper one a - b (a from the lower lane)
+            const int mask = 1 << (lh - 3);
+            const bool upper = (lane & mask) != 0;
 #pragma unroll
-        for (int g = 0; g < V / 4; ++g)
-            sts128(sc.addr(v * V + 4 * g), make_uint4(__float_as_uint(f[4 * g]), __float_as_uint(f[4 * g + 1]),
-                                                      __float_as_uint(f[4 * g + 2]), __float_as_uint(f[4 * g + 3])));
-    }
-    __syncthreads();
-    // the remaining stages, pairs (i, i + h) inside each block
-    for (int lh = ilog2_const(V); (1 << lh) < q.had; ++lh) {
-        const int h = 1 << lh;
-        for (int pidx = threadIdx.x; pidx < K / 2; pidx += NT) {
-            const int i = ((pidx >> lh) << (lh + 1)) | (pidx & (h - 1));
-            const uint32_t ai = sc.addr(i), bi = sc.addr(i + h);
-            const float a = lds_f32(ai), b = lds_f32(bi);
-            sts_f32(ai, __fadd_rn(a, b));
-            sts_f32(bi, __fsub_rn(a, b));
+            for (int e = 0; e < 8; ++e) {
+                const float o = __shfl_xor_sync(0xffffffffu, f[e], mask);
+                f[e] = upper ? __fsub_rn(o, f[e]) : __fadd_rn(f[e], o);
+            }
         }
-        __syncthreads();
-    }
-    // β of the rotated row (eight elements per item: two 16-byte reads)
-    auto item = [&](int v, float (&f)[8]) {
-        const uint4 u0 = lds128_after(sc.addr(8 * v)), u1 = lds128_after(sc.addr(8 * v + 4));
-        f[0] = __uint_as_float(u0.x);
-        f[1] = __uint_as_float(u0.y);
-        f[2] = __uint_as_float(u0.z);
-        f[3] = __uint_as_float(u0.w);
-        f[4] = __uint_as_float(u1.x);
-        f[5] = __uint_as_float(u1.y);
-        f[6] = __uint_as_float(u1.z);
-        f[7] = __uint_as_float(u1.w);
-    };
-    float mx = 0.0f;
-    for (int v = threadIdx.x; v < K / 8; v += NT) {
-        float f[8];
-        item(v, f);
+        const int e0 = 256 * (warp + j * kW) + 8 * lane;
+        if (e0 < K) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));  // exact, order-free
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
+            sts128(sc.addr(e0), make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                           __float_as_uint(f[3])));
+            sts128(sc.addr(e0 + 4), make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]),
+                                               __float_as_uint(f[6]), __float_as_uint(f[7])));
+        }
     }
+    // the stages from 256 up, two or three per pass (5 → 3 + 2, 4 → 2 + 2)
+    for (int lh = lsh; lh < lhad;) {
+        const int rest = lhad - lh;
+        const int r = rest == 4 ? 2 : rest < 3 ? rest : 3;
+        __syncthreads();
+        mx = r == 1 ? rotate_pass<2>(sc, K, lh, NT) : r == 2 ? rotate_pass<4>(sc, K, lh, NT) : rotate_pass<8>(sc, K, lh, NT);
+        lh += r;
+    }
+    // β of the rotated row: the max over the last values every thread wrote
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    __syncthreads();  // red[] free from any previous use
-    if ((threadIdx.x & 31) == 0) red[0][threadIdx.x >> 5] = mx;
+    __syncthreads();  // red[] free from any previous use; the scratch is complete
+    if (lane == 0) red[0][warp] = mx;
     __syncthreads();
     float bmax = red[0][0];
 #pragma unroll
-    for (int w = 1; w < NT / 32; ++w) bmax = fmaxf(bmax, red[0][w]);
+    for (int w = 1; w < kW; ++w) bmax = fmaxf(bmax, red[0][w]);
     const float beta = __fadd_rn(bmax, 1e-8f);
     const float qf = quant_factor(beta, qmax);
-    // codes
+    // codes, eight elements per item
     int qsum = 0;
     for (int v = threadIdx.x; v < K / 8; v += NT) {
-        float f[8];
-        item(v, f);
+        const uint4 u0 = lds128_after(sc.addr(8 * v)), u1 = lds128_after(sc.addr(8 * v + 4));
+        const float f[8] = {__uint_as_float(u0.x), __uint_as_float(u0.y), __uint_as_float(u0.z), __uint_as_float(u0.w),
+                            __uint_as_float(u1.x), __uint_as_float(u1.y), __uint_as_float(u1.z), __uint_as_float(u1.w)};
         uint32_t wq[2];
         quantize_codes<8>(f, beta, qf, wq, qmax);
         qsum = dp4a_s8s8(0x01010101u, wq[0], qsum);
@@ -449,7 +504,7 @@ __device__ void fused_rotate_quantize_row(const QRow& q, const RotScratch& sc, i
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
-    if ((threadIdx.x & 31) == 0) atomicAdd(&xsum[q.slot][q.m], qsum);  // integer: exact in any order
+    if (lane == 0) atomicAdd(&xsum[q.slot][q.m], qsum);  // integer: exact in any order
     if (threadIdx.x == 0) {
         xbeta[q.slot][q.m] = beta;
         if (q.out) q.beta[q.m] = beta;
