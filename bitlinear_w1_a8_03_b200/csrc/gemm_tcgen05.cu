@@ -63,10 +63,10 @@ constexpr size_t kSmemLimit = 232448;  // opt-in dynamic shared memory per block
 #define BL_GEMM_SW_256 4
 #endif
 #ifndef BL_GEMM_SA_128
-#define BL_GEMM_SA_128 3
+#define BL_GEMM_SA_128 5
 #endif
 #ifndef BL_GEMM_SB_128
-#define BL_GEMM_SB_128 8
+#define BL_GEMM_SB_128 5
 #endif
 #ifndef BL_GEMM_SW_128
 #define BL_GEMM_SW_128 8
@@ -116,12 +116,12 @@ struct TileRef {
     int p, m0, n0, kblocks;
 };
 
-template <int NT>
+template <int NT, int ROWS = kRowsTile>
 __device__ __forceinline__ TileRef locate(const GemmParams& P, int tile) {
     int p = 0;
     while (p + 1 < P.count && tile >= P.p[p + 1].tile_begin) ++p;
     const int local = tile - P.p[p].tile_begin;
-    return TileRef{p, (local % P.p[p].tiles_m) * NT, (local / P.p[p].tiles_m) * kRowsTile, P.p[p].kblocks};
+    return TileRef{p, (local % P.p[p].tiles_m) * NT, (local / P.p[p].tiles_m) * ROWS, P.p[p].kblocks};
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -252,8 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     uint64_t* fullA = reinterpret_cast<uint64_t*>(ringW + (size_t)SW * C::kWBytes);
     uint64_t* emptyA = fullA + SA;
     uint64_t* fullB = emptyA + SA;
-    uint64_t* emptyB = fullB + SB;
-    uint64_t* fullW = emptyB + SB;
+    // with equal ring depths one MMA commit releases A slot s and x̃ slot s
+    // together (a commit costs the tensor pipe a few hundred cycles)
+    constexpr bool kOneRelease = SA == SB;
+    uint64_t* emptyB = kOneRelease ? emptyA : fullB + SB;
+    uint64_t* fullW = fullB + 2 * SB;
     uint64_t* emptyW = fullW + SW;
     uint64_t* accFull = emptyW + SW;  // [2]
     uint64_t* accEmpty = accFull + 2;  // [2]
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         for (int s = 0; s < SB; ++s) {
             mbar_init(smem_addr(&fullB[s]), 1);
-            mbar_init(smem_addr(&emptyB[s]), 1);
+            if (!kOneRelease) mbar_init(smem_addr(&emptyB[s]), 1);
         }
         for (int s = 0; s < SW; ++s) {
             mbar_init(smem_addr(&fullW[s]), 1);
@@ -341,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         mma_i8(d, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k), idesc,
                                (kb > 0 || k > 0) ? 1u : 0u);
                     mma_commit(smem_addr(&emptyA[sa]));
-                    mma_commit(smem_addr(&emptyB[sb]));
+                    if constexpr (!kOneRelease) mma_commit(smem_addr(&emptyB[sb]));
                 }
                 if (!ok) break;
                 mma_commit(smem_addr(&accFull[b]));
@@ -445,6 +448,333 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
 }
 
+// ---------------------------------------------------------------- few tokens
+// For at most 64 tokens the MMA is short (N = NT) and the shared-memory
+// traffic of expanded code tiles, not the tensor pipe, sets the pace.  This
+// variant expands the codes into TENSOR memory (tcgen05.st) and the MMA takes
+// its A operand from there.  Codes stay unsigned, c = ŵ + 1 ∈ {0, 1, 2}
+// (kind::i8 with A unsigned, B = x̃ signed), and TMEM lane 127 carries a row
+// of ones, so D[t][m] = Σ_k c·x̃ and D[127][m] = Σ_k x̃: acc = D[t] - D[127],
+// exact in int32.  A tile is 127 weight rows × NT tokens; K runs in stages of
+// 512 (16 MMAs of 128×NT×32 per stage and barrier round trip).
+namespace tm {
+constexpr int kKS = 512;                // K per stage
+constexpr int kWS = kKS / 4;            // packed bytes of one row per stage
+constexpr int kRows = 127;              // weight rows per tile
+constexpr int kOnes = 127;              // TMEM lane of the ones row
+constexpr int kSA = 3;                  // A stages in tensor memory
+constexpr uint32_t kACols = kKS / 4;    // 32-bit columns of one A stage
+constexpr uint32_t kAccCols = 128;      // accumulators in columns [0, 2·NT)
+constexpr uint32_t kTmemCols = 512;
+static_assert(kAccCols + kSA * kACols <= kTmemCols, "tensor memory budget");
+}  // namespace tm
+
+template <int NT>
+struct CfgTM {
+    static constexpr int kWBytes = 128 * tm::kWS;  // a W slot: 127 rows × 128 B, 1024-aligned
+    static constexpr int kWBox = tm::kRows * tm::kWS;
+    static constexpr int kBBytes = NT * tm::kKS;   // four boxes of NT rows × 128 B
+    static constexpr int kSW = 6;
+    static constexpr int kSB = tm::kSA;  // x̃ and A stages share one ring index and one release
+    static constexpr int kBars = 2 * tm::kSA + 2 * kSW + 7;
+    static constexpr size_t kSmem =
+        1024 + (size_t)kSW * kWBytes + (size_t)kSB * kBBytes + kBars * 8 + 16 + 2 * NT * sizeof(int);
+    static_assert(kSmem <= kSmemLimit, "shared memory budget");
+    static_assert(kSmem > kSmemLimit / 2, "one CTA per SM (the tensor memory is sized for one)");
+    static_assert(NT % 16 == 0 && 2 * NT <= (int)tm::kAccCols, "accumulator columns");
+};
+
+// Instruction descriptor: u8 (A, codes) × s8 (B, x̃) -> s32, both K-major, M = 128, N = NT.
+template <int NT>
+__host__ __device__ constexpr uint32_t instr_desc_u8s8() {
+    return (2u << 4)  // D format s32
+           | (0u << 7)  // A unsigned 8-bit
+           | (1u << 10)  // B signed 8-bit
+           | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kRowsTile >> 4) << 24);
+}
+
+// MMA with A read from tensor memory (M rows in lanes 0..127, four 8-bit K
+// elements per 32-bit column).
+__device__ __forceinline__ void mma_i8_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// This thread's lane, 32 consecutive 32-bit columns from taddr.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// A TMA producer that fills each ring slot with BOXES boxes (box b at
+// slot + b·box_stride, all completing on the slot's barrier).
+template <int S, int BOXES, int ROWS, int NT, typename Coord>
+__device__ void tma_producer_n(uint8_t* ring, uint32_t slot_bytes, uint32_t box_stride, uint32_t expect_bytes,
+                               uint64_t* full, uint64_t* empty, const GemmParams& P, volatile int* abort_flag,
+                               Coord coord) {
+    int it = 0;
+    for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+        const TileRef tr = locate<NT, ROWS>(P, tile);
+        for (int st = 0; st < tr.kblocks; ++st, ++it) {
+            const int s = it % S;
+            if (it >= S && !wait_or_abort(smem_addr(&empty[s]), ((it / S) - 1) & 1, abort_flag)) goto drain;
+            mbar_arrive_expect_tx(smem_addr(&full[s]), expect_bytes);
+#pragma unroll
+            for (int b = 0; b < BOXES; ++b) {
+                int x, y;
+                const CUtensorMap* map = coord(tr, st, b, x, y);
+                tma_load_2d(smem_addr(ring + (size_t)s * slot_bytes + (size_t)b * box_stride), map, x, y,
+                            smem_addr(&full[s]));
+            }
+        }
+    }
+drain:
+    for (int j = it - 1; j >= 0 && j >= it - S; --j)
+        if (!mbar_wait_bounded(smem_addr(&full[j % S]), (j / S) & 1)) record_timeout(abort_flag);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_constant__ GemmParams P) {
+    using C = CfgTM<NT>;
+    constexpr int SA = tm::kSA, SB = C::kSB, SW = C::kSW;
+    static_assert(SA == SB, "one ring index for the A and x̃ stages");
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* ringW = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ringB = ringW + (size_t)SW * C::kWBytes;
+    // A stage s (expander warps) and x̃ stage s (TMA) complete one barrier and
+    // are released by one MMA commit (a commit costs the tensor pipe ~300 cycles)
+    uint64_t* stageReady = reinterpret_cast<uint64_t*>(ringB + (size_t)SB * C::kBBytes);
+    uint64_t* stageFree = stageReady + SA;
+    uint64_t* fullW = stageFree + SA;
+    uint64_t* emptyW = fullW + SW;
+    uint64_t* accFull = emptyW + SW;    // [2]
+    uint64_t* accEmpty = accFull + 2;   // [2]
+    uint64_t* onesReady = accEmpty + 2; // [2]
+    uint64_t* drain = onesReady + 2;    // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* ones_sum = reinterpret_cast<int*>(tmem_slot + 4);  // [2][NT]: Σ x̃ of each token of the tile
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    griddep_launch_dependents();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(smem_addr(&stageReady[s]), kExpWarps + 1);
+            mbar_init(smem_addr(&stageFree[s]), 1);
+        }
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(smem_addr(&fullW[s]), 1);
+            mbar_init(smem_addr(&emptyW[s]), kExpWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_addr(&accFull[b]), 1);
+            mbar_init(smem_addr(&accEmpty[b]), kEpiWarps);
+            mbar_init(smem_addr(&onesReady[b]), 1);
+        }
+        mbar_init(smem_addr(drain), 1);
+        *abort_flag = 0;
+    }
+    fence_mbar_init();
+    if (warp == kWarpMma) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                     "r"(tm::kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_slot;
+
+    if (warp == kWarpTmaX) {
+        // ---- x̃: four 128-byte boxes per stage (written by the preceding kernel under PDL)
+        if (lane == 0) {
+            griddep_wait();
+            tma_producer_n<SB, 4, tm::kRows, NT>(ringB, C::kBBytes, NT * kKB, C::kBBytes, stageReady, stageFree, P, abort_flag,
+                                                 [&](const TileRef& tr, int st, int b, int& x, int& y) {
+                                                     x = st * tm::kKS + b * kKB;
+                                                     y = tr.m0;
+                                                     return &P.xmap[tr.p];
+                                                 });
+        }
+    } else if (warp == kWarpTmaW) {
+        // ---- packed codes: 127 rows × 128 B per stage (128-byte swizzle)
+        if (lane == 0)
+            tma_producer_n<SW, 1, tm::kRows, NT>(ringW, C::kWBytes, 0, C::kWBox, fullW, emptyW, P, abort_flag,
+                                                 [&](const TileRef& tr, int st, int, int& x, int& y) {
+                                                     x = st * tm::kWS;
+                                                     y = tr.n0;
+                                                     return &P.wmap[tr.p];
+                                                 });
+    } else if (warp == kWarpMma) {
+        // ---- MMA issue: 16 per stage, A from tensor memory
+        if (lane == 0) {
+            constexpr uint32_t idesc = instr_desc_u8s8<NT>();
+            int it = 0, j = 0;
+            for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+                const int stages = locate<NT, tm::kRows>(P, tile).kblocks;
+                const int b = j & 1;
+                if (j >= 2 && !wait_or_abort(smem_addr(&accEmpty[b]), ((j >> 1) - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_d + (uint32_t)(b * NT);
+                bool ok = true;
+                for (int st = 0; st < stages; ++st, ++it) {
+                    const int sa = it % SA;
+                    if (!(ok = wait_or_abort(smem_addr(&stageReady[sa]), (it / SA) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    const uint32_t a_col = tmem_d + tm::kAccCols + (uint32_t)sa * tm::kACols;
+                    const uint32_t b_addr = smem_addr(ringB + (size_t)sa * C::kBBytes);
+#pragma unroll
+                    for (int k = 0; k < tm::kKS / 32; ++k)
+                        mma_i8_ta(d, a_col + 8u * k, smem_desc_sw128(b_addr + (k >> 2) * (NT * kKB) + 32 * (k & 3)),
+                                  idesc, (st > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(smem_addr(&stageFree[sa]));
+                }
+                if (!ok) break;
+                mma_commit(smem_addr(&accFull[b]));
+            }
+            mma_commit(smem_addr(drain));
+            if (!mbar_wait_bounded(smem_addr(drain), 0)) record_timeout(abort_flag);
+        }
+    } else if (warp < kWarpEpi0) {
+        // ---- expand tile row t (= TMEM lane t) into the A stage; lane 127 is the ones row
+        const int q = warp & 3;
+        const int t = 32 * q + lane;
+        const bool ones = t == tm::kOnes;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        // row t's 128 bytes, chunk j stored at chunk j ^ (t & 7) (128-byte swizzle)
+        const uint32_t w_row = (uint32_t)t * tm::kWS;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+            const int stages = locate<NT, tm::kRows>(P, tile).kblocks;
+            bool ok = true;
+            for (int st = 0; st < stages; ++st, ++it) {
+                const int sw = it % SW, sa = it % SA;
+                if (!(ok = wait_or_abort(smem_addr(&fullW[sw]), (it / SW) & 1, abort_flag))) break;
+                uint32_t wd[32];
+                const uint32_t src = smem_addr(ringW + (size_t)sw * C::kWBytes) + w_row;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    // the ones row: 0x55 bytes hold code 1 in every field
+                    const uint4 u = ones ? make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u)
+                                         : lds128(src + 16u * (uint32_t)(c ^ (t & 7)));
+                    wd[4 * c + 0] = u.x;
+                    wd[4 * c + 1] = u.y;
+                    wd[4 * c + 2] = u.z;
+                    wd[4 * c + 3] = u.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive1(smem_addr(&emptyW[sw]));  // codes are in registers
+                if (it >= SA && !(ok = wait_or_abort(smem_addr(&stageFree[sa]), ((it / SA) - 1) & 1, abort_flag)))
+                    break;
+                tc_fence_after();
+                const uint32_t a_col = tmem_d + lane_base + tm::kAccCols + (uint32_t)sa * tm::kACols;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    // word 8g + i holds weights 16(8g+i) .. +15; field f of it -> column 4(8g+i) + f
+                    uint32_t r[32];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t w = wd[8 * g + i];
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) r[4 * i + f] = (w >> (2 * f)) & 0x03030303u;
+                    }
+                    tmem_st32(a_col + 32u * g, r);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive1(smem_addr(&stageReady[sa]));
+            }
+            if (!ok) break;
+        }
+    } else {
+        // ---- epilogue: tile row t; acc = D[t] - D[127]
+        griddep_wait();
+        const int q = warp & 3;
+        const int t = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int j = 0;
+        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+            const TileRef tr = locate<NT, tm::kRows>(P, tile);
+            const int M = P.p[tr.p].M, N = P.p[tr.p].N;
+            const float* beta_p = P.p[tr.p].beta;
+            const float* bias_p = P.p[tr.p].bias;
+            float* y = P.p[tr.p].y;
+            int32_t* acc_out = P.p[tr.p].acc_out;
+            const float alpha = *P.p[tr.p].alpha;
+            const int b = j & 1;
+            const int m0 = tr.m0;
+            const int row = tr.n0 + t;
+            const bool row_ok = t < tm::kRows && row < N;
+            const float bias = (row_ok && bias_p) ? bias_p[row] : 0.0f;
+            if (!wait_or_abort(smem_addr(&accFull[b]), (j >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            int* ones_b = ones_sum + b * NT;
+            if (q == 3) {
+                // lane 31 of this warp reads TMEM lane 127: publish Σ x̃ of every token
+#pragma unroll 1
+                for (int c = 0; c < NT; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c), r);
+                    if (lane == 31) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) ones_b[c + i] = (int)r[i];
+                    }
+                }
+                __syncwarp();
+                if (lane == 31) mbar_arrive1(smem_addr(&onesReady[b]));
+            }
+            if (!wait_or_abort(smem_addr(&onesReady[b]), (j >> 1) & 1, abort_flag)) break;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NT; c0 += 32) {
+                const int my_tok = m0 + c0 + lane;
+                const float my_scale = my_tok < M ? dequant_scale(alpha, beta_p[my_tok]) : 0.0f;
+#pragma unroll
+                for (int h = 0; h < 2 && c0 + 16 * h < NT; ++h) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c0 + 16 * h), r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float sc = __shfl_sync(0xffffffffu, my_scale, 16 * h + i);
+                        const int tok = m0 + c0 + 16 * h + i;
+                        if (row_ok && tok < M) {
+                            const int acc = (int)r[i] - ones_b[c0 + 16 * h + i];
+                            float out = __fmul_rn((float)acc, sc);
+                            if (bias_p) out = __fadd_rn(out, bias);
+                            y[(int64_t)tok * N + row] = out;
+                            if (acc_out) acc_out[(int64_t)tok * N + row] = acc;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive1(smem_addr(&accEmpty[b]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(tm::kTmemCols));
+    }
+}
+
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -477,9 +807,22 @@ cudaError_t encode_u8(CUtensorMap* map, const void* base, int64_t cols, int64_t 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int NT>
+// Launches gemm_tc_kernel<NT> (TMEM_A = false: tiles of 128 rows, K blocks of
+// 128, codes expanded in shared memory) or gemm_tm_kernel<NT> (TMEM_A = true:
+// tiles of 127 rows, stages of 512, codes expanded in tensor memory).
+template <int NT, bool TMEM_A>
 cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl) {
-    using C = Cfg<NT>;
+    constexpr int kRows = TMEM_A ? tm::kRows : kRowsTile;
+    constexpr int kStageK = TMEM_A ? tm::kKS : kKB;
+    size_t kSmem;
+    const void* kernel;
+    if constexpr (TMEM_A) {
+        kSmem = CfgTM<NT>::kSmem;
+        kernel = reinterpret_cast<const void*>(gemm_tm_kernel<NT>);
+    } else {
+        kSmem = Cfg<NT>::kSmem;
+        kernel = reinterpret_cast<const void*>(gemm_tc_kernel<NT>);
+    }
     DeviceInfo dev;
     cudaError_t err = device_info(&dev);
     if (err != cudaSuccess) return err;
@@ -501,7 +844,10 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
         err = encode_u8(&P.xmap[i], pr.x_q, pr.K, pr.M, kKB, NT, CU_TENSOR_MAP_SWIZZLE_128B);
         if (err != cudaSuccess) return err;
         const int64_t row_bytes = (int64_t)bitlinear_packed_row_bytes(pr.K);
-        err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, kWB, kRowsTile, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (TMEM_A)
+            err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, tm::kWS, tm::kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+        else
+            err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, kWB, kRowsTile, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (err != cudaSuccess) return err;
         GemmProblem& q = P.p[i];
         q.alpha = pr.alpha;
@@ -511,27 +857,28 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
         q.acc_out = pr.acc_out;
         q.M = (int)pr.M;
         q.N = (int)pr.N;
-        q.kblocks = (int)((pr.K + kKB - 1) / kKB);
+        q.kblocks = (int)((pr.K + kStageK - 1) / kStageK);
         q.tiles_m = (int)((pr.M + NT - 1) / NT);
         q.tile_begin = tiles;
-        tiles += q.tiles_m * (int)((pr.N + kRowsTile - 1) / kRowsTile);
+        tiles += q.tiles_m * (int)((pr.N + kRows - 1) / kRows);
     }
     P.tiles = tiles;
 
     // the opt-in is per device: set once on each device that launches the kernel
-    err = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tc_kernel<NT>), (int)C::kSmem);
+    err = set_max_dynamic_smem(kernel, (int)kSmem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<NT>, P);
+    void* args[] = {&P};
+    return cudaLaunchKernelExC(&cfg, kernel, args);
 }
 
 }  // namespace
@@ -551,11 +898,11 @@ cudaError_t launch_gemm_tc(const bitlinear_forward_problem* problems, int count,
         tiles16 += ((problems[i].M + 15) / 16) * ((problems[i].N + kRowsTile - 1) / kRowsTile);
     }
     if (tiles16 >= ((int64_t)1 << 30)) return cudaErrorInvalidValue;  // tile numbers are int
-    if (max_m <= 16) return launch_nt<16>(problems, count, stream, pdl);
-    if (max_m <= 32) return launch_nt<32>(problems, count, stream, pdl);
-    if (max_m <= 64) return launch_nt<64>(problems, count, stream, pdl);
-    if (max_m <= 128) return launch_nt<128>(problems, count, stream, pdl);
-    return launch_nt<256>(problems, count, stream, pdl);
+    if (max_m <= 16) return launch_nt<16, true>(problems, count, stream, pdl);
+    if (max_m <= 32) return launch_nt<32, true>(problems, count, stream, pdl);
+    if (max_m <= 64) return launch_nt<64, true>(problems, count, stream, pdl);
+    if (max_m <= 128) return launch_nt<128, false>(problems, count, stream, pdl);
+    return launch_nt<256, false>(problems, count, stream, pdl);
 }
 
 cudaError_t read_gemm_error(int* code) {

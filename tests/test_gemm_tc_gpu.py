@@ -39,9 +39,17 @@ def test_gemm_token_counts(M):
     run_case(M, 256, 200, seed=600 + M, bias=(M % 2 == 1))
 
 
-@pytest.mark.parametrize("K,N", [(16, 130), (48, 128), (128, 127), (192, 257), (1024, 384), (4096 + 64, 256)])
+@pytest.mark.parametrize("K,N", [(16, 130), (48, 128), (128, 127), (192, 257), (1024, 384), (4096 + 64, 256),
+                                 (512, 254), (1536, 381)])
 def test_gemm_ragged_k_and_rows(K, N):
     run_case(37, K, N, seed=700 + K + N)
+
+
+@pytest.mark.parametrize("M", [8, 16, 24, 48])
+def test_gemm_few_tokens_many_stages_and_tiles(M):
+    """The few-token tensor-core path (tiles of 127 rows, K stages of 512)
+    over several stages, a ragged last stage and a one-row last tile."""
+    run_case(M, 2560 + 64, 127 * 4 + 1, seed=650 + M, bias=(M == 24))
 
 
 def test_gemm_prefill_shape_small_rows():
