@@ -110,6 +110,7 @@ struct GemmParams {
     GemmProblem p[kMaxGroup];
     int count;
     int tiles;
+    int cs;  // few-token kernel: CTAs per cluster, each taking 1/cs of every tile's K stages
 };
 
 struct TileRef {
@@ -474,11 +475,13 @@ struct CfgTM {
     static constexpr int kWBytes = 128 * tm::kWS;  // a W slot: 127 rows × 128 B, 1024-aligned
     static constexpr int kWBox = tm::kRows * tm::kWS;
     static constexpr int kBBytes = NT * tm::kKS;   // four boxes of NT rows × 128 B
-    static constexpr int kSW = 6;
+    static constexpr int kSW = NT >= 64 ? 5 : 6;
     static constexpr int kSB = tm::kSA;  // x̃ and A stages share one ring index and one release
-    static constexpr int kBars = 2 * tm::kSA + 2 * kSW + 7;
-    static constexpr size_t kSmem =
-        1024 + (size_t)kSW * kWBytes + (size_t)kSB * kBBytes + kBars * 8 + 16 + 2 * NT * sizeof(int);
+    static constexpr int kBars = 2 * tm::kSA + 2 * kSW + 9;
+    static constexpr int kRedStride = NT + 4;  // ints per row of the partial-sum buffer (conflict-free 16-byte access)
+    static constexpr size_t kRedBytes = (size_t)128 * kRedStride * sizeof(int);
+    static constexpr size_t kSmem = 1024 + (size_t)kSW * kWBytes + (size_t)kSB * kBBytes + kRedBytes + kBars * 8 + 16 +
+                                    2 * NT * sizeof(int);
     static_assert(kSmem <= kSmemLimit, "shared memory budget");
     static_assert(kSmem > kSmemLimit / 2, "one CTA per SM (the tensor memory is sized for one)");
     static_assert(NT % 16 == 0 && 2 * NT <= (int)tm::kAccCols, "accumulator columns");
@@ -518,16 +521,78 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---- thread-block clusters: split K between the CTAs of a cluster and sum
+// the partial accumulators in the first CTA's shared memory
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kPollSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+// wait_or_abort for a barrier that threads of the other CTA of the cluster
+// arrive on (their writes before the arrival are visible after it)
+__device__ __forceinline__ bool wait_or_abort_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_test_wait_cluster(bar, parity)) return true;
+    for (uint32_t i = 0; i < kPollLimit; ++i) {
+        if (*abort_flag) return false;
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+    }
+    record_timeout(abort_flag);
+    return false;
+}
+// The address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Every thread of every CTA of the cluster.  All paths through the kernel
+// reach each call (every wait before it is bounded).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Stages [s0, s1) of a tile's S that CTA `rank` of a cs-CTA cluster takes.
+__device__ __forceinline__ void stage_range(int S, int rank, int cs, int& s0, int& s1) {
+    s0 = (rank * S) / cs;
+    s1 = ((rank + 1) * S) / cs;
+}
+
 // A TMA producer that fills each ring slot with BOXES boxes (box b at
-// slot + b·box_stride, all completing on the slot's barrier).
+// slot + b·box_stride, all completing on the slot's barrier), over the tiles
+// tile0, tile0 + tstep, … and stages [s0, s1) of each (this CTA's share).
 template <int S, int BOXES, int ROWS, int NT, typename Coord>
 __device__ void tma_producer_n(uint8_t* ring, uint32_t slot_bytes, uint32_t box_stride, uint32_t expect_bytes,
                                uint64_t* full, uint64_t* empty, const GemmParams& P, volatile int* abort_flag,
-                               Coord coord) {
+                               int tile0, int tstep, int rank, Coord coord) {
     int it = 0;
-    for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+    for (int tile = tile0; tile < P.tiles; tile += tstep) {
         const TileRef tr = locate<NT, ROWS>(P, tile);
-        for (int st = 0; st < tr.kblocks; ++st, ++it) {
+        int s0, s1;
+        stage_range(tr.kblocks, rank, P.cs, s0, s1);
+        for (int st = s0; st < s1; ++st, ++it) {
             const int s = it % S;
             if (it >= S && !wait_or_abort(smem_addr(&empty[s]), ((it / S) - 1) & 1, abort_flag)) goto drain;
             mbar_arrive_expect_tx(smem_addr(&full[s]), expect_bytes);
@@ -555,14 +620,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
     uint8_t* ringB = ringW + (size_t)SW * C::kWBytes;
     // A stage s (expander warps) and x̃ stage s (TMA) complete one barrier and
     // are released by one MMA commit (a commit costs the tensor pipe ~300 cycles)
-    uint64_t* stageReady = reinterpret_cast<uint64_t*>(ringB + (size_t)SB * C::kBBytes);
+    int* red_buf = reinterpret_cast<int*>(ringB + (size_t)SB * C::kBBytes);  // [128][kRedStride]: the partner's partial
+    uint64_t* stageReady = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red_buf) + C::kRedBytes);
     uint64_t* stageFree = stageReady + SA;
     uint64_t* fullW = stageFree + SA;
     uint64_t* emptyW = fullW + SW;
     uint64_t* accFull = emptyW + SW;    // [2]
     uint64_t* accEmpty = accFull + 2;   // [2]
     uint64_t* onesReady = accEmpty + 2; // [2]
-    uint64_t* drain = onesReady + 2;    // [1]
+    uint64_t* partsIn = onesReady + 2;  // first CTA of a cluster: the second CTA's partial is in red_buf
+    uint64_t* bufFree = partsIn + 1;    // second CTA: the first one has read red_buf
+    uint64_t* drain = bufFree + 1;      // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* ones_sum = reinterpret_cast<int*>(tmem_slot + 4);  // [2][NT]: Σ x̃ of each token of the tile
@@ -585,6 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
             mbar_init(smem_addr(&accEmpty[b]), kEpiWarps);
             mbar_init(smem_addr(&onesReady[b]), 1);
         }
+        mbar_init(smem_addr(partsIn), kEpiWarps * 32);
+        mbar_init(smem_addr(bufFree), kEpiWarps * 32);
         mbar_init(smem_addr(drain), 1);
         *abort_flag = 0;
     }
@@ -598,13 +668,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_d = *tmem_slot;
+    // cluster of cs CTAs (1 or 2): cluster cl takes tiles cl, cl + ncl, …; CTA
+    // `rank` of it takes stages [rank·S/cs, (rank+1)·S/cs) of each
+    const int cs = P.cs;
+    const int rank = (int)(blockIdx.x % (unsigned)cs);
+    const int cl = (int)(blockIdx.x / (unsigned)cs), ncl = (int)(gridDim.x / (unsigned)cs);
+    if (cs > 1) cluster_sync_all();  // the partner's barriers are initialised before any remote arrive
 
     if (warp == kWarpTmaX) {
         // ---- x̃: four 128-byte boxes per stage (written by the preceding kernel under PDL)
         if (lane == 0) {
             griddep_wait();
             tma_producer_n<SB, 4, tm::kRows, NT>(ringB, C::kBBytes, NT * kKB, C::kBBytes, stageReady, stageFree, P, abort_flag,
-                                                 [&](const TileRef& tr, int st, int b, int& x, int& y) {
+                                                 cl, ncl, rank, [&](const TileRef& tr, int st, int b, int& x, int& y) {
                                                      x = st * tm::kKS + b * kKB;
                                                      y = tr.m0;
                                                      return &P.xmap[tr.p];
@@ -614,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
         // ---- packed codes: 127 rows × 128 B per stage (128-byte swizzle)
         if (lane == 0)
             tma_producer_n<SW, 1, tm::kRows, NT>(ringW, C::kWBytes, 0, C::kWBox, fullW, emptyW, P, abort_flag,
-                                                 [&](const TileRef& tr, int st, int, int& x, int& y) {
+                                                 cl, ncl, rank, [&](const TileRef& tr, int st, int, int& x, int& y) {
                                                      x = st * tm::kWS;
                                                      y = tr.n0;
                                                      return &P.wmap[tr.p];
@@ -624,14 +700,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc_u8s8<NT>();
             int it = 0, j = 0;
-            for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
-                const int stages = locate<NT, tm::kRows>(P, tile).kblocks;
+            for (int tile = cl; tile < P.tiles; tile += ncl, ++j) {
+                int s0, s1;
+                stage_range(locate<NT, tm::kRows>(P, tile).kblocks, rank, cs, s0, s1);
                 const int b = j & 1;
                 if (j >= 2 && !wait_or_abort(smem_addr(&accEmpty[b]), ((j >> 1) - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_d + (uint32_t)(b * NT);
                 bool ok = true;
-                for (int st = 0; st < stages; ++st, ++it) {
+                for (int st = s0; st < s1; ++st, ++it) {
                     const int sa = it % SA;
                     if (!(ok = wait_or_abort(smem_addr(&stageReady[sa]), (it / SA) & 1, abort_flag))) break;
                     tc_fence_after();
@@ -640,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
 #pragma unroll
                     for (int k = 0; k < tm::kKS / 32; ++k)
                         mma_i8_ta(d, a_col + 8u * k, smem_desc_sw128(b_addr + (k >> 2) * (NT * kKB) + 32 * (k & 3)),
-                                  idesc, (st > 0 || k > 0) ? 1u : 0u);
+                                  idesc, (st > s0 || k > 0) ? 1u : 0u);
                     mma_commit(smem_addr(&stageFree[sa]));
                 }
                 if (!ok) break;
@@ -658,10 +735,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
         // row t's 128 bytes, chunk j stored at chunk j ^ (t & 7) (128-byte swizzle)
         const uint32_t w_row = (uint32_t)t * tm::kWS;
         int it = 0;
-        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
-            const int stages = locate<NT, tm::kRows>(P, tile).kblocks;
+        for (int tile = cl; tile < P.tiles; tile += ncl) {
+            int s0, s1;
+            stage_range(locate<NT, tm::kRows>(P, tile).kblocks, rank, cs, s0, s1);
             bool ok = true;
-            for (int st = 0; st < stages; ++st, ++it) {
+            for (int st = s0; st < s1; ++st, ++it) {
                 const int sw = it % SW, sa = it % SA;
                 if (!(ok = wait_or_abort(smem_addr(&fullW[sw]), (it / SW) & 1, abort_flag))) break;
                 uint32_t wd[32];
@@ -702,13 +780,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
             if (!ok) break;
         }
     } else {
-        // ---- epilogue: tile row t; acc = D[t] - D[127]
+        // ---- epilogue: tile row t; acc = D[t] - D[127] (with two CTAs per
+        // cluster: the second sends its partial D to the first, which adds it)
         griddep_wait();
         const int q = warp & 3;
         const int t = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const uint32_t red_row = smem_addr(red_buf + t * C::kRedStride);
         int j = 0;
-        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+        for (int tile = cl; tile < P.tiles; tile += ncl, ++j) {
+            const int b = j & 1;
+            if (!wait_or_abort(smem_addr(&accFull[b]), (j >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            if (rank == 1) {
+                // second CTA: once the first has read the previous partial, store
+                // this row's partial into its buffer and tell it
+                if (j > 0 && !wait_or_abort_cluster(smem_addr(bufFree), (j - 1) & 1, abort_flag)) break;
+                const uint32_t dst = mapa_shared(red_row, 0);
+#pragma unroll 1
+                for (int c = 0; c < NT; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c), r);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        st_cluster_v4(dst + 4u * (uint32_t)(c + 4 * v), r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                }
+                mbar_arrive_remote(mapa_shared(smem_addr(partsIn), 0));
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive1(smem_addr(&accEmpty[b]));
+                continue;
+            }
+            const bool add_part = cs > 1;
+            if (add_part && !wait_or_abort_cluster(smem_addr(partsIn), j & 1, abort_flag)) break;
             const TileRef tr = locate<NT, tm::kRows>(P, tile);
             const int M = P.p[tr.p].M, N = P.p[tr.p].N;
             const float* beta_p = P.p[tr.p].beta;
@@ -716,13 +820,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
             float* y = P.p[tr.p].y;
             int32_t* acc_out = P.p[tr.p].acc_out;
             const float alpha = *P.p[tr.p].alpha;
-            const int b = j & 1;
             const int m0 = tr.m0;
             const int row = tr.n0 + t;
             const bool row_ok = t < tm::kRows && row < N;
             const float bias = (row_ok && bias_p) ? bias_p[row] : 0.0f;
-            if (!wait_or_abort(smem_addr(&accFull[b]), (j >> 1) & 1, abort_flag)) break;
-            tc_fence_after();
             int* ones_b = ones_sum + b * NT;
             if (q == 3) {
                 // lane 31 of this warp reads TMEM lane 127: publish Σ x̃ of every token
@@ -732,7 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
                     tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c), r);
                     if (lane == 31) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) ones_b[c + i] = (int)r[i];
+                        for (int i = 0; i < 16; ++i) ones_b[c + i] = (int)r[i] + (add_part ? red_buf[127 * C::kRedStride + c + i] : 0);
                     }
                 }
                 __syncwarp();
@@ -747,6 +848,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
                 for (int h = 0; h < 2 && c0 + 16 * h < NT; ++h) {
                     uint32_t r[16];
                     tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c0 + 16 * h), r);
+                    if (add_part) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const uint4 u = lds128(red_row + 4u * (uint32_t)(c0 + 16 * h + 4 * v));
+                            r[4 * v] += u.x;
+                            r[4 * v + 1] += u.y;
+                            r[4 * v + 2] += u.z;
+                            r[4 * v + 3] += u.w;
+                        }
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float sc = __shfl_sync(0xffffffffu, my_scale, 16 * h + i);
@@ -761,6 +872,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
                     }
                 }
             }
+            // red_buf row t has been read: the second CTA may overwrite it
+            if (add_part) mbar_arrive_remote(mapa_shared(smem_addr(bufFree), 1));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive1(smem_addr(&accEmpty[b]));
@@ -768,6 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tm_kernel(const __grid_const
     }
     tc_fence_before();
     __syncthreads();
+    // no CTA leaves while its partner may still write to or arrive in its shared memory
+    if (cs > 1) cluster_sync_all();
     if (warp == kWarpMma) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(tm::kTmemCols));
@@ -805,6 +920,56 @@ cudaError_t encode_u8(CUtensorMap* map, const void* base, int64_t cols, int64_t 
                      CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The longest CTA's work, in stages (+1 per tile for the partial-sum exchange
+// when cs = 2), with tiles dealt round-robin to `clusters` clusters of cs CTAs
+// that split every tile's K stages.
+int64_t split_makespan(const GemmParams& P, int clusters, int cs) {
+    int64_t worst = 0;
+    for (int c = 0; c < clusters; ++c) {
+        int64_t sum = 0;
+        int p = 0;
+        for (int tile = c; tile < P.tiles; tile += clusters) {
+            while (p + 1 < P.count && tile >= P.p[p + 1].tile_begin) ++p;
+            sum += (P.p[p].kblocks + cs - 1) / cs + (cs > 1 ? 1 : 0);
+        }
+        worst = std::max(worst, sum);
+    }
+    return worst;
+}
+
+// Clusters of two CTAs of gemm_tm_kernel<NT> (one per SM) that the device
+// can hold at once, cached per device.
+template <int NT>
+cudaError_t cluster_pairs(const void* kernel, int smem, int* out) {
+    static std::mutex mu;
+    static int cache[64] = {};  // per device: the count + 1 (0: not yet asked)
+    int devi = 0;
+    cudaError_t err = cudaGetDevice(&devi);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(mu);
+    if (devi < 64 && cache[devi] > 0) {
+        *out = cache[devi] - 1;
+        return cudaSuccess;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    err = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+    if (err != cudaSuccess) return err;
+    if (devi < 64) cache[devi] = n + 1;
+    *out = n;
+    return cudaSuccess;
 }
 
 // Launches gemm_tc_kernel<NT> (TMEM_A = false: tiles of 128 rows, K blocks of
@@ -863,6 +1028,7 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
         tiles += q.tiles_m * (int)((pr.N + kRows - 1) / kRows);
     }
     P.tiles = tiles;
+    P.cs = 1;
 
     // the opt-in is per device: set once on each device that launches the kernel
     err = set_max_dynamic_smem(kernel, (int)kSmem);
@@ -872,11 +1038,33 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if constexpr (TMEM_A) {
+        // Split every tile's K between the two CTAs of a cluster when that
+        // shortens the longest CTA: few tiles for the SMs, long K.
+        int ncl2 = 0;
+        if (cluster_pairs<NT>(kernel, (int)kSmem, &ncl2) == cudaSuccess && ncl2 > 0) {
+            int stages_min = INT32_MAX;
+            for (int i = 0; i < count; ++i) stages_min = std::min(stages_min, P.p[i].kblocks);
+            if (stages_min >= 2) {
+                const int64_t one = split_makespan(P, std::min(tiles, dev.sm_count), 1);
+                const int64_t two = split_makespan(P, std::min(tiles, ncl2), 2);
+                if (two < one) {
+                    P.cs = 2;
+                    cfg.gridDim = dim3((unsigned)(2 * std::min(tiles, ncl2)));
+                    attr[1].id = cudaLaunchAttributeClusterDimension;
+                    attr[1].val.clusterDim.x = 2;
+                    attr[1].val.clusterDim.y = 1;
+                    attr[1].val.clusterDim.z = 1;
+                    cfg.numAttrs = 2;
+                }
+            }
+        }
+    }
     void* args[] = {&P};
     return cudaLaunchKernelExC(&cfg, kernel, args);
 }

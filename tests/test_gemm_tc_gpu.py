@@ -52,6 +52,15 @@ def test_gemm_few_tokens_many_stages_and_tiles(M):
     run_case(M, 2560 + 64, 127 * 4 + 1, seed=650 + M, bias=(M == 24))
 
 
+@pytest.mark.parametrize("M,K,N", [(16, 512 * 6 + 64, 300), (64, 512 * 6 + 64, 300), (16, 4096, 127 * 150),
+                                   (40, 512 * 5 + 64, 127 * 4 + 1)])
+def test_gemm_few_tokens_split_k_pairs(M, K, N):
+    """Few tiles with long K: the two CTAs of a cluster each take half of
+    every tile's K stages (an odd stage count; three tiles per cluster with
+    150 tiles) and the first adds the second's partial accumulators."""
+    run_case(M, K, N, seed=660 + M + K % 97)
+
+
 def test_gemm_prefill_shape_small_rows():
     """2048 tokens (the prefill token count) on a few hundred rows."""
     run_case(2048, 1024, 256, seed=800, dtype="f32")
