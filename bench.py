@@ -860,8 +860,9 @@ def run_scales(args, world, local_rank):
                      "replicas": replicas, "clocks": clocks}
         del reps, arrs
     return {"metric": "decode GB/s with one alpha per row / per 128-block",
-            "workload": "7B decode layer set, M=1, bf16 x with outliers; bitlinear_linear_scaled (act quant + scaled "
-                        "GEMV, 2 launches per step)", **out}
+            "workload": "7B decode layer set, M=1, bf16 x with outliers; bitlinear_linear_scaled: one alpha per row "
+                        "runs as one launch (the streaming GEMV quantises x in its prologue, the epilogue applies "
+                        "the row's alpha); per 128-block as act quant + scaled GEMV (2 launches per step)", **out}
 
 
 # ----------------------------------------------------------------------------- 4-bit activation leg
@@ -906,7 +907,8 @@ def run_a4(args, world, local_rank):
     peak = float(load_peaks()[0]["hbm_gbs"])
     gbs = bps / (ms * 1e-3) / 1e9
     return {"metric": "decode GB/s with 4-bit activations",
-            "workload": "7B decode layer set, M=1, bf16 x with outliers; bitlinear_linear_a4 (2 launches per step)",
+            "workload": "7B decode layer set, M=1, bf16 x with outliers; bitlinear_linear_a4 (one launch per step: "
+                        "the streaming GEMV quantises x to 4 bits in its prologue)",
             "us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
             "bytes_per_step": bps, "steps": K, "replicas": replicas, "clocks": clocks}
 

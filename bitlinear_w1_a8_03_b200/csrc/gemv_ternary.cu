@@ -1359,6 +1359,22 @@ cudaError_t launch_generic(const bitlinear_forward_problem* problems, int count,
 
 }  // namespace
 
+// Three or four tokens on large weights: the tensor-core GEMM (x̃ quantised by
+// its own launch) is faster than the streaming GEMV, whose dp4a work grows
+// with the token count (100B-shaped matrices at four tokens: 33 against 46 µs).
+constexpr int64_t kGemmFewTokenMinBytes = 8 << 20;
+
+bool prefer_gemm_few_tokens(const bitlinear_forward_problem* problems, int count, int64_t max_m) {
+    if (max_m < 3 || max_m > kGemvMaxTokens) return false;
+    int64_t bytes = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_forward_problem& s = problems[i];
+        if (s.K % 16 != 0 || (reinterpret_cast<uintptr_t>(s.x_q) & 15) != 0 || !gemm_tc_supported(s)) return false;
+        bytes += s.N * (int64_t)bitlinear_packed_row_bytes(s.K);
+    }
+    return bytes >= kGemmFewTokenMinBytes;
+}
+
 cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl,
                            bool alpha_rows) {
     DeviceInfo dev;
@@ -1376,7 +1392,7 @@ cudaError_t launch_forward(const bitlinear_forward_problem* problems, int count,
         if (max_m == 2) return launch_stream<2>(problems, count, dev, stream, pdl, nullptr, false, nullptr, false, true);
         return launch_stream<4>(problems, count, dev, stream, pdl, nullptr, false, nullptr, false, true);
     }
-    if (max_m > kGemvMaxTokens) {
+    if (max_m > kGemvMaxTokens || (!alpha_rows && prefer_gemm_few_tokens(problems, count, max_m))) {
         // many tokens: the int8 tensor cores, all problems in one launch
         bool tc = fast;
         for (int i = 0; i < count; ++i) tc = tc && gemm_tc_supported(problems[i]);
@@ -1411,6 +1427,8 @@ cudaError_t launch_linear_fused(const bitlinear_forward_problem* problems, const
             return cudaSuccess;
         if (s.M > max_m) max_m = s.M;
     }
+    // three or four tokens on large weights: act quant + tensor-core GEMM instead
+    if (!always && !alpha_rows && !a4 && prefer_gemm_few_tokens(problems, count, max_m)) return cudaSuccess;
     const bool bf16 = dtype == BL_BF16;
     if (max_m == 1)
         return launch_stream<1>(problems, count, dev, stream, pdl, in, bf16, launched, always, alpha_rows, a4);

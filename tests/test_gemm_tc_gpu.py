@@ -61,6 +61,38 @@ def test_gemm_few_tokens_split_k_pairs(M, K, N):
     run_case(M, K, N, seed=660 + M + K % 97)
 
 
+@pytest.mark.parametrize("M", [3, 4])
+def test_gemm_three_four_tokens_large_weights(M):
+    """Three or four tokens on 8 MB of weights go to the tensor-core GEMM
+    rather than the streaming GEMV (checked: the same results)."""
+    run_case(M, 4096, 8192, seed=690 + M)
+
+
+@pytest.mark.parametrize("M", [3, 4])
+def test_linear_grouped_three_four_tokens_large_weights(M, fusion):
+    """bitlinear_linear_grouped at three or four tokens over 8 MB of weights:
+    act quant + GEMM by default, the fused GEMV when fusion is forced on."""
+    K, N = 4096, 8192
+    W = synth.weights(710 + M, N, K, 0.02)
+    x = synth.activations(720 + M, M, K, outliers=True)
+    Wd, Wo = as_input(W, "f32")
+    packed, alpha = bl.bitlinear_quantize_weights(Wd)
+    _, a_ref, codes = oracle.quantize_weights(Wo)
+    xd, xo = as_input(x, "bf16")
+    p = dict(x=xd, x_q=torch.empty((M, K), dtype=torch.int8, device="cuda"),
+             beta=torch.empty(M, dtype=torch.float32, device="cuda"), W_packed=packed, alpha=alpha, N=N,
+             y=torch.empty((M, N), dtype=torch.float32, device="cuda"),
+             acc_out=torch.empty((M, N), dtype=torch.int32, device="cuda"))
+    bl.bitlinear_linear_grouped([p])
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    xq_r, beta_r, acc_r, y_r = oracle.forward(xo, codes, a_ref, threads=8)
+    assert np.array_equal(np_(p["x_q"]), xq_r) and np.array_equal(np_(p["beta"]), beta_r)
+    assert np.array_equal(np_(p["acc_out"]), acc_r)
+    err = np.abs(np_(p["y"]).astype(np.float64) - y_r)
+    assert np.all(err <= 1e-5 * np.abs(y_r) + 1e-37)
+
+
 def test_gemm_prefill_shape_small_rows():
     """2048 tokens (the prefill token count) on a few hundred rows."""
     run_case(2048, 1024, 256, seed=800, dtype="f32")
