@@ -690,7 +690,8 @@ def run_batched_100b(args, world, local_rank):
             gbs = bps / (ms * 1e-3) / 1e9
             per_m[f"M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
                               "frac": round(gbs / peak, 4), "pct_of_8TBps": round(100 * gbs / 8000.0, 2),
-                              "kernel": "gemv_stream_kernel (CUDA cores)" if M <= 4 else "gemm_tc_kernel (tcgen05 i8)"}
+                              "kernel": ("gemv_stream_kernel (CUDA cores)" if M <= 2 else
+                                         "gemm_tm_kernel (tcgen05 i8, codes expanded into tensor memory)")}
         out[f"K{K}_N{N}"] = {"weight_bytes": wbytes, "replicas": replicas, **per_m}
         del packed, p0
     with torch.cuda.stream(stream):
