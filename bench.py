@@ -316,58 +316,49 @@ def run_native(args, rank, world, local_rank):
     stream.synchronize()
     clocks = sampler.stop()
 
-    # end to end through the public binding: every step copies its inputs from
-    # pinned host memory and reads its results back, double-buffered the way a
-    # serving loop would run it: step i+1's upload overlaps step i's kernels,
-    # step i's download overlaps step i+1's kernels (two copy streams, events)
+    # end to end through the C ABI with host buffers: every step is one
+    # bitlinear_linear_grouped_host call that copies the step's inputs from
+    # pinned host memory, runs the linear and copies the results back (one
+    # merged copy each way). Steps alternate between two streams with their own
+    # buffers, so one step's copies overlap the other's kernel.
     x_pinned = [torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory() for _ in range(2)]
     y_pinned = [torch.empty(y_dev.numel(), dtype=torch.float32).pin_memory() for _ in range(2)]
     x_dev2 = [x_dev, torch.empty_like(x_dev)]
     y_dev2 = [y_dev, torch.empty_like(y_dev)]
+    xq2 = [xq, [torch.empty_like(t) for t in xq]]
+    beta2 = [beta, [torch.empty_like(t) for t in beta]]
 
     def e2e_problems(bi, r):
-        out, ox, oy = [], 0, 0
+        out, io, ox, oy = [], [], 0, 0
         for i, s in enumerate(specs):
-            out.append(dict(x=x_dev2[bi][ox:ox + s.M * s.K].view(s.M, s.K), x_q=xq[i], beta=beta[i],
+            out.append(dict(x=x_dev2[bi][ox:ox + s.M * s.K].view(s.M, s.K), x_q=xq2[bi][i], beta=beta2[bi][i],
                             W_packed=packed[r][i], alpha=alphas[i], N=s.N, y=y_dev2[bi][oy:oy + s.M * s.N].view(s.M, s.N)))
+            io.append((x_pinned[bi][ox:ox + s.M * s.K], y_pinned[bi][oy:oy + s.M * s.N]))
             ox += s.M * s.K
             oy += s.M * s.N
-        return out
-    e2e_arr = [[bl.make_linear_problems(e2e_problems(bi, r)) for r in range(replicas)] for bi in range(2)]
-    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("h2d", "done", "d2h")}
+        return bl.make_linear_problems(out), bl.make_host_io(io)
+    e2e_arr = [[e2e_problems(bi, r) for r in range(replicas)] for bi in range(2)]
+    e2e_streams = [torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)]
 
     def e2e_step(i):
         bi = i % 2
-        with torch.cuda.stream(up):
-            if i >= 2:
-                up.wait_event(ev["done"][bi])  # step i-2 finished reading this input buffer
-            x_dev2[bi].copy_(x_pinned[bi], non_blocking=True)
-            ev["h2d"][bi].record(up)
-        stream.wait_event(ev["h2d"][bi])
-        if i >= 2:
-            stream.wait_event(ev["d2h"][bi])  # step i-2's results left this output buffer
-        bl.check(L.bitlinear_linear_grouped(e2e_arr[bi][i % replicas], nprob, bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
-                                            sh), "linear")
-        ev["done"][bi].record(stream)
-        with torch.cuda.stream(down):
-            down.wait_event(ev["done"][bi])
-            y_pinned[bi].copy_(y_dev2[bi], non_blocking=True)
-            ev["d2h"][bi].record(down)
+        arr, io = e2e_arr[bi][i % replicas]
+        bl.check(L.bitlinear_linear_grouped_host(arr, io, nprob, bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
+                                                 e2e_streams[bi].cuda_stream), "linear_host")
 
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    for i in range(3):
+    for i in range(4):
         e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    e0.record(stream)
+    e0.record(e2e_streams[0])
+    e2e_streams[1].wait_event(e0)
     for i in range(K):
         e2e_step(i)
-    stream.wait_stream(up)
-    stream.wait_stream(down)
-    e1.record(stream)
+    e2e_streams[0].wait_stream(e2e_streams[1])
+    e1.record(e2e_streams[0])
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
@@ -423,8 +414,9 @@ def run_native(args, rank, world, local_rank):
             "unit": "GB/s",
             "h2d_bytes_per_step": int(x_host.nbytes),
             "d2h_bytes_per_step": int(y_dev.numel() * 4),
-            "how": "public binding per step: pinned x -> device, bitlinear_linear_grouped, y -> pinned host; "
-                   "double-buffered on two copy streams so copies overlap the neighbouring steps' kernels",
+            "how": "per step one C-ABI call with host buffers, bitlinear_linear_grouped_host: pinned x -> device "
+                   "(one merged copy), the grouped linear, y -> pinned host (one merged copy); steps alternate "
+                   "between two streams with their own buffers",
         },
         "gpu_launches": K,
         "clocks": clocks,

@@ -52,6 +52,10 @@ class ForwardProblem(ctypes.Structure):
                 ("K", ctypes.c_int64)]
 
 
+class HostIO(ctypes.Structure):
+    _fields_ = [("x_host", ctypes.c_void_p), ("y_host", ctypes.c_void_p)]
+
+
 class LinearProblem(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("x_q", ctypes.c_void_p), ("beta", ctypes.c_void_p),
                 ("W_packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("bias", ctypes.c_void_p),
@@ -93,6 +97,8 @@ def lib():
             L.bitlinear_forward_grouped.argtypes = [ctypes.POINTER(ForwardProblem), i32, p]
             L.bitlinear_linear.argtypes = [p, i32, i64, i64, p, p, i64, p, p, p, p, p, p]
             L.bitlinear_linear_grouped.argtypes = [ctypes.POINTER(LinearProblem), i32, i32, ctypes.c_uint32, p]
+            L.bitlinear_linear_grouped_host.argtypes = [ctypes.POINTER(LinearProblem), ctypes.POINTER(HostIO), i32,
+                                                        i32, ctypes.c_uint32, p]
             L.bitlinear_linear_block.argtypes = [ctypes.POINTER(ActSumProblem), i32, ctypes.POINTER(ForwardProblem), i32,
                                                  ctypes.c_uint32, p]
             L.bitlinear_hadamard_block.argtypes = [i64]
@@ -259,6 +265,22 @@ def make_linear_problems(problems):
         arr[i] = LinearProblem(_ptr(p["x"]), _ptr(p["x_q"]), _ptr(p["beta"]), _ptr(p["W_packed"]), _ptr(p["alpha"]),
                                _ptr(p.get("bias")), _ptr(p["y"]), _ptr(p.get("acc_out")), M, p["N"], K)
     return arr
+
+
+def make_host_io(pairs):
+    """ctypes array for bitlinear_linear_grouped_host from (x_host, y_host)
+    pairs of CPU tensors (pinned for asynchronous copies)."""
+    arr = (HostIO * len(pairs))()
+    for i, (xh, yh) in enumerate(pairs):
+        arr[i] = HostIO(xh.data_ptr(), yh.data_ptr())
+    return arr
+
+
+def bitlinear_linear_grouped_host(problems, io, dtype_code: int, flags: int = 0, stream=None):
+    """bitlinear_linear_grouped with x copied from and y copied to host memory
+    on the stream (ctypes arrays from make_linear_problems and make_host_io)."""
+    check(lib().bitlinear_linear_grouped_host(problems, io, len(problems), dtype_code, flags, _stream(stream)),
+          "bitlinear_linear_grouped_host")
 
 
 def bitlinear_linear_grouped(problems, dtype_code: int | None = None, flags: int = 0, stream=None):

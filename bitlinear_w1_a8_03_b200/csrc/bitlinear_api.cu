@@ -261,6 +261,77 @@ bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_problem* proble
     return from_cuda(bl::launch_forward(fwd, count, s, true));
 }
 
+// Copies `count` (dst[i], src[i], bytes[i]) on `stream`, one cudaMemcpyAsync
+// per run of pairs that are adjacent on both sides, skipping a pair equal to an
+// earlier one (problems sharing an input).
+static cudaError_t copy_runs(void* const* dst, const void* const* src, const size_t* bytes, int count,
+                             cudaMemcpyKind kind, cudaStream_t s) {
+    int i = 0;
+    while (i < count) {
+        bool repeat = false;
+        for (int j = 0; j < i && !repeat; ++j) repeat = dst[j] == dst[i] && src[j] == src[i] && bytes[j] == bytes[i];
+        if (repeat) {
+            ++i;
+            continue;
+        }
+        size_t run = bytes[i];
+        int k = i + 1;
+        while (k < count && static_cast<const char*>(dst[i]) + run == dst[k] &&
+               static_cast<const char*>(src[i]) + run == src[k]) {
+            run += bytes[k];
+            ++k;
+        }
+        cudaError_t err = cudaMemcpyAsync(dst[i], src[i], run, kind, s);
+        if (err != cudaSuccess) return err;
+        i = k;
+    }
+    return cudaSuccess;
+}
+
+bitlinear_status bitlinear_linear_grouped_host(const bitlinear_linear_problem* problems, const bitlinear_host_io* io,
+                                               int count, bitlinear_dtype dtype, uint32_t flags,
+                                               bitlinear_stream_t stream) {
+    if (!problems || !io) return BL_ERR_NULL;
+    if (count < 1 || count > BITLINEAR_MAX_GROUP) return BL_ERR_COUNT;
+    if (!valid_dtype(dtype)) return BL_ERR_DTYPE;
+    if (flags & ~(uint32_t)(BL_LINEAR_WEIGHTS_STATIC | BL_LINEAR_HADAMARD)) return BL_ERR_FLAGS;
+    void* xd[BITLINEAR_MAX_GROUP];
+    const void* xh[BITLINEAR_MAX_GROUP];
+    void* yh[BITLINEAR_MAX_GROUP];
+    const void* yd[BITLINEAR_MAX_GROUP];
+    size_t xb[BITLINEAR_MAX_GROUP], yb[BITLINEAR_MAX_GROUP];
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) {
+        const bitlinear_linear_problem& q = problems[i];
+        if (!io[i].x_host || !io[i].y_host) return BL_ERR_NULL;
+        // the shapes are checked by the grouped call below; the copy sizes are
+        // only formed once M, N, K are known to be in range
+        const bitlinear_act_problem a{q.x, q.x_q, q.beta, q.M, q.K};
+        const bitlinear_forward_problem f{q.x_q, q.beta, q.W_packed, q.alpha, q.bias, q.y, q.acc_out, q.M, q.N, q.K};
+        bitlinear_status st = check_act(a);
+        if (st == BL_OK) st = check_forward(f);
+        if (st != BL_OK) return st;
+        if (misaligned(q.x, dtype == BL_F32 ? 4 : 2)) return BL_ERR_ALIGN;
+        if ((flags & BL_LINEAR_HADAMARD) && bitlinear_hadamard_block(q.K) < 2) return BL_ERR_SHAPE;
+        rows += q.M;
+        xd[i] = const_cast<void*>(q.x);
+        xh[i] = io[i].x_host;
+        xb[i] = (size_t)q.M * (size_t)q.K * (dtype == BL_F32 ? 4 : 2);
+        yd[i] = q.y;
+        yh[i] = io[i].y_host;
+        yb[i] = (size_t)q.M * (size_t)q.N * 4;
+    }
+    if (rows >= kMaxRows) return BL_ERR_SHAPE;
+    bitlinear_status st = check_device();
+    if (st != BL_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = from_cuda(copy_runs(xd, xh, xb, count, cudaMemcpyHostToDevice, s));
+    if (st != BL_OK) return st;
+    st = bitlinear_linear_grouped(problems, count, dtype, flags, stream);
+    if (st != BL_OK) return st;
+    return from_cuda(copy_runs(yh, yd, yb, count, cudaMemcpyDeviceToHost, s));
+}
+
 bitlinear_status bitlinear_linear_block(const bitlinear_act_sum_problem* acts, int n_acts,
                                         const bitlinear_forward_problem* fwd, int n_fwd, uint32_t flags,
                                         bitlinear_stream_t stream) {

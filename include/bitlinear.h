@@ -250,6 +250,32 @@ BITLINEAR_API bitlinear_status bitlinear_linear_grouped(const bitlinear_linear_p
                                                         bitlinear_dtype dtype, uint32_t flags,
                                                         bitlinear_stream_t stream);
 
+/* Host-side input and output of one problem of bitlinear_linear_grouped_host. */
+typedef struct bitlinear_host_io {
+    const void* x_host; /* [M][K] `dtype`, HOST memory: copied into the problem's device x */
+    float* y_host;      /* [M][N] float32, HOST memory: receives the problem's device y */
+} bitlinear_host_io;
+
+/* bitlinear_linear_grouped with the inputs and outputs in HOST memory (the
+ * inference path of "1.58-bit 大模型极限量化实战", chenxutan.com/d/5049.html
+ * §4.2, seen from a host program): enqueues on `stream` the copy of every
+ * io[i].x_host into problems[i].x, the grouped linear, and the copy of every
+ * problems[i].y into io[i].y_host.  The device buffers of `problems` are used
+ * as by bitlinear_linear_grouped (x is overwritten by the copy).  Copies of
+ * problems whose host and device buffers are both adjacent are merged into one
+ * cudaMemcpyAsync, and a problem whose x (and x_host) repeats an earlier
+ * problem's is copied once.  Host memory should be page-locked: with pageable
+ * memory CUDA performs the copies synchronously.  The call returns once the
+ * work is enqueued; y_host is valid after the stream reaches the end of it,
+ * and neither host buffer may be modified before then.  `io` is a HOST array
+ * of `count` entries.
+ * Errors: as bitlinear_linear_grouped, plus BL_ERR_NULL (io or a host pointer
+ * NULL) and BL_ERR_CUDA from a copy (work already enqueued stays enqueued). */
+BITLINEAR_API bitlinear_status bitlinear_linear_grouped_host(const bitlinear_linear_problem* problems,
+                                                             const bitlinear_host_io* io, int count,
+                                                             bitlinear_dtype dtype, uint32_t flags,
+                                                             bitlinear_stream_t stream);
+
 /* One input of bitlinear_linear_block: x = a, or x = a + b added element-wise
  * in binary32 (round to nearest) when b is not NULL — the residual addition
  * that stays in floating point between BitLinear layers while every BitLinear

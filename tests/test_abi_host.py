@@ -210,3 +210,27 @@ def test_train_argument_errors(L):
     assert t(P, 0, 8, 64, None, 0, 1, P, P, P, P, P, P, ws, None) == NULL
     assert t(P, 0, 8, 64, P, 0, 0, P, P, P, P, P, P, ws, None) == SHAPE
     assert t(P, 0, 8, 64, P, 0, 1, P, P, P, P, P, P, 0, None) == WORKSPACE
+
+
+def test_linear_grouped_host_argument_errors(L):
+    """bitlinear_linear_grouped_host checks every argument before its first
+    copy: nothing is enqueued for a bad call."""
+    assert ctypes.sizeof(bl.HostIO) == 2 * 8
+    lin = (bl.LinearProblem * 1)()
+    io = (bl.HostIO * 1)()
+    h = L.bitlinear_linear_grouped_host
+    lin[0] = bl.LinearProblem(P, P, P, P, P, None, P, None, 1, 8, 64)
+    assert h(None, io, 1, 0, 0, None) == NULL
+    assert h(lin, None, 1, 0, 0, None) == NULL
+    assert h(lin, io, 1, 0, 0, None) == NULL            # host pointers left empty
+    io[0] = bl.HostIO(0x1000, 0x2000)
+    assert h(lin, io, 0, 0, 0, None) == COUNT
+    assert h(lin, io, 17, 0, 0, None) == COUNT
+    assert h(lin, io, 1, 7, 0, None) == DTYPE
+    assert h(lin, io, 1, 0, 4, None) == FLAGS
+    lin[0] = bl.LinearProblem(P, P, P, P, P, None, P, None, 0, 8, 64)
+    assert h(lin, io, 1, 0, 0, None) == SHAPE
+    lin[0] = bl.LinearProblem(P + 2, P, P, P, P, None, P, None, 1, 8, 64)
+    assert h(lin, io, 1, 0, 0, None) == ALIGN
+    lin[0] = bl.LinearProblem(P, P, P, P, P, None, None, None, 1, 8, 64)
+    assert h(lin, io, 1, 0, 0, None) == NULL            # device y missing

@@ -168,3 +168,56 @@ def test_prefill_grouped_three_shapes_graph():
             assert np.array_equal(np_(p["acc_out"])[:, rows], acc_r), (st, s.name)
             _check_y(np_(p["y"])[:, rows], y_r)
     del g
+
+
+def test_linear_grouped_host_7b_decode_set_two_streams():
+    """The end-to-end call the benchmark times: bitlinear_linear_grouped_host
+    copies x from pinned host memory, runs the seven 7B linears and copies y
+    back to pinned host memory.  Two steps on two streams with their own
+    buffers; problem 1 reads problem 0's input (copied once), the others lie
+    back to back (merged copies).  Every y equals the oracle's forward within
+    1e-5, and x_q, β the oracle's quantisation."""
+    specs = workloads.decode_7b_layer_set(M=1)
+    assert specs[0].K == specs[1].K
+    base = [_weights(s) for s in specs]
+    L = bl.lib()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    own = [i for i in range(len(specs)) if i != 1]
+    k_tot = sum(specs[i].K for i in own)
+    n_tot = sum(s.N for s in specs)
+    steps = []
+    for st in range(2):
+        bits = {i: synth.f32_to_bf16_bits(synth.activations(specs[i].x_seed + 500 * st, 1, specs[i].K, outliers=True))
+                for i in own}
+        x_host = torch.from_numpy(np.concatenate([bits[i].reshape(-1) for i in own]).view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+        y_host = torch.full((n_tot,), float("nan"), dtype=torch.float32).pin_memory()
+        x_dev = torch.empty(k_tot, dtype=torch.bfloat16, device="cuda")
+        y_dev = torch.empty(n_tot, dtype=torch.float32, device="cuda")
+        off, ox = {}, 0
+        for i in own:
+            off[i] = ox
+            ox += specs[i].K
+        off[1] = off[0]
+        bits[1] = bits[0]
+        probs, io, oy = [], [], 0
+        for i, s in enumerate(specs):
+            probs.append(dict(x=x_dev[off[i]:off[i] + s.K].view(1, s.K),
+                              x_q=torch.empty((1, s.K), dtype=torch.int8, device="cuda"),
+                              beta=torch.empty(1, dtype=torch.float32, device="cuda"), W_packed=base[i][0],
+                              alpha=base[i][1], N=s.N, y=y_dev[oy:oy + s.N].view(1, s.N)))
+            io.append((x_host[off[i]:off[i] + s.K], y_host[oy:oy + s.N]))
+            oy += s.N
+        arr, hio = bl.make_linear_problems(probs), bl.make_host_io(io)
+        bl.bitlinear_linear_grouped_host(arr, hio, bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC, streams[st])
+        steps.append((bits, probs, y_host))
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    for bits, probs, y_host in steps:
+        oy = 0
+        for i, s in enumerate(specs):
+            xq_r, beta_r, _, y_r = oracle.forward(bits[i].reshape(1, s.K), base[i][2], base[i][3], threads=8)
+            assert np.array_equal(np_(probs[i]["x_q"]), xq_r) and np.array_equal(np_(probs[i]["beta"]), beta_r)
+            y = y_host[oy:oy + s.N].numpy().astype(np.float64).reshape(1, s.N)
+            assert np.all(np.abs(y - y_r) <= 1e-5 * np.abs(y_r) + 1e-37), s.name
+            oy += s.N
