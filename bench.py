@@ -319,14 +319,15 @@ def run_native(args, rank, world, local_rank):
     # end to end through the C ABI with host buffers: every step is one
     # bitlinear_linear_grouped_host call that copies the step's inputs from
     # pinned host memory, runs the linear and copies the results back (one
-    # merged copy each way). Steps alternate between two streams with their own
-    # buffers, so one step's copies overlap the other's kernel.
-    x_pinned = [torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory() for _ in range(2)]
-    y_pinned = [torch.empty(y_dev.numel(), dtype=torch.float32).pin_memory() for _ in range(2)]
-    x_dev2 = [x_dev, torch.empty_like(x_dev)]
-    y_dev2 = [y_dev, torch.empty_like(y_dev)]
-    xq2 = [xq, [torch.empty_like(t) for t in xq]]
-    beta2 = [beta, [torch.empty_like(t) for t in beta]]
+    # merged copy each way). Steps rotate over three streams with their own
+    # buffers, so a step's copies overlap the other steps' kernels.
+    NB = 3
+    x_pinned = [torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory() for _ in range(NB)]
+    y_pinned = [torch.empty(y_dev.numel(), dtype=torch.float32).pin_memory() for _ in range(NB)]
+    x_dev2 = [x_dev] + [torch.empty_like(x_dev) for _ in range(NB - 1)]
+    y_dev2 = [y_dev] + [torch.empty_like(y_dev) for _ in range(NB - 1)]
+    xq2 = [xq] + [[torch.empty_like(t) for t in xq] for _ in range(NB - 1)]
+    beta2 = [beta] + [[torch.empty_like(t) for t in beta] for _ in range(NB - 1)]
 
     def e2e_problems(bi, r):
         out, io, ox, oy = [], [], 0, 0
@@ -337,11 +338,11 @@ def run_native(args, rank, world, local_rank):
             ox += s.M * s.K
             oy += s.M * s.N
         return bl.make_linear_problems(out), bl.make_host_io(io)
-    e2e_arr = [[e2e_problems(bi, r) for r in range(replicas)] for bi in range(2)]
-    e2e_streams = [torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)]
+    e2e_arr = [[e2e_problems(bi, r) for r in range(replicas)] for bi in range(NB)]
+    e2e_streams = [torch.cuda.Stream(device=dev) for _ in range(NB)]
 
     def e2e_step(i):
-        bi = i % 2
+        bi = i % NB
         arr, io = e2e_arr[bi][i % replicas]
         bl.check(L.bitlinear_linear_grouped_host(arr, io, nprob, bl.BL_BF16, bl.BL_LINEAR_WEIGHTS_STATIC,
                                                  e2e_streams[bi].cuda_stream), "linear_host")
@@ -354,10 +355,12 @@ def run_native(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     e0.record(e2e_streams[0])
-    e2e_streams[1].wait_event(e0)
+    for s_ in e2e_streams[1:]:
+        s_.wait_event(e0)
     for i in range(K):
         e2e_step(i)
-    e2e_streams[0].wait_stream(e2e_streams[1])
+    for s_ in e2e_streams[1:]:
+        e2e_streams[0].wait_stream(s_)
     e1.record(e2e_streams[0])
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -415,8 +418,8 @@ def run_native(args, rank, world, local_rank):
             "h2d_bytes_per_step": int(x_host.nbytes),
             "d2h_bytes_per_step": int(y_dev.numel() * 4),
             "how": "per step one C-ABI call with host buffers, bitlinear_linear_grouped_host: pinned x -> device "
-                   "(one merged copy), the grouped linear, y -> pinned host (one merged copy); steps alternate "
-                   "between two streams with their own buffers",
+                   "(one merged copy), the grouped linear, y -> pinned host (one merged copy); steps rotate "
+                   "over three streams with their own buffers",
         },
         "gpu_launches": K,
         "clocks": clocks,

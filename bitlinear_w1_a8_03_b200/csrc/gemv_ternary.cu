@@ -37,6 +37,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "bl_common.cuh"
 #include "bl_launch.h"
@@ -1220,6 +1221,58 @@ int cta_ranges(GParams& P, int G, const double* pro) {
     return fill(hi, true);
 }
 
+// cta_ranges for a call whose shapes match a recent call's: the split
+// depends only on G, the problems' row-group counts, steps per row group,
+// prologue costs and which neighbours share an input, so it is looked up
+// (the bisection costs several microseconds of host time per call).
+int cta_ranges_cached(GParams& P, int G, const double* pro) {
+    struct Key {
+        int G, count, fused;
+        uint64_t same;  // bit p: problem p has the input of problem p-1
+        int32_t rgn[kMaxGroup], S[kMaxGroup];
+        double pro[kMaxGroup];
+    };
+    struct Entry {
+        Key key;
+        int grid;
+        int32_t begin[kMaxCta + 1];
+    };
+    constexpr int kEntries = 8;
+    static std::mutex mu;
+    static Entry cache[kEntries];
+    static int used = 0, next = 0;
+    Key k;
+    std::memset(&k, 0, sizeof(k));
+    k.G = G;
+    k.count = P.count;
+    k.fused = pro ? 1 : 0;
+    for (int p = 0; p < P.count; ++p) {
+        k.rgn[p] = P.p[p].rgn;
+        k.S[p] = P.p[p].S;
+        k.pro[p] = pro ? pro[p] : 0.0;
+        if (p > 0 && P.p[p].x == P.p[p - 1].x && P.p[p].x2 == P.p[p - 1].x2 && P.p[p].K == P.p[p - 1].K &&
+            P.p[p].M == P.p[p - 1].M)
+            k.same |= (uint64_t)1 << p;
+    }
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int e = 0; e < used; ++e)
+            if (std::memcmp(&cache[e].key, &k, sizeof(Key)) == 0) {
+                std::memcpy(P.cta_begin, cache[e].begin, sizeof(int32_t) * (cache[e].grid + 1));
+                return cache[e].grid;
+            }
+    }
+    const int grid = cta_ranges(P, G, pro);
+    std::lock_guard<std::mutex> lock(mu);
+    Entry& e = cache[next];
+    next = (next + 1) % kEntries;
+    if (used < kEntries) ++used;
+    e.key = k;
+    e.grid = grid;
+    std::memcpy(e.begin, P.cta_begin, sizeof(int32_t) * (grid + 1));
+    return grid;
+}
+
 // Launches gemv_stream_kernel<MT, W, MINB, RG, CPL, D, fused>; with `fused` (one entry per
 // problem) the kernel quantises x itself, if every CTA's range meets at most
 // two problems, the slots fit shared memory and the CTAs' input reads stay
@@ -1271,7 +1324,7 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
         double pro[kMaxGroup];
         for (int i = 0; i < count; ++i)  // a rotation about doubles the prologue
             pro[i] = prologue_cost(W, CPL, P.p[i].K) * std::min<int>(P.p[i].M, MT) * (P.had ? 2 : 1);
-        grid = cta_ranges(P, G, pro);
+        grid = cta_ranges_cached(P, G, pro);
         // Every CTA reads its problems' whole input rows before its main loop;
         // that pays off only while those reads are small next to the weights.
         auto input_bytes = [&](const GProblem& q) {
@@ -1293,7 +1346,7 @@ cudaError_t launch_stream_cfg(const bitlinear_forward_problem* problems, int cou
         }
         smem += (size_t)kMaxSlots * MT * slot_row;
     } else {
-        grid = cta_ranges(P, G, nullptr);
+        grid = cta_ranges_cached(P, G, nullptr);
     }
     if (smem > smem_cap) return cudaErrorInvalidConfiguration;  // a shape that does not fit (not built)
     const void* kernel = fused ? reinterpret_cast<const void*>(gemv_stream_kernel<MT, W, MINB, RG, CPL, D, 1>)
