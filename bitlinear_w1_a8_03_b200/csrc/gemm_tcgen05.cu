@@ -7,23 +7,26 @@
 // GEMM-shaped batched case) and the dequantisation y = fp32(acc)·α·β/127 +
 // bias ("1.58-bit 大模型极限量化实战", chenxutan.com/d/5049.html §2.4–§2.5, §4.2).
 //
-// Persistent kernel, one CTA per SM.  A tile is 128 weight rows (the MMA's M
-// side) × NT tokens (its N side); K runs in blocks of 128.  Tiles are dealt
-// round-robin to the CTAs.  Warp roles (11 warps):
+// Persistent kernel, one CTA per SM.  A tile is 256 weight rows (two MMAs of
+// M = 128 that share each x̃ tile, which halves the x̃ bytes per MAC) × NT
+// tokens (the MMA's N side); K runs in blocks of 128.  Tiles are dealt
+// round-robin to the CTAs.  Warp roles (15 warps):
 //   warp 0      one thread loads x̃ tiles [NT tokens][128 B] by TMA (128-byte
 //               swizzle) into ring B;
-//   warp 10     one thread loads packed-code tiles [128 rows][32 B] by TMA
+//   warp 10     one thread loads packed-code tiles [256 rows][32 B] by TMA
 //               into ring W, running ahead of the tensor cores;
-//   warps 2-5   expand the 2-bit codes of one row each (one row per thread)
+//   warps 2-5   expand the 2-bit codes of two rows each (rows t and 128 + t)
 //               from ring W into signed bytes {-1, 0, +1} in ring A, laid out
 //               K-major with the 128-byte swizzle the MMA descriptors expect;
-//   warp 1      owns the tensor memory (two NT-column int32 accumulators) and
-//               one thread issues tcgen05.mma.kind::i8 (4 per K block) and the
-//               commits that free ring slots / publish an accumulator;
-//   warps 6-9   epilogue: tcgen05.ld of a row's accumulators, scale by the
-//               token's α·β/127, add bias, store (consecutive threads write
-//               consecutive rows); overlaps the next tile's MMAs because the
-//               accumulator is double-buffered.
+//   warp 1      owns the tensor memory (the accumulators: two per tile, twice
+//               over when they fit) and one thread issues
+//               tcgen05.mma.kind::i8 (8 per K block) and the commits that free
+//               ring slots / publish an accumulator;
+//   warps 6-9,  epilogue: tcgen05.ld of a row's accumulators, scale by the
+//   11-14       token's α·β/127, add bias, store (consecutive threads write
+//               consecutive rows); the two groups take half of the token
+//               columns each.
+// For at most 64 tokens gemm_tm_kernel below is used instead.
 // Every wait is bounded; on expiry the kernel records BL_ERR_TIMEOUT, the
 // other roles stop at their next wait, copies and MMAs in flight drain
 // (bounded) and the tensor memory is freed.
@@ -49,39 +52,53 @@ constexpr int kWarps = 11;
 constexpr int kThreads = kWarps * 32;
 constexpr int kWarpTmaX = 0, kWarpMma = 1, kWarpExp0 = 2, kWarpEpi0 = 6, kWarpTmaW = 10;
 constexpr int kExpWarps = 4, kEpiWarps = 4;
+// the many-token kernel has a second group of four epilogue warps (11-14) that
+// drains the other half of each accumulator's columns
+constexpr int kWarpsTC = 15;
+constexpr int kThreadsTC = kWarpsTC * 32;
+constexpr int kEpiWarpsTC = 8;
 constexpr size_t kSmemLimit = 232448;  // opt-in dynamic shared memory per block on sm_100
 
 // Ring depths (expanded codes A, x̃ tiles B, packed codes W) for the two
 // large tile widths; build-time knobs, the shared-memory budget is checked below.
 #ifndef BL_GEMM_SA_256
-#define BL_GEMM_SA_256 4
+#define BL_GEMM_SA_256 3
 #endif
 #ifndef BL_GEMM_SB_256
-#define BL_GEMM_SB_256 4
+#define BL_GEMM_SB_256 3
 #endif
 #ifndef BL_GEMM_SW_256
-#define BL_GEMM_SW_256 4
+#define BL_GEMM_SW_256 3
 #endif
 #ifndef BL_GEMM_SA_128
-#define BL_GEMM_SA_128 5
+#define BL_GEMM_SA_128 4
 #endif
 #ifndef BL_GEMM_SB_128
-#define BL_GEMM_SB_128 5
+#define BL_GEMM_SB_128 4
 #endif
 #ifndef BL_GEMM_SW_128
-#define BL_GEMM_SW_128 8
+#define BL_GEMM_SW_128 4
 #endif
+
+// A tile is kHalves × 128 weight rows: two MMAs of M = 128 per K step share
+// each x̃ (B) tile, which halves the x̃ bytes every MAC needs.
+constexpr int kHalves = 2;
+constexpr int kTileRows = kHalves * kRowsTile;
 
 template <int NT>
 struct Cfg {
-    static constexpr int kABytes = kRowsTile * kKB;  // 16 KiB of expanded codes
-    static constexpr int kBBytes = NT * kKB;         // NT × 128 B of x̃
-    static constexpr int kWBytes = kRowsTile * kWB;  // 4 KiB of packed codes
-    static constexpr int kSA = NT >= 256 ? BL_GEMM_SA_256 : (NT >= 128 ? BL_GEMM_SA_128 : 4);
-    static constexpr int kSW = NT >= 256 ? BL_GEMM_SW_256 : (NT >= 128 ? BL_GEMM_SW_128 : 16);
-    static constexpr int kSB = NT >= 256 ? BL_GEMM_SB_256 : (NT >= 128 ? BL_GEMM_SB_128 : (NT >= 64 ? 10 : 12));
+    static constexpr int kAHalf = kRowsTile * kKB;     // 16 KiB of expanded codes per 128 rows
+    static constexpr int kABytes = kHalves * kAHalf;    // the tile's rows
+    static constexpr int kBBytes = NT * kKB;            // NT × 128 B of x̃
+    static constexpr int kWBytes = kTileRows * kWB;     // packed codes of the tile's rows
+    static constexpr int kSA = NT >= 256 ? BL_GEMM_SA_256 : BL_GEMM_SA_128;
+    static constexpr int kSW = NT >= 256 ? BL_GEMM_SW_256 : BL_GEMM_SW_128;
+    static constexpr int kSB = NT >= 256 ? BL_GEMM_SB_256 : BL_GEMM_SB_128;
     static constexpr int kBars = 2 * (kSA + kSB + kSW) + 5;
-    static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;  // two accumulators
+    // accumulators: kHalves × NT columns each; two of them when they fit
+    static constexpr int kAccBufs = 2 * kHalves * NT <= 512 ? 2 : 1;
+    static constexpr int kTmemCols = 512;
+    static_assert(kAccBufs * kHalves * NT <= kTmemCols, "tensor memory budget");
     static constexpr size_t kRingBytes =
         (size_t)kSA * kABytes + (size_t)kSB * kBBytes + (size_t)kSW * kWBytes;
     static constexpr size_t kSmem = 1024 + kRingBytes + kBars * 8 + 16;
@@ -227,7 +244,7 @@ __device__ void tma_producer(uint8_t* ring, uint32_t slot_bytes, uint64_t* full,
                              const GemmParams& P, volatile int* abort_flag, Coord coord) {
     int it = 0;
     for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
-        const TileRef tr = locate<NT>(P, tile);
+        const TileRef tr = locate<NT, kTileRows>(P, tile);
         for (int kb = 0; kb < tr.kblocks; ++kb, ++it) {
             const int s = it % S;
             if (it >= S && !wait_or_abort(smem_addr(&empty[s]), ((it / S) - 1) & 1, abort_flag)) goto drain;
@@ -243,7 +260,7 @@ drain:
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(kThreadsTC, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
     using C = Cfg<NT>;
     constexpr int SA = C::kSA, SB = C::kSB, SW = C::kSW;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -264,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     uint64_t* drain = accEmpty + 2;    // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    constexpr int AB = C::kAccBufs;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -284,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_addr(&accFull[b]), 1);
-            mbar_init(smem_addr(&accEmpty[b]), kEpiWarps);
+            mbar_init(smem_addr(&accEmpty[b]), kEpiWarpsTC);
         }
         mbar_init(smem_addr(drain), 1);
         *abort_flag = 0;
@@ -326,11 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             constexpr uint32_t idesc = instr_desc_i8<NT>();
             int it = 0, j = 0;
             for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
-                const int kblocks = locate<NT>(P, tile).kblocks;
-                const int b = j & 1;
-                if (j >= 2 && !wait_or_abort(smem_addr(&accEmpty[b]), ((j >> 1) - 1) & 1, abort_flag)) break;
+                const int kblocks = locate<NT, kTileRows>(P, tile).kblocks;
+                const int b = j % AB;
+                if (j >= AB && !wait_or_abort(smem_addr(&accEmpty[b]), ((j / AB) - 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t d = tmem_d + (uint32_t)(b * NT);
+                const uint32_t d = tmem_d + (uint32_t)(b * kHalves * NT);  // half h at + h·NT
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int sa = it % SA, sb = it % SB;
@@ -342,8 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     const uint32_t b_addr = smem_addr(ringB + (size_t)sb * C::kBBytes);
 #pragma unroll
                     for (int k = 0; k < kKB / 32; ++k)
-                        mma_i8(d, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k), idesc,
-                               (kb > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int h = 0; h < kHalves; ++h)
+                            mma_i8(d + (uint32_t)(h * NT), smem_desc_sw128(a_addr + h * C::kAHalf + 32 * k),
+                                   smem_desc_sw128(b_addr + 32 * k), idesc, (kb > 0 || k > 0) ? 1u : 0u);
                     mma_commit(smem_addr(&emptyA[sa]));
                     if constexpr (!kOneRelease) mma_commit(smem_addr(&emptyB[sb]));
                 }
@@ -357,32 +377,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else if (warp < kWarpEpi0) {
         // ---- expand the codes of tile row t from ring W into ring A
         const int t = 32 * (warp & 3) + lane;
-        const uint32_t w_off = (uint32_t)t * kWB;
         const uint32_t a_row = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128);
         int it = 0;
         for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
-            const int kblocks = locate<NT>(P, tile).kblocks;
+            const int kblocks = locate<NT, kTileRows>(P, tile).kblocks;
             bool ok = true;
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 const int sw = it % SW, sa = it % SA;
                 if (!(ok = wait_or_abort(smem_addr(&fullW[sw]), (it / SW) & 1, abort_flag))) break;
-                const uint32_t wsrc = smem_addr(ringW + (size_t)sw * C::kWBytes) + w_off;
-                const uint4 pk0 = lds128(wsrc);
-                const uint4 pk1 = lds128(wsrc + 16);
-                uint4 out[8];
+                // rows t (first half) and 128 + t (second half) of the tile
+                uint4 pk[kHalves][2];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    // weights 16q .. 16q+15 of the block: fields 0..3 of packed word q
-                    const uint32_t w = word_of(q < 4 ? pk0 : pk1, q & 3);
-                    out[q] = make_uint4(field_s8(w, 0), field_s8(w, 1), field_s8(w, 2), field_s8(w, 3));
+                for (int h = 0; h < kHalves; ++h) {
+                    const uint32_t wsrc =
+                        smem_addr(ringW + (size_t)sw * C::kWBytes) + (uint32_t)(h * kRowsTile + t) * kWB;
+                    pk[h][0] = lds128(wsrc);
+                    pk[h][1] = lds128(wsrc + 16);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive1(smem_addr(&emptyW[sw]));  // codes are in registers
                 if (it >= SA && !(ok = wait_or_abort(smem_addr(&emptyA[sa]), ((it / SA) - 1) & 1, abort_flag)))
                     break;
-                uint8_t* rowp = ringA + (size_t)sa * C::kABytes + a_row;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(rowp + ((q ^ (t & 7)) << 4)) = out[q];
+                for (int h = 0; h < kHalves; ++h) {
+                    uint8_t* rowp = ringA + (size_t)sa * C::kABytes + h * C::kAHalf + a_row;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        // weights 16q .. 16q+15 of the block: fields 0..3 of packed word q
+                        const uint32_t w = word_of(q < 4 ? pk[h][0] : pk[h][1], q & 3);
+                        *reinterpret_cast<uint4*>(rowp + ((q ^ (t & 7)) << 4)) =
+                            make_uint4(field_s8(w, 0), field_s8(w, 1), field_s8(w, 2), field_s8(w, 3));
+                    }
+                }
                 fence_proxy_async_smem();  // generic writes -> tensor-core reads
                 __syncwarp();
                 if (lane == 0) mbar_arrive1(smem_addr(&fullA[sa]));
@@ -397,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         int j = 0;
         for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
-            const TileRef tr = locate<NT>(P, tile);
+            const TileRef tr = locate<NT, kTileRows>(P, tile);
             // this tile's problem, copied out of the parameter block once
             // (dynamically indexed parameter reads inside the store loop are slow)
             const int M = P.p[tr.p].M, N = P.p[tr.p].N;
@@ -406,32 +432,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             float* y = P.p[tr.p].y;
             int32_t* acc_out = P.p[tr.p].acc_out;
             const float alpha = *P.p[tr.p].alpha;
-            const int b = j & 1;
+            const int b = j % AB;
             const int m0 = tr.m0;
-            const int row = tr.n0 + t;
-            const bool row_ok = row < N;
-            const float bias = (row_ok && bias_p) ? bias_p[row] : 0.0f;
-            if (!wait_or_abort(smem_addr(&accFull[b]), (j >> 1) & 1, abort_flag)) break;
+            if (!wait_or_abort(smem_addr(&accFull[b]), (j / AB) & 1, abort_flag)) break;
             tc_fence_after();
+            // warps 6-9 take the first half of the token columns, 11-14 the second
+            const int cbeg = warp > kWarpTmaW ? NT / 2 : 0;
 #pragma unroll 1
-            for (int c0 = 0; c0 < NT; c0 += 32) {
-                // lane l holds the scale of token m0 + c0 + l; shuffled to the writers below
-                const int my_tok = m0 + c0 + lane;
-                const float my_scale = my_tok < M ? dequant_scale(alpha, beta_p[my_tok]) : 0.0f;
+            for (int hh = 0; hh < kHalves; ++hh) {
+                const int row = tr.n0 + hh * kRowsTile + t;
+                const bool row_ok = row < N;
+                const float bias = (row_ok && bias_p) ? bias_p[row] : 0.0f;
+                const uint32_t col0 = (uint32_t)((b * kHalves + hh) * NT);
+#pragma unroll 1
+                for (int c0 = cbeg; c0 < cbeg + NT / 2; c0 += 32) {
+                    // lane l holds the scale of token m0 + c0 + l; shuffled to the writers below
+                    const int my_tok = m0 + c0 + lane;
+                    const float my_scale = my_tok < M ? dequant_scale(alpha, beta_p[my_tok]) : 0.0f;
 #pragma unroll
-                for (int h = 0; h < 2 && c0 + 16 * h < NT; ++h) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem_d + lane_base + (uint32_t)(b * NT + c0 + 16 * h), r);
+                    for (int h = 0; h < 2 && c0 + 16 * h < NT; ++h) {
+                        uint32_t r[16];
+                        tmem_ld16(tmem_d + lane_base + col0 + (uint32_t)(c0 + 16 * h), r);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float sc = __shfl_sync(0xffffffffu, my_scale, 16 * h + i);
-                        const int tok = m0 + c0 + 16 * h + i;
-                        if (row_ok && tok < M) {
-                            const int acc = (int)r[i];
-                            float out = __fmul_rn((float)acc, sc);
-                            if (bias_p) out = __fadd_rn(out, bias);
-                            y[(int64_t)tok * N + row] = out;
-                            if (acc_out) acc_out[(int64_t)tok * N + row] = acc;
+                        for (int i = 0; i < 16; ++i) {
+                            const float sc = __shfl_sync(0xffffffffu, my_scale, 16 * h + i);
+                            const int tok = m0 + c0 + 16 * h + i;
+                            if (row_ok && tok < M) {
+                                const int acc = (int)r[i];
+                                float out = __fmul_rn((float)acc, sc);
+                                if (bias_p) out = __fadd_rn(out, bias);
+                                y[(int64_t)tok * N + row] = out;
+                                if (acc_out) acc_out[(int64_t)tok * N + row] = acc;
+                            }
                         }
                     }
                 }
@@ -977,7 +1009,7 @@ cudaError_t cluster_pairs(const void* kernel, int smem, int* out) {
 // tiles of 127 rows, stages of 512, codes expanded in tensor memory).
 template <int NT, bool TMEM_A>
 cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cudaStream_t stream, bool pdl) {
-    constexpr int kRows = TMEM_A ? tm::kRows : kRowsTile;
+    constexpr int kRows = TMEM_A ? tm::kRows : kTileRows;
     constexpr int kStageK = TMEM_A ? tm::kKS : kKB;
     size_t kSmem;
     const void* kernel;
@@ -1012,7 +1044,7 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
         if (TMEM_A)
             err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, tm::kWS, tm::kRows, CU_TENSOR_MAP_SWIZZLE_128B);
         else
-            err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, kWB, kRowsTile, CU_TENSOR_MAP_SWIZZLE_NONE);
+            err = encode_u8(&P.wmap[i], pr.W_packed, row_bytes, pr.N, kWB, kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (err != cudaSuccess) return err;
         GemmProblem& q = P.p[i];
         q.alpha = pr.alpha;
@@ -1035,7 +1067,7 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)(tiles < dev.sm_count ? tiles : dev.sm_count));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(TMEM_A ? kThreads : kThreadsTC);
     cfg.dynamicSmemBytes = kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
