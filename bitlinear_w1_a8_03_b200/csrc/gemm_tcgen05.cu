@@ -34,6 +34,8 @@
 
 #include <algorithm>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "bl_common.cuh"
 #include "bl_launch.h"
@@ -121,6 +123,9 @@ struct GemmProblem {
 
 // Several independent problems in one persistent launch: tiles are numbered
 // problem after problem and dealt round-robin to the CTAs.
+constexpr int kMaxListCtas = 256;
+constexpr int kMaxListTiles = 2048;
+
 struct GemmParams {
     CUtensorMap xmap[kMaxGroup];  // x̃ [M][K] of each problem
     CUtensorMap wmap[kMaxGroup];  // packed codes [N][row bytes] of each problem
@@ -128,7 +133,24 @@ struct GemmParams {
     int count;
     int tiles;
     int cs;  // few-token kernel: CTAs per cluster, each taking 1/cs of every tile's K stages
+    // many-token kernel: tiles of CTA c are tile_list[cta_start[c] .. cta_start[c+1])
+    // (a longest-first greedy balance of K blocks), else round-robin
+    int use_list;
+    uint16_t cta_start[kMaxListCtas + 1];
+    uint16_t tile_list[kMaxListTiles];
 };
+
+static_assert(sizeof(GemmParams) <= 32764, "kernel parameter block");
+
+// The n-th tile of this CTA (or -1): from the host's list, else round-robin.
+__device__ __forceinline__ int nth_tile(const GemmParams& P, int n) {
+    if (P.use_list) {
+        const int i = P.cta_start[blockIdx.x] + n;
+        return i < P.cta_start[blockIdx.x + 1] ? P.tile_list[i] : -1;
+    }
+    const int64_t t = (int64_t)blockIdx.x + (int64_t)n * gridDim.x;
+    return t < P.tiles ? (int)t : -1;
+}
 
 struct TileRef {
     int p, m0, n0, kblocks;
@@ -243,7 +265,7 @@ template <int NT, int S, typename Coord>
 __device__ void tma_producer(uint8_t* ring, uint32_t slot_bytes, uint64_t* full, uint64_t* empty,
                              const GemmParams& P, volatile int* abort_flag, Coord coord) {
     int it = 0;
-    for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+    for (int n = 0, tile; (tile = nth_tile(P, n)) >= 0; ++n) {
         const TileRef tr = locate<NT, kTileRows>(P, tile);
         for (int kb = 0; kb < tr.kblocks; ++kb, ++it) {
             const int s = it % S;
@@ -343,7 +365,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) gemm_tc_kernel(const __grid_con
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc_i8<NT>();
             int it = 0, j = 0;
-            for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+            for (int tile; (tile = nth_tile(P, j)) >= 0; ++j) {
                 const int kblocks = locate<NT, kTileRows>(P, tile).kblocks;
                 const int b = j % AB;
                 if (j >= AB && !wait_or_abort(smem_addr(&accEmpty[b]), ((j / AB) - 1) & 1, abort_flag)) break;
@@ -379,7 +401,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) gemm_tc_kernel(const __grid_con
         const int t = 32 * (warp & 3) + lane;
         const uint32_t a_row = (uint32_t)((t >> 3) * 1024 + (t & 7) * 128);
         int it = 0;
-        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x) {
+        for (int n = 0, tile; (tile = nth_tile(P, n)) >= 0; ++n) {
             const int kblocks = locate<NT, kTileRows>(P, tile).kblocks;
             bool ok = true;
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
@@ -422,7 +444,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) gemm_tc_kernel(const __grid_con
         const int t = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         int j = 0;
-        for (int tile = blockIdx.x; tile < P.tiles; tile += gridDim.x, ++j) {
+        for (int tile; (tile = nth_tile(P, j)) >= 0; ++j) {
             const TileRef tr = locate<NT, kTileRows>(P, tile);
             // this tile's problem, copied out of the parameter block once
             // (dynamically indexed parameter reads inside the store loop are slow)
@@ -1061,6 +1083,41 @@ cudaError_t launch_nt(const bitlinear_forward_problem* problems, int count, cuda
     }
     P.tiles = tiles;
     P.cs = 1;
+    P.use_list = 0;
+    if constexpr (!TMEM_A) {
+        // Longest-first greedy: each tile (numbered longest K first) goes to
+        // the CTA with the fewest K blocks so far, so the CTAs end together
+        // even when a few long tiles meet many short ones.
+        const int G = tiles < dev.sm_count ? tiles : dev.sm_count;
+        if (tiles <= kMaxListTiles && G <= kMaxListCtas) {
+            static thread_local std::vector<std::pair<int64_t, int>> heap;
+            static thread_local std::vector<int> owner;
+            heap.clear();
+            owner.assign((size_t)tiles, 0);
+            for (int c = 0; c < G; ++c) heap.emplace_back(0, c);
+            auto later = [](const std::pair<int64_t, int>& a, const std::pair<int64_t, int>& b) {
+                return a.first != b.first ? a.first > b.first : a.second > b.second;
+            };
+            std::make_heap(heap.begin(), heap.end(), later);
+            int p = 0;
+            int count_per[kMaxListCtas] = {};
+            for (int t = 0; t < tiles; ++t) {
+                while (p + 1 < count && t >= P.p[p + 1].tile_begin) ++p;
+                std::pop_heap(heap.begin(), heap.end(), later);
+                auto& top = heap.back();
+                owner[t] = top.second;
+                ++count_per[top.second];
+                top.first += P.p[p].kblocks;
+                std::push_heap(heap.begin(), heap.end(), later);
+            }
+            P.cta_start[0] = 0;
+            for (int c = 0; c < G; ++c) P.cta_start[c + 1] = (uint16_t)(P.cta_start[c] + count_per[c]);
+            int fill[kMaxListCtas];
+            for (int c = 0; c < G; ++c) fill[c] = P.cta_start[c];
+            for (int t = 0; t < tiles; ++t) P.tile_list[fill[owner[t]]++] = (uint16_t)t;
+            P.use_list = 1;
+        }
+    }
 
     // the opt-in is per device: set once on each device that launches the kernel
     err = set_max_dynamic_smem(kernel, (int)kSmem);
