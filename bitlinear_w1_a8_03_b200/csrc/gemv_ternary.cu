@@ -1119,7 +1119,7 @@ struct StreamCfg<1> {
 };
 template <>
 struct StreamCfg<2> {
-    static constexpr int W = 12, MINB = 1, RG = 4, CPL = 1, D = 4;
+    static constexpr int W = 12, MINB = 1, RG = 8, CPL = 1, D = 3;
 };
 template <>
 struct StreamCfg<4> {
