@@ -30,7 +30,10 @@ namespace bl {
 namespace {
 
 constexpr int kRows = 4;     // rows per work item
-constexpr int kWarps = 8;    // warps per CTA
+// warps per CTA: 16 for one token (more loads in flight per SM: one α per
+// 128-block went from 60 to 41 µs on the 7B set), 8 for more tokens, whose
+// larger register sets would spill at 16
+__host__ __device__ constexpr int warps_for(int MT) { return MT == 1 ? 16 : 8; }
 constexpr int kPerSM = 2;    // CTAs per SM in the grid (one resident per SM by registers)
 
 struct ScProblem {
@@ -138,7 +141,8 @@ enum ScaleMode { kTensor = 0, kRow = 1, kBlocks = 2 };
 // MT tokens per pass; MODE: one α (tensor), one per row, several per row
 // (binary64 sums of α_b·acc_b); A4: packed 4-bit activations.
 template <int MT, int MODE, bool A4>
-__global__ void __launch_bounds__(kWarps * 32, 1) gemv_scaled_kernel(const __grid_constant__ ScParams P) {
+__global__ void __launch_bounds__(warps_for(MT) * 32, 1) gemv_scaled_kernel(const __grid_constant__ ScParams P) {
+    constexpr int kWarps = warps_for(MT);
     constexpr int V = kRows * MT;
     constexpr bool BLOCKS = MODE == kBlocks;
     using Acc = typename std::conditional<BLOCKS, double, int>::type;
@@ -295,6 +299,7 @@ cudaError_t launch_scaled_mt(const ScaledProblem* problems, int count, cudaStrea
         items += (int64_t)q.rgn * q.tgn;
     }
     P.total_items = items;
+    constexpr int kWarps = warps_for(MT);
     int64_t grid = (int64_t)dev.sm_count * kPerSM;
     const int64_t need = (items + kWarps - 1) / kWarps;
     if (grid > need) grid = need;
