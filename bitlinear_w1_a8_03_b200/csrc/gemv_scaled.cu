@@ -34,7 +34,7 @@ constexpr int kRows = 4;     // rows per work item
 // 128-block went from 60 to 41 µs on the 7B set), 8 for more tokens, whose
 // larger register sets would spill at 16
 __host__ __device__ constexpr int warps_for(int MT) { return MT == 1 ? 16 : 8; }
-constexpr int kPerSM = 2;    // CTAs per SM in the grid (one resident per SM by registers)
+constexpr int kPerSM = 3;    // CTAs per SM in the grid (one resident per SM by registers; later waves even out the end)
 
 struct ScProblem {
     const int8_t* xq;
