@@ -177,7 +177,8 @@ BITLINEAR_API bitlinear_status bitlinear_quantize_act_grouped(const bitlinear_ac
                                                 bitlinear_dtype dtype, bitlinear_stream_t stream);
 
 /* One problem of a grouped forward; fields as in bitlinear_forward.  Above
- * four tokens all problems of a call share one tensor-core launch. */
+ * four tokens (and at three or four tokens when the call's weights total
+ * 8 MB or more) all problems of a call share one tensor-core launch. */
 typedef struct bitlinear_forward_problem {
     const int8_t* x_q;
     const float* beta;
