@@ -133,6 +133,20 @@ def decode_config(specs) -> dict:
     }
 
 
+def kernels_per_call(fn, stream) -> int:
+    """CUDA kernels one eager call of fn launches, counted by the torch
+    profiler outside any timed region (the library picks launch shapes at
+    run time, e.g. one act-quant launch per CTA size)."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    stream.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        with torch.cuda.stream(stream):
+            fn()
+        stream.synchronize()
+    return sum(1 for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA)
+
+
 # ----------------------------------------------------------------------------- ranks
 def max_over_ranks(values, device, world: int):
     """Element-wise max of per-rank timings (ms) over all ranks; identity at N=1."""
@@ -461,6 +475,7 @@ def run_prefill(args, world, local_rank):
         for _ in range(max(args.warmup, 3)):
             step()
     stream.synchronize()
+    launches_per_step = kernels_per_call(step, stream)
     K = args.steps
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -608,7 +623,7 @@ def run_prefill(args, world, local_rank):
                          "bytes": wq_bytes, "what": "absmean (exact sum) + ternarise + 2-bit pack of the three fp32 "
                                                    "prefill matrices, once per matrix (not on the step path)"},
         "cublas_int8_tops_context": cublas,
-        "gpu_launches": 2 * K,  # grouped act quant + one grouped GEMM per step
+        "gpu_launches": launches_per_step * K,  # act quant (one launch per CTA size) + one grouped GEMM per step
         "clocks": clocks,
     }
 
@@ -1067,6 +1082,7 @@ def run_stack(args, world, local_rank):
             for _ in range(max(args.warmup, 3)):
                 st.run(stream)
         stream.synchronize()
+        stack_launches = kernels_per_call(lambda: st.run(stream), stream)
         K = max(10, args.steps // 4)
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
@@ -1102,7 +1118,7 @@ def run_stack(args, world, local_rank):
             "frac_of_hbm": round(bytes_step / (ms * 1e-3) / 1e9 / float(load_peaks()[0]["hbm_gbs"]), 4),
             "bytes_per_step": bytes_step,
             "steps": K,
-            "gpu_launches_per_step": st.launches(),
+            "gpu_launches_per_step": stack_launches,
             "device_error": err,
             "clocks": clocks,
         }

@@ -266,29 +266,21 @@ cudaError_t launch_quantize_act(const bitlinear_act_problem* problems, int count
     return launch_quantize_act_jobs(jobs, count, dtype, stream, pdl, early_trigger);
 }
 
-cudaError_t launch_quantize_act_jobs(const ActJob* problems, int count, bitlinear_dtype dtype, cudaStream_t stream,
-                                     bool pdl, bool early_trigger) {
+namespace {
+
+// One launch of act_quant_kernel over `count` jobs with `threads` per row.
+cudaError_t launch_act_rows(const ActJob* jobs, int count, bitlinear_dtype dtype, cudaStream_t stream, bool pdl,
+                            bool early_trigger, int threads) {
     ActParams P{};
     P.count = count;
     P.early_trigger = early_trigger ? 1 : 0;
-    int64_t rows = 0, kmax = 0;
+    int64_t rows = 0;
     for (int i = 0; i < count; ++i) {
-        P.p[i] = problems[i];
+        P.p[i] = jobs[i];
         P.row_begin[i] = rows;
-        rows += problems[i].M;
-        kmax = problems[i].K > kmax ? problems[i].K : kmax;
+        rows += jobs[i].M;
     }
     P.row_begin[count] = rows;
-    DeviceInfo dev;
-    cudaError_t err = device_info(&dev);
-    if (err != cudaSuccess) return err;
-    // many rows: kVecPerThread vectors per thread (at least 2 warps); few rows: 512 threads
-    int threads = kMaxThreads;
-    if (rows >= 2 * (int64_t)dev.sm_count) {
-        const int64_t nvec = (kmax * (dtype == BL_BF16 ? 2 : 4) + 15) / 16;
-        const int64_t want = ((nvec + kVecPerThread - 1) / kVecPerThread + 31) / 32 * 32;
-        threads = (int)(want < 64 ? 64 : (want > kMaxThreads ? kMaxThreads : want));
-    }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)rows);
     cfg.blockDim = dim3(threads);
@@ -300,6 +292,43 @@ cudaError_t launch_quantize_act_jobs(const ActJob* problems, int count, bitlinea
     cfg.numAttrs = 1;
     if (dtype == BL_BF16) return cudaLaunchKernelEx(&cfg, act_quant_kernel<uint16_t>, P);
     return cudaLaunchKernelEx(&cfg, act_quant_kernel<float>, P);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_act_jobs(const ActJob* problems, int count, bitlinear_dtype dtype, cudaStream_t stream,
+                                     bool pdl, bool early_trigger) {
+    DeviceInfo dev;
+    cudaError_t err = device_info(&dev);
+    if (err != cudaSuccess) return err;
+    int64_t rows = 0;
+    for (int i = 0; i < count; ++i) rows += problems[i].M;
+    // few rows: 512 threads per row.  Many rows: kVecPerThread vectors per
+    // thread (at least 2 warps), sized for each problem's K; problems that
+    // want different CTA sizes get a launch each (a 4096-wide row in CTAs
+    // sized for an 11008-wide one leaves too few bytes in flight per SM).
+    if (rows < 2 * (int64_t)dev.sm_count) return launch_act_rows(problems, count, dtype, stream, pdl, early_trigger,
+                                                                 kMaxThreads);
+    auto threads_for = [&](int64_t K) {
+        const int64_t nvec = (K * (dtype == BL_BF16 ? 2 : 4) + 15) / 16;
+        const int64_t want = ((nvec + kVecPerThread - 1) / kVecPerThread + 31) / 32 * 32;
+        return (int)(want < 64 ? 64 : (want > kMaxThreads ? kMaxThreads : want));
+    };
+    ActJob group[kMaxGroup];
+    bool done[kMaxGroup] = {};
+    for (int i = 0; i < count; ++i) {
+        if (done[i]) continue;
+        const int t = threads_for(problems[i].K);
+        int n = 0;
+        for (int j = i; j < count; ++j)
+            if (!done[j] && threads_for(problems[j].K) == t) {
+                group[n++] = problems[j];
+                done[j] = true;
+            }
+        err = launch_act_rows(group, n, dtype, stream, pdl, early_trigger, t);
+        if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace bl
