@@ -123,3 +123,29 @@ def test_gemm_grouped_problems(M):
         assert np.array_equal(np_(pr["acc_out"]), acc_r)
         err = np.abs(np_(pr["y"]).astype(np.float64) - y_r)
         assert np.all(err <= 1e-5 * np.abs(y_r) + 1e-37)
+
+
+def test_gemm_more_tiles_than_the_host_deal_lists():
+    """More than 2048 tiles (here 32 token tiles × 66 row tiles): the kernel
+    deals them round-robin instead of from the host's per-CTA lists.  Checked
+    on every token of 96 sampled rows (and the last row)."""
+    M, K, N = 8192, 64, 256 * 65 + 7
+    W = synth.weights(910, N, K, 0.02)
+    x = synth.activations(911, M, K, outliers=True)
+    Wd, Wo = as_input(W, "f32")
+    packed, alpha = bl.bitlinear_quantize_weights(Wd)
+    _, a_ref, codes = oracle.quantize_weights(Wo)
+    xd, xo = as_input(x, "bf16")
+    xq, beta = bl.bitlinear_quantize_act(xd)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    y = bl.bitlinear_forward(xq, beta, packed, alpha, N, acc_out=acc)
+    torch.cuda.synchronize()
+    assert bl.bitlinear_device_error() == 0
+    xq_r, beta_r = oracle.quantize_act(xo)
+    assert np.array_equal(np_(xq), xq_r)
+    rows = np.unique(np.concatenate([np.random.default_rng(912).choice(N, 96, replace=False), [N - 1]]))
+    acc_r = oracle.ternary_matmul(xq_r, codes[rows], threads=8)
+    y_r = oracle.dequant(acc_r, beta_r, a_ref).astype(np.float64)
+    assert np.array_equal(acc[:, torch.from_numpy(rows).cuda()].cpu().numpy(), acc_r)
+    err = np.abs(y[:, torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64) - y_r)
+    assert np.all(err <= 1e-5 * np.abs(y_r) + 1e-37)
