@@ -655,6 +655,6 @@ const char* bitlinear_status_string(bitlinear_status status) {
     return "unknown status";
 }
 
-int bitlinear_version(void) { return 101; }
+int bitlinear_version(void) { return 102; }
 
 }  // extern "C"

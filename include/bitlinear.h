@@ -483,7 +483,7 @@ BITLINEAR_API bitlinear_status bitlinear_selftest_timeout(uint32_t polls, bitlin
 /* Static description of a status code. */
 BITLINEAR_API const char* bitlinear_status_string(bitlinear_status status);
 
-/* ABI version: 100·major + minor. */
+/* ABI version: 100·major + minor (1.02 added bitlinear_linear_grouped_host). */
 BITLINEAR_API int bitlinear_version(void);
 
 #ifdef __cplusplus

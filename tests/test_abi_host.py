@@ -34,7 +34,7 @@ def test_header_symbols_exported(L):
     assert {"bitlinear_quantize_weights", "bitlinear_quantize_act", "bitlinear_forward"} <= set(names)
     for n in names:
         assert hasattr(L, n), f"{n} declared in bitlinear.h but not exported"
-    assert L.bitlinear_version() == 101
+    assert L.bitlinear_version() == 102  # 1.02: bitlinear_linear_grouped_host added
 
 
 def test_struct_layout_matches_header():
