@@ -25,7 +25,11 @@ constexpr int kThreads = 256;
 constexpr int kLimbs = 10;          // 320 bits: 2^-149 .. 2^128 times up to 2^40 terms
 constexpr int kMaxPartials = 1024;  // partial sums written to the workspace
 
-// Adds |w|·2^149 into the limb accumulator.
+// Adds |w|·2^149 into the limb accumulator.  The significand lands in limbs
+// li and li + 1 (li = p / 32 ≤ 7 for every finite w); a switch on li keeps
+// the accumulator in registers and costs a few instructions per element where
+// a select over all ten limbs cost about forty (the weights of a matrix have
+// few distinct li, so a warp rarely diverges on it).
 __device__ __forceinline__ void add_abs(uint64_t (&acc)[kLimbs], float w) {
     const uint32_t bits = __float_as_uint(w) & 0x7FFFFFFFu;
     const uint32_t e = bits >> 23;
@@ -35,10 +39,23 @@ __device__ __forceinline__ void add_abs(uint64_t (&acc)[kLimbs], float w) {
     const uint32_t li = p >> 5;
     const uint64_t v = (uint64_t)sig << (p & 31u);
     const uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
-#pragma unroll
-    for (int j = 0; j < kLimbs; ++j) {
-        acc[j] += (j == (int)li) ? lo : 0u;
-        acc[j] += (j == (int)li + 1) ? hi : 0u;
+    switch (li) {
+#define BL_ADD_AT(L)       \
+    case L:                \
+        acc[L] += lo;      \
+        acc[L + 1] += hi;  \
+        break;
+        BL_ADD_AT(0)
+        BL_ADD_AT(1)
+        BL_ADD_AT(2)
+        BL_ADD_AT(3)
+        BL_ADD_AT(4)
+        BL_ADD_AT(5)
+        BL_ADD_AT(6)
+        BL_ADD_AT(7)
+#undef BL_ADD_AT
+        default:  // not reached: p <= 254, so li <= 7
+            break;
     }
 }
 
