@@ -168,3 +168,24 @@ def test_fast_quantisation_non_finite_and_huge_rows():
                 want = _exact_code(x, beta, scale)
             want = np.where(np.isnan(want), -scale, want)  # the kernels' clip maps NaN to -scale
             assert np.array_equal(got, want)
+
+
+def test_exact_sum_limb_positions_cover_every_exponent():
+    """The weight quantiser's exact Σ|W| adds |w|·2^149 (a 24-bit significand
+    at bit position p = max(e, 1) - 1) into limbs p // 32 and p // 32 + 1 of a
+    ten-limb (320-bit) integer, dispatching on p // 32 with cases 0 … 7.
+    Every exponent field, subnormals and e = 255 included, lands in a case
+    that exists, and the value's top bit stays inside the two limbs it
+    touches (so no bit of any |w| is dropped)."""
+    seen = set()
+    for e in range(256):
+        p = max(e, 1) - 1
+        li = p >> 5
+        assert 0 <= li <= 7 and li + 1 < 10
+        top = (p & 31) + 23  # highest significand bit within the 64-bit two-limb window
+        assert top < 64
+        seen.add(li)
+    assert seen == set(range(8))
+    # a normal w = 1.0 (e = 127): 2^149 = 2^(32·4 + 21), i.e. limb 4, bit 21
+    p = 127 - 1
+    assert (p >> 5, (p & 31) + 23) == (3, 53)  # significand bit 23 of limb pair (3, 4) = bit 21 of limb 4
